@@ -1,0 +1,419 @@
+"""Pins of the CPU oracle to facts outside itself (CPU only, no GPU).
+
+Each check ties a part of the oracle to something it does not compute
+itself: a library routine (numpy's IEEE fp16 conversion, scipy's Sylvester
+Hadamard matrix, scipy's softmax, math.fsum), a closed form evaluated in
+fp64, published known-answer values, hand-worked layouts, or an invariant the
+pages state.  A plausible slip in the oracle (a dropped term, a wrong sign or
+index, a transposed operand, the L_{-1} "norm" the nsep+pchan post warns
+about) fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import scipy.special
+
+import oracle
+from kv_cache_bit_b200 import synth
+from tests.modes import f16bits, oracle_cfg
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+T = oracle.T
+
+
+def ulp16(v):
+    """fp16 spacing at |v| (subnormal spacing 2^-24 at the bottom)."""
+    a = np.maximum(np.abs(np.asarray(v, np.float64)), 2.0 ** -14)
+    return 2.0 ** (np.floor(np.log2(a)) - 10)
+
+
+def f16val(bits):
+    return np.asarray(bits, np.uint16).view(np.float16).astype(np.float64)
+
+
+def near_f16(stored_bits, exact, rel=1e-5):
+    """stored fp16 == exact rounded to fp16, allowing either neighbour only
+    when `exact` sits within `rel` of a rounding midpoint."""
+    s = f16val(stored_bits)
+    return np.abs(s - exact) <= 0.5 * ulp16(exact) + rel * np.abs(exact) + 2.0 ** -25
+
+
+# ------------------------------------------------------------- fp16 format
+
+def test_f32_to_f16_matches_numpy():
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([
+        rng.standard_normal(200000).astype(np.float32) * np.float32(10.0) ** rng.integers(-9, 6, 200000),
+        np.array([0.0, -0.0, 65504, 65519.99, 65520, 1e9, -1e9, np.inf, -np.inf,
+                  2 ** -24, 2 ** -25, 3 * 2 ** -26, 2 ** -14, 2 ** -14 - 2 ** -25,
+                  1 + 2 ** -11, 1 + 3 * 2 ** -11, 2049, 2051, 0.1, 1 / 3], np.float32),
+    ]).astype(np.float32)
+    ours = oracle.f32_to_f16_bits(vals)
+    ref = vals.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_f16_to_f32_all_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.f16_bits_to_f32(bits)
+    ref = bits.view(np.float16).astype(np.float32)
+    fin = np.isfinite(ref)
+    assert np.array_equal(ours[fin], ref[fin])
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+
+
+# ------------------------------------------------------------- signs / RNG
+
+def test_splitmix64_known_answers():
+    want = [int(l, 16) for l in open(os.path.join(GOLD, "splitmix64_seed0.txt"))
+            if l.strip() and not l.startswith("#")]
+    assert oracle.splitmix64(0, len(want)) == want
+
+
+def test_signs_are_pm1_and_seeded():
+    s = oracle.make_signs(12345, 128)
+    assert set(np.unique(s).tolist()) <= {-1, 1}
+    assert 30 < int((s < 0).sum()) < 98
+    assert np.array_equal(s, oracle.make_signs(12345, 128))
+    assert not np.array_equal(s, oracle.make_signs(12346, 128))
+    # bit 63 of the SplitMix64 stream decides the sign
+    top = [(z >> 63) & 1 for z in oracle.splitmix64(0, 3)]
+    assert [1 if t else 0 for t in top] == [int(v < 0) for v in oracle.make_signs(0, 3)]
+
+
+# ------------------------------------------------------------- Hadamard
+
+@pytest.mark.parametrize("d", [8, 64, 128])
+def test_fwht_columns_equal_sylvester_matrix(d):
+    H = scipy.linalg.hadamard(d).astype(np.float32)
+    cols = oracle.fwht(np.eye(d, dtype=np.float32))      # row i = FWHT(e_i)
+    assert np.array_equal(cols, H.T)
+    assert np.array_equal(H @ H.T, d * np.eye(d, dtype=np.float32))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_rotation_orthonormal(d):
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((50, d)).astype(np.float32) * 5
+    s = oracle.make_signs(7, d).astype(np.float32)
+    H = scipy.linalg.hadamard(d).astype(np.float64)
+    y = oracle.fwht(x * s) / np.float32(np.sqrt(d))
+    ref = (x.astype(np.float64) * s) @ H.T / np.sqrt(d)
+    assert np.max(np.abs(y - ref)) <= 1e-6 * np.max(np.linalg.norm(x, axis=1))
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-6)
+    back = (oracle.fwht(y) / np.float32(np.sqrt(d))) * s
+    assert np.max(np.abs(back - x)) <= 1e-5
+
+
+# ------------------------------------------------------------- pairwise sum
+
+def test_pairwise_sum_close_to_exact():
+    rng = np.random.default_rng(3)
+    for n in (1, 2, 4, 128, 1024):
+        v = (rng.standard_normal(n) * 10.0 ** rng.integers(-3, 4, n)).astype(np.float32)
+        exact = math.fsum(v.astype(np.float64))
+        bound = math.ceil(math.log2(max(n, 2))) * 2.0 ** -24 * float(np.abs(v).astype(np.float64).sum())
+        assert abs(float(oracle.pairwise_sum(v)) - exact) <= bound + 1e-30
+    ints = rng.integers(-1000, 1000, 128).astype(np.float32)
+    assert float(oracle.pairwise_sum(ints)) == float(ints.astype(np.int64).sum())
+
+
+# ------------------------------------------------------------- packing
+
+def _gold_pack():
+    for line in open(os.path.join(GOLD, "pack_layout.txt")):
+        if not line.strip() or line.startswith("#"):
+            continue
+        b, qs, hx = (p.strip() for p in line.split("|"))
+        yield int(b), np.array([int(v) for v in qs.split()], np.int8), bytes.fromhex(hx.replace(" ", ""))
+
+
+def test_pack_layout_hand_worked():
+    for bits, q, want in _gold_pack():
+        got = oracle.pack_rows(q[None, :], bits)[0].tobytes()
+        assert got == want, (bits, got.hex(), want.hex())
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
+def test_pack_roundtrip_and_no_zero_code(bits):
+    rng = np.random.default_rng(bits)
+    qm = oracle.qmax(bits)
+    q = rng.integers(-qm, qm + 1, (64, 128)).astype(np.int8)
+    packed = oracle.pack_rows(q, bits)
+    assert packed.shape[1] == oracle.row_bytes(128, bits)
+    back, bad = oracle.unpack_rows(packed, 128, bits)
+    assert bad == 0 and np.array_equal(back, q)
+    zero = np.zeros_like(packed)
+    assert oracle.unpack_rows(zero, 128, bits)[1] == 64 * 128
+
+
+def test_qmax_formula():
+    # alpha = max|X| / (2^(N-1) - 1): INT4 +-7 as in the post, INT3 +-3, INT2 +-1
+    assert [oracle.qmax(b) for b in (2, 3, 4, 8)] == [1, 3, 7, 127]
+
+
+# ------------------------------------------------------------- quantizer
+
+def _data(seed, B=1, H=2, S=256, d=128, outl=True, sigma=0.6):
+    w = synth.Workload("pin", B=B, Hq=H, Hkv=H, d=d, S=S, sigma_n=sigma,
+                       k_outliers=synth.Outliers("mul", 4, factors=(50.0,) * 4) if outl else None,
+                       seed=seed)
+    K, V = synth.kv(w)
+    return K, V
+
+
+def _unpack_cache(cache, d, bits):
+    B, H, S, rb = cache["codes"].shape
+    q, bad = oracle.unpack_rows(cache["codes"].reshape(-1, rb), d, bits)
+    return q.reshape(B, H, S, d).astype(np.int64), bad
+
+
+def _check_codes(u64, sig16, q, qm, bits_ok_frac=1e-4):
+    """codes == clamp(rne(u / sigma16)), except within 1e-5 of a half point."""
+    inv = np.where(sig16 > 0, 1.0 / np.where(sig16 > 0, sig16, 1.0), 0.0)
+    y = u64 * inv
+    ref = np.clip(np.rint(y), -qm, qm)
+    frac = np.abs(np.abs(y - np.trunc(y)) - 0.5)
+    tie = frac < 1e-5
+    mism = ref != q
+    assert not np.any(mism & ~tie), int((mism & ~tie).sum())
+    assert np.abs(q).max() <= qm
+    return int(tie.sum())
+
+
+@pytest.mark.parametrize("bits", [4, 3, 2])
+@pytest.mark.parametrize("d", [64, 128])
+def test_nsep_pchan_closed_form(bits, d):
+    K, _ = _data(10 + bits, d=d)
+    x = K.astype(np.float64)
+    cfg = oracle_cfg("nsep+pchan", d, bits)
+    c = oracle.quantize(cfg, f16bits(K))
+    qm = oracle.qmax(bits)
+    # [P1] norm: FP16 of the L2 norm along the channel dimension
+    n64 = np.linalg.norm(x, axis=-1)
+    assert np.all(near_f16(c["tok"][..., 0], n64))
+    # the L_{-1} "norm" bug of the post would not pass this check
+    lm1 = 1.0 / np.sum(1.0 / np.abs(np.where(x == 0, 1e-3, x)), axis=-1)
+    assert not np.all(near_f16(c["tok"][..., 0], lm1))
+    # [P1]+[P2] unit direction, per-channel absmax over each 128-token block
+    u = x / n64[..., None]
+    B, H, S, _ = x.shape
+    ub = u.reshape(B, H, S // T, T, d)
+    m = np.abs(ub).max(axis=3)
+    assert np.all(near_f16(c["chan"], m / qm))
+    sig = f16val(c["chan"])[:, :, :, None, :]
+    q, bad = _unpack_cache(c, d, bits)
+    assert bad == 0
+    _check_codes(ub, sig, q.reshape(ub.shape), qm)
+    # the arg-max token of every channel codes to +-qmax
+    qb = q.reshape(ub.shape)
+    am = np.abs(ub).argmax(axis=3)
+    hit = np.take_along_axis(np.abs(qb), am[:, :, :, None, :], axis=3)
+    assert np.all(hit == qm)
+
+
+def test_naive_closed_form():
+    K, _ = _data(21)
+    x = K.astype(np.float64)
+    cfg = oracle_cfg("naive", 128, 4)
+    c = oracle.quantize(cfg, f16bits(K))
+    m = np.abs(x).max(axis=-1)
+    assert np.all(near_f16(c["tok"][..., 0], m / 7))
+    q, _ = _unpack_cache(c, 128, 4)
+    _check_codes(x, f16val(c["tok"][..., 0])[..., None], q, 7)
+
+
+def test_rht_closed_form():
+    d = 128
+    K, _ = _data(31)
+    x = K.astype(np.float64)
+    cfg = oracle_cfg("rht+nsep+pchan", d, 4)
+    R = scipy.linalg.hadamard(d) * cfg.signs[None, :].astype(np.float64) / np.sqrt(d)
+    c = oracle.quantize(cfg, f16bits(K))
+    n64 = np.linalg.norm(x, axis=-1)
+    assert np.all(near_f16(c["tok"][..., 0], n64))
+    u = (x @ R.T) / n64[..., None]                     # R x / ||x||
+    B, H, S, _ = x.shape
+    ub = u.reshape(B, H, S // T, T, d)
+    assert np.all(near_f16(c["chan"], np.abs(ub).max(axis=3) / 7, rel=1e-4))
+    q, _ = _unpack_cache(c, d, 4)
+    _check_codes(ub, f16val(c["chan"])[:, :, :, None, :], q.reshape(ub.shape), 7)
+
+
+@pytest.mark.parametrize("had", [True, False])
+def test_nsn_closed_form(had):
+    d = 128
+    w = synth.WORKLOADS["throughput"].scaled(B=1, Hkv=2, Hq=2, S=256)
+    K, _ = synth.kv(w)
+    x = K.astype(np.float64)
+    cfg = oracle_cfg("nsn+hadamard" if had else "nsn", d, 4)
+    c = oracle.quantize(cfg, f16bits(K))
+    sd = math.sqrt(d)
+    n1 = np.linalg.norm(x, axis=-1)
+    # [P3] normalize: token norm sqrt(d), s1 = ||x|| / sqrt(d)
+    assert np.all(near_f16(c["tok"][..., 0], n1 / sd))
+    a = x * (sd / n1[..., None])
+    B, H, S, _ = x.shape
+    ab = a.reshape(B, H, S // T, T, d)
+    # [P3] shift: per-channel mean over the block
+    o = ab.mean(axis=3)
+    assert np.all(near_f16(c["off"], o, rel=1e-5))
+    b = ab - f16val(c["off"])[:, :, :, None, :]
+    # [P3] normalize again: s2 = ||b|| / sqrt(d)
+    n2 = np.linalg.norm(b, axis=-1)
+    assert np.all(near_f16(c["tok"][..., 1].reshape(n2.shape), n2 / sd))
+    if had:
+        Hm = scipy.linalg.hadamard(d) / sd
+        u = (b @ Hm.T) / n2[..., None]
+    else:
+        u = b / n2[..., None]
+    assert np.all(near_f16(c["chan"], np.abs(u).max(axis=3) / 7, rel=1e-4))
+    q, _ = _unpack_cache(c, d, 4)
+    _check_codes(u, f16val(c["chan"])[:, :, :, None, :], q.reshape(u.shape), 7)
+    # after the shift the block channel means of b vanish (up to the fp16 mean)
+    assert np.max(np.abs((ab - o[:, :, :, None, :]).mean(axis=3))) < 1e-12
+
+
+# ------------------------------------------------------------- dequantize
+
+@pytest.mark.parametrize("mode,bits", [("nsep+pchan", 4), ("nsep+pchan", 3), ("nsep+pchan", 2),
+                                       ("naive", 4), ("rht+nsep+pchan", 4),
+                                       ("nsn+hadamard", 4), ("nsn+hadamard", 2), ("nsn", 4)])
+def test_reconstruction_within_quantization_bound(mode, bits):
+    d = 128
+    K, _ = _data(41 + bits, outl=True)
+    if mode.startswith("nsn"):
+        K, _ = synth.kv(synth.WORKLOADS["throughput"].scaled(B=1, Hkv=2, Hq=2, S=256))
+    x = K.astype(np.float64)
+    cfg = oracle_cfg(mode, d, bits)
+    c = oracle.quantize(cfg, f16bits(K))
+    xh, bad = oracle.dequantize(cfg, c, 0, x.shape[2])
+    assert bad == 0
+    B, H, S, _ = x.shape
+    err = np.linalg.norm(xh - x, axis=-1)
+    if mode == "naive":
+        s = f16val(c["tok"][..., 0])
+        bound = 0.5 * s * math.sqrt(d) * 1.001 + 1e-6
+    else:
+        sig = np.repeat(f16val(c["chan"]), T, axis=2)            # [B,H,S,d]
+        half = 0.5 * np.linalg.norm(sig, axis=-1)                # ||u - w|| bound
+        if mode.startswith("nsn"):
+            s1 = f16val(c["tok"][..., 0]); s2 = f16val(c["tok"][..., 1])
+            ob = np.repeat(f16val(c["off"]), T, axis=2)
+            sd = math.sqrt(d)
+            # x = s1 (s2 sqrt(d) R^T u + o); errors from codes and fp16 params
+            n1 = np.linalg.norm(x, axis=-1)
+            bound = s1 * s2 * sd * half * 1.01 + 2e-3 * n1 * (1 + np.linalg.norm(ob, axis=-1) / sd)
+        else:
+            n = f16val(c["tok"][..., 0])
+            bound = n * half * 1.001 + np.abs(n - np.linalg.norm(x, axis=-1)) + 1e-4 * n
+    assert np.all(err <= bound), float(np.max(err - bound))
+
+
+def test_on_grid_roundtrip_exact():
+    """Vectors already on the grid come back bit-exactly (INT4/3/2, d=64/128)."""
+    rng = np.random.default_rng(5)
+    cases = {4: [7, 3, 2, 1, 1], 3: [3, 2, 1, 1, 1], 2: [1, 1, 1, 1]}
+    for d in (64, 128):
+        for bits, mags in cases.items():
+            s = 2.0 ** rng.integers(-3, 3)
+            q = np.zeros((T, d), np.int64)
+            for t in range(T):
+                first = t % d
+                others = rng.choice([c for c in range(d) if c != first], len(mags) - 1, replace=False)
+                chans = [first, *others]
+                q[t, chans] = np.array(mags) * rng.choice([-1, 1], len(mags))
+            x = (q * s).astype(np.float16)[None, None]
+            cfg = oracle_cfg("nsep+pchan", d, bits)
+            c = oracle.quantize(cfg, f16bits(x))
+            got, _ = _unpack_cache(c, d, bits)
+            assert np.array_equal(got[0, 0], q)
+            xh, _ = oracle.dequantize(cfg, c, 0, T)
+            assert np.array_equal(xh[0, 0], x[0, 0].astype(np.float32))
+    # naive INT4 on its own grid: per-token max 7 s
+    q = rng.integers(-7, 8, (T, 128)); q[:, 5] = 7
+    x = (q * 0.25).astype(np.float16)[None, None]
+    cfg = oracle_cfg("naive", 128, 4)
+    c = oracle.quantize(cfg, f16bits(x))
+    xh, _ = oracle.dequantize(cfg, c, 0, T)
+    assert np.array_equal(xh[0, 0], x[0, 0].astype(np.float32))
+
+
+def test_zero_vectors_and_tiny_scales():
+    d = 128
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((1, 1, T, d)).astype(np.float16)
+    x[0, 0, :, 11] = 0                   # a zero channel
+    x[0, 0, :, 12] = np.float16(1e-6)    # a channel whose scale is an fp16 subnormal
+    x[0, 0, 3, 12] = np.float16(-3e-6)
+    x[0, 0, 7] = 0                       # a zero token
+    for mode in ("nsep+pchan", "naive", "nsn+hadamard", "rht+nsep+pchan"):
+        cfg = oracle_cfg(mode, d, 4)
+        c = oracle.quantize(cfg, f16bits(x))
+        q, bad = _unpack_cache(c, d, 4)
+        assert bad == 0 and np.abs(q).max() <= 7
+        xh, _ = oracle.dequantize(cfg, c, 0, T)
+        assert np.all(np.isfinite(xh))
+        if mode != "nsn+hadamard":
+            assert np.all(xh[0, 0, 7] == 0)
+        if mode == "nsep+pchan":
+            assert np.all(q[0, 0, :, 11] == 0)
+            assert f16val(c["tok"][0, 0, 7, 0]) == 0
+
+
+# ------------------------------------------------------------- attention
+
+def test_attention_matches_scipy_softmax():
+    rng = np.random.default_rng(8)
+    B, Hq, Hkv, L, d = 2, 6, 2, 77, 64
+    q = rng.standard_normal((B, Hq, d)).astype(np.float16)
+    k = (rng.standard_normal((B, Hkv, L, d)) * 3).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, L, d)).astype(np.float32)
+    out = oracle.attention(f16bits(q), k, v, None)
+    g = Hq // Hkv
+    for b in range(B):
+        for j in range(Hq):
+            h = j // g
+            lg = (k[b, h].astype(np.float64) @ q[b, j].astype(np.float64)) / math.sqrt(d)
+            p = scipy.special.softmax(lg)
+            ref = p @ v[b, h].astype(np.float64)
+            assert np.allclose(out[b, j], ref, rtol=1e-12, atol=1e-13)
+    assert np.all(oracle.attention(f16bits(q), k[:, :, :0], v[:, :, :0]) == 0)
+
+
+def test_attention_error_nonincreasing_in_bits():
+    w = synth.WORKLOADS["tiny"]
+    K, V = synth.kv(w)
+    q = synth.queries(w)
+    ref = oracle.attention(f16bits(q), K.astype(np.float32), V.astype(np.float32))
+    errs = []
+    for bits in (2, 3, 4, 6, 8):
+        cfg = oracle_cfg("nsep+pchan", w.d, bits)
+        ck = oracle.quantize(cfg, f16bits(K)); cv = oracle.quantize(cfg, f16bits(V))
+        kh, _ = oracle.dequantize(cfg, ck, 0, w.S); vh, _ = oracle.dequantize(cfg, cv, 0, w.S)
+        errs.append(float(np.max(np.abs(oracle.attention(f16bits(q), kh, vh) - ref))))
+    assert all(b <= a * 1.05 for a, b in zip(errs, errs[1:])), errs
+    assert errs[-1] < errs[0] / 20, errs
+
+
+def test_outlier_channels_do_not_take_over_scales():
+    """Injected outlier channels no longer dominate the other channels'
+    resolution under nsep+pchan, while per-token absmax INT4 degrades."""
+    d = 128
+    res = {}
+    for outl in (False, True):
+        K, _ = _data(51, B=1, H=4, S=512, outl=outl)
+        chans = synth.outlier_channels(synth.Workload("pin", 1, 4, 4, d, 512, seed=51,
+                                                      k_outliers=synth.Outliers("mul", 4, (50.0,) * 4)))
+        keep = np.setdiff1d(np.arange(d), chans)
+        x = K.astype(np.float64)
+        for mode in ("nsep+pchan", "naive"):
+            cfg = oracle_cfg(mode, d, 4)
+            xh, _ = oracle.dequantize(cfg, oracle.quantize(cfg, f16bits(K)), 0, 512)
+            e = xh[..., keep] - x[..., keep]
+            res[(mode, outl)] = math.sqrt(np.mean(e ** 2) / np.mean(x[..., keep] ** 2))
+    assert res[("nsep+pchan", True)] <= 2.0 * res[("nsep+pchan", False)], res
+    assert res[("naive", True)] >= 5.0 * res[("naive", False)], res
