@@ -1,0 +1,408 @@
+#!/usr/bin/env python3
+"""Benchmark of the hot path on the throughput workload (the largest of the
+five configurations): batch 64, 32 query heads / 8 kv heads, head dim 128,
+8192 prefilled tokens + 256 tokens streamed one per decode step, NSN +
+plain Hadamard, INT4 codes.
+
+One step = one pass of the whole path over one batch:
+  kvq_quantize_block over the 8192-token prefill (K and V), then 256 x
+  [kvq_append_token (two of them flush a block) + kvq_decode_attention].
+`value` = algorithmic bytes of every call in the step / step time (GB/s);
+decode dominates it.  Inputs (1 GiB each of K and V, the queries and the
+streamed tokens) are resident in HBM before the timed region; the 604 MB
+packed cache is larger than the 126 MB L2, so no flush is needed between
+iterations.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun each rank runs its own batch (weak scaling, no collective on
+the data path); the step time is the max over ranks.  `--impl reference`
+times the CPU oracle (the plain C reference of the method) on the host
+cores over a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_bit_b200 import accounting, synth  # noqa: E402
+
+WORKLOAD = "throughput"
+MODE = "nsn+hadamard"
+BITS = 4
+METRIC = "INT4-KV decode attention GB/s (% of HBM peak) & tokens/s; quantize GB/s"
+
+
+def measured_peak_gbs():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def flags_of(mode: str) -> int:
+    names, _ = synth.MODES[mode]
+    m = {"NORM_SEP": 1, "PER_CHANNEL": 2, "NSN": 4, "HADAMARD": 8}
+    f = 0
+    for n in names:
+        f |= m[n]
+    return f
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while the
+    timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.uuid:
+            cmd[1:1] = ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle sample
+
+def run_oracle_sample(w, mode, bits, pairs, threads):
+    """The CPU oracle over `pairs` (batch row, kv head) slices of the
+    workload: quantize of the prefill (K and V), then one decode attention of
+    the slices' query heads over the quantized cache (dequantize + fp64
+    attention).  Returns (decode bytes, decode seconds, quantize bytes,
+    quantize seconds)."""
+    import oracle
+    names, seeded = synth.MODES[mode]
+    flags = flags_of(mode)
+    cfg = oracle.Cfg(d=w.d, bits=bits, flags=flags,
+                     signs=oracle.make_signs(synth.SIGN_SEED, w.d) if seeded else None)
+    G = w.Hq // w.Hkv
+    # sample slices: the first `pairs` kv heads of batch row 0 (more rows if needed)
+    ws = w.scaled(B=max(1, (pairs + w.Hkv - 1) // w.Hkv))
+    K, V = synth.kv(ws)
+    q = synth.queries(ws)
+    Kb = K.reshape(-1, 1, w.S, w.d)[:pairs]
+    Vb = V.reshape(-1, 1, w.S, w.d)[:pairs]
+    k16 = np.ascontiguousarray(Kb).view(np.uint16)
+    v16 = np.ascontiguousarray(Vb).view(np.uint16)
+    t0 = time.perf_counter()
+    ck = oracle.quantize(cfg, k16, threads=threads)
+    cv = oracle.quantize(cfg, v16, threads=threads)
+    tq = time.perf_counter() - t0
+    qh = q.reshape(-1, G, w.d)[:pairs]                      # [pairs, G, d]
+    t0 = time.perf_counter()
+    kh, _ = oracle.dequantize(cfg, ck, 0, w.S, threads)
+    vh, _ = oracle.dequantize(cfg, cv, 0, w.S, threads)
+    oracle.attention(np.ascontiguousarray(qh).view(np.uint16).reshape(pairs, G, w.d), kh, vh, None, threads)
+    td = time.perf_counter() - t0
+    bq = accounting.quantize_bytes(w.d, bits, flags, pairs, 1, w.S)
+    bd = accounting.decode_bytes(w.d, bits, flags, pairs, 1, G, w.S)
+    return bd, td, bq, tq
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[WORKLOAD]
+    threads = host_cores()
+    pairs = 4
+    for _ in range(args.warmup):
+        run_oracle_sample(w, MODE, BITS, pairs, threads)
+    tot_b, tot_s = 0.0, 0.0
+    for _ in range(args.steps):
+        bd, td, bq, tq = run_oracle_sample(w, MODE, BITS, pairs, threads)
+        tot_b += bd
+        tot_s += td
+    gbs = tot_b / tot_s / 1e9
+    sample = (f"{pairs} (batch row, kv head) slices of the {WORKLOAD} workload per step "
+              f"({w.S} tokens, {w.Hq // w.Hkv} query heads each): oracle dequantize + fp64 attention")
+    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "mode": MODE, "bits": BITS, "batch": w.B, "q_heads": w.Hq,
+                       "kv_heads": w.Hkv, "head_dim": w.d, "seq_len": w.S, "streamed": w.stream},
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank: int, world: int):
+    import torch
+    from kv_cache_bit_b200 import kvq
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[WORKLOAD].scaled(seed=rank)
+    flags = flags_of(MODE)
+    G = w.Hq // w.Hkv
+    n_stream = w.stream
+    cap = ((w.S + n_stream + 127) // 128) * 128
+
+    # inputs, resident before timing
+    K, V = synth.kv(w)
+    ks, vs = synth.stream_tokens(w)
+    qs = synth.queries(w, steps=n_stream)
+    tod = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
+    Kd, Vd, ksd, vsd, qsd = tod(K), tod(V), tod(ks), tod(vs), tod(qs)
+    cfg = kvq.Config(w.d, BITS, flags, None, device=dev)
+    cache = kvq.KVCache.allocate(cfg, w.B, w.Hkv, cap, device=dev)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    ws_bytes = kvq.kvq_decode_workspace_bytes(cfg, cache, w.Hq)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = []
+
+    def step(record: bool):
+        cache.c.len = 0
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True); e0.record(stream)
+        kvq.kvq_quantize_block(cfg, cache, Kd, Vd, 0, w.S, stream)
+        if record:
+            e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
+            ev.append(("quantize", e0, e1))
+        for i in range(n_stream):
+            kvq.kvq_append_token(cfg, cache, ksd[i], vsd[i], stream)
+            if record:
+                d0 = torch.cuda.Event(enable_timing=True); d0.record(stream)
+            kvq.kvq_decode_attention(cfg, cache, qsd[i], w.Hq, 0.0, out, ws, ws_bytes, stream)
+            if record:
+                d1 = torch.cuda.Event(enable_timing=True); d1.record(stream)
+                ev.append(("decode", d0, d1))
+
+    # algorithmic bytes of one step
+    step_bytes = accounting.quantize_bytes(w.d, BITS, flags, w.B, w.Hkv, w.S)
+    dec_bytes = []
+    for i in range(n_stream):
+        length = w.S + i + 1
+        step_bytes += accounting.append_bytes(w.d, BITS, flags, w.B, w.Hkv, flush=(length % 128 == 0))
+        db = accounting.decode_bytes(w.d, BITS, flags, w.B, w.Hkv, w.Hq, length)
+        dec_bytes.append(db)
+        step_bytes += db
+    launches_per_step = 1 + n_stream * (1 + 2)
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.5)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    q_ms = [a.elapsed_time(b) for k, a, b in ev if k == "quantize"]
+    d_ms = [a.elapsed_time(b) for k, a, b in ev if k == "decode"]
+    dec_avg_bytes = sum(dec_bytes) / len(dec_bytes)
+    dec_avg_s = (sum(d_ms) / len(d_ms)) / 1e3
+    q_avg_s = (sum(q_ms) / len(q_ms)) / 1e3
+    q_bytes = accounting.quantize_bytes(w.d, BITS, flags, w.B, w.Hkv, w.S)
+    peak, peak_kind = measured_peak_gbs()
+    dec_gbs = dec_avg_bytes / dec_avg_s / 1e9
+    q_gbs = q_bytes / q_avg_s / 1e9
+    value = world * step_bytes / (ms / 1e3) / 1e9
+
+    # end to end through the public calls, host buffers, copies inside the region
+    e2e = run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, dev, step_bytes, world)
+
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "mode": MODE, "bits": BITS, "batch": w.B, "q_heads": w.Hq,
+                   "kv_heads": w.Hkv, "head_dim": w.d, "seq_len": w.S, "streamed": n_stream,
+                   "l2": "inputs larger than L2 (packed cache 604 MB, fp16 prefill 2 GiB)",
+                   "parallelism": f"weak x{world} (independent batches, no collective)"},
+        "decode": {"gbs": dec_gbs, "frac_of_hbm": dec_gbs / peak, "us_per_call": dec_avg_s * 1e6,
+                   "tokens_per_s": world * w.B / dec_avg_s, "bytes_per_call": dec_avg_bytes},
+        "quantize": {"gbs": q_gbs, "frac_of_hbm": q_gbs / peak, "us_per_call": q_avg_s * 1e6,
+                     "bytes_per_call": q_bytes},
+        "tokens_per_s": world * w.B * n_stream / (ms / 1e3),
+        "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
+                     "traffic": None, "kernel": "kvq_decode_attention (split + combine launches)",
+                     "peak_kind": f"{peak_kind} copy bandwidth"},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        bd, td, bq, tq = run_oracle_sample(w, MODE, BITS, 4, host_cores())
+        line["cpu_baseline"] = {"value": bd / td / 1e9, "unit": "GB/s", "cores": host_cores(), "kind": "oracle",
+                                "sample": f"4 (batch row, kv head) slices x {w.S} tokens, {G} query heads: "
+                                          f"oracle dequantize + fp64 attention ({td:.1f} s); "
+                                          f"quantize {bq / tq / 1e9:.3f} GB/s ({tq:.1f} s)"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, dev, step_bytes, world):
+    """Same step through the public calls with pinned HOST inputs: the prefill,
+    the streamed tokens and the queries are copied host->device inside the
+    timed region, and every decode output is copied back."""
+    import torch
+    from kv_cache_bit_b200 import kvq
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()
+    Kh, Vh, ksh, vsh, qsh = pin(K), pin(V), pin(ks), pin(vs), pin(qs)
+    Kd = torch.empty_like(Kh, device=dev)
+    Vd = torch.empty_like(Vh, device=dev)
+    ktok = torch.empty_like(ksh[0], device=dev)
+    vtok = torch.empty_like(vsh[0], device=dev)
+    qd = torch.empty_like(qsh[0], device=dev)
+    outh = torch.empty((w.stream,) + tuple(out.shape), dtype=torch.float32).pin_memory()
+
+    def step():
+        cache.c.len = 0
+        Kd.copy_(Kh, non_blocking=True)
+        Vd.copy_(Vh, non_blocking=True)
+        kvq.kvq_quantize_block(cfg, cache, Kd, Vd, 0, w.S, stream)
+        for i in range(w.stream):
+            ktok.copy_(ksh[i], non_blocking=True)
+            vtok.copy_(vsh[i], non_blocking=True)
+            qd.copy_(qsh[i], non_blocking=True)
+            kvq.kvq_append_token(cfg, cache, ktok, vtok, stream)
+            kvq.kvq_decode_attention(cfg, cache, qd, w.Hq, 0.0, out, ws, ws_bytes, stream)
+            outh[i].copy_(out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 3))
+    if world > 1:
+        torch.distributed.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = (Kh.numel() + Vh.numel()) * 2 + w.stream * (ksh[0].numel() + vsh[0].numel() + qsh[0].numel()) * 2
+    d2h = w.stream * out.numel() * 4
+    return {"value": world * step_bytes / (ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        return run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,216 @@
+/*
+ * kvq.h -- C ABI of libkvq: low-bit KV-cache quantization (norm separation +
+ * per-channel block scales, optional randomized Hadamard rotation, optional
+ * Normalize-Shift-Normalize) and decode attention over the packed cache,
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Sources the calls follow (page title, section):
+ *  - "KV cache INT4 quantization ... nsep+pchan" post, section "Fix
+ *    (nsep+pchan)": each K/V vector becomes an FP16 norm plus a unit
+ *    direction; the direction is quantized with per-channel scales and
+ *    symmetric round-to-nearest codes (+-7 at INT4); a drop-in step in front
+ *    of the cache, with no training or calibration.
+ *  - "Rotated Runtime Smooth" analysis, master equation and symbol list: the
+ *    rotation R = (1/sqrt(K)) [+-1] with R R^T = I, the runtime per-channel
+ *    scale s_j = max over tokens of |channel j|, alpha = max|X|/(2^(N-1)-1).
+ *  - "NSNQuant" explainer, "Method" (Normalize-Shift-Normalize with side
+ *    products s1, o, s2; Hadamard transform) and "Implementation details"
+ *    (quantized part plus a full-precision residual that is flushed into the
+ *    quantized part when full; attention computed directly from the codes with
+ *    the side products folded into the kernel).
+ *  - "Activation-guided compensation and orthogonal residuals" abstract:
+ *    randomized Hadamard rotation with random sign patterns.
+ *
+ * Conventions for every call:
+ *  - All data pointers are DEVICE pointers unless a comment says "host".
+ *    The library never allocates or frees memory; the caller owns every
+ *    buffer.  Device pointers must be 16-byte aligned.
+ *  - fp16 data is passed as uint16_t bit patterns (IEEE binary16).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    only enqueue work and never synchronize.
+ *  - Every argument is checked on the host before anything is enqueued; a
+ *    failed check returns an error and changes no state.  Errors reported by
+ *    the CUDA runtime at launch are returned as KVQ_ERR_CUDA.
+ *  - The library holds no global state; calls on distinct caches may be made
+ *    from several host threads.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1, /* null or misaligned pointer, bad size or range */
+    KVQ_ERR_UNSUPPORTED = 2, /* head_dim / bits / flag set not built for the GPU */
+    KVQ_ERR_CAPACITY = 3,    /* write past the cache capacity */
+    KVQ_ERR_WORKSPACE = 4,   /* decode workspace missing or too small */
+    KVQ_ERR_CUDA = 5         /* the CUDA runtime reported an error */
+} kvq_status;
+
+/* Quantizer flags. */
+enum {
+    KVQ_NORM_SEP = 1u,    /* split off the FP16 L2 norm; quantize the unit direction */
+    KVQ_PER_CHANNEL = 2u, /* per-channel scale over each 128-token block (else per token) */
+    KVQ_NSN = 4u,         /* Normalize-Shift-Normalize before quantization */
+    KVQ_HADAMARD = 8u     /* (randomized) Hadamard rotation of the direction */
+};
+
+#define KVQ_BLOCK_TOKENS 128
+
+/*
+ * Quantizer configuration.  Flag sets built for the GPU:
+ *   NORM_SEP | PER_CHANNEL            nsep+pchan
+ *   NORM_SEP | PER_CHANNEL | HADAMARD randomized Hadamard, then nsep+pchan
+ *   0                                  naive per-token absmax
+ *   NSN | PER_CHANNEL [| HADAMARD]     NSN (+ Hadamard), per-channel codes
+ * head_dim in {64, 128}; bits in {2, 3, 4}.
+ */
+typedef struct {
+    int32_t head_dim;
+    int32_t bits;
+    uint32_t flags;
+    int32_t reserved;    /* must be 0 */
+    const int8_t* signs; /* device [head_dim] of +-1 used by HADAMARD (the same
+                            vector rotates K, V, queries and outputs); NULL means
+                            all +1, i.e. the plain Hadamard transform */
+} kvq_config;
+
+/*
+ * The packed cache.  Caller-allocated; index [2] selects K (0) or V (1).
+ * Shapes (row-major, B = batch, H = kv_heads, S = capacity, nb = S / 128):
+ *   codes[i] uint8  [B][H][S][row_bytes]   row_bytes = kvq_row_bytes(head_dim, bits)
+ *   tok[i]   fp16   [B][H][S][ntok]        ntok = kvq_tok_params(flags):
+ *                                          nsep: norm; naive: scale; NSN: s1, s2
+ *   chan[i]  fp16   [B][H][nb][head_dim]   per-channel block scale (PER_CHANNEL, else NULL)
+ *   off[i]   fp16   [B][H][nb][head_dim]   NSN per-channel block mean (NSN, else NULL)
+ *   resid[i] fp16   [B][H][128][head_dim]  residual tokens not yet quantized
+ * Code layout per token row: offset-binary e = q + 2^(bits-1) (never 0);
+ *   INT4 byte j = e[2j] | e[2j+1] << 4; INT2 byte j = e[4j] | e[4j+1] << 2 |
+ *   e[4j+2] << 4 | e[4j+3] << 6; INT3 = head_dim/4 bytes of (e & 3) in the
+ *   INT2 layout followed by head_dim/8 bytes whose bit i of byte j is bit 2
+ *   of e[8j+i].
+ * `len` is the number of tokens stored: tokens [0, 128*floor(len/128)) are in
+ * the quantized blocks, the remaining len % 128 are residual slots
+ * 0 .. len%128-1.  The library updates `len` on the host struct after a
+ * successful enqueue of kvq_quantize_block or kvq_append_token.
+ */
+typedef struct {
+    int32_t batch, kv_heads, head_dim, capacity;
+    int64_t len;
+    uint8_t* codes[2];
+    uint16_t* tok[2];
+    uint16_t* chan[2];
+    uint16_t* off[2];
+    uint16_t* resid[2];
+} kvq_cache;
+
+/* Bytes of one packed token row; 0 for an unsupported (head_dim, bits). */
+int32_t kvq_row_bytes(int32_t head_dim, int32_t bits);
+
+/* fp16 per-token parameters stored for a flag set (ntok above); -1 if the
+   flag set is not built for the GPU. */
+int32_t kvq_tok_params(uint32_t flags);
+
+/*
+ * Random signs of the randomized Hadamard rotation ("random sign patterns",
+ * randomized Hadamard abstract; R = (1/sqrt(K))[+-1], Rotated Runtime Smooth
+ * symbol list).  HOST function: writes head_dim values of +-1 to host_out.
+ * sign_c = -1 iff bit 63 of the c-th SplitMix64 output from state `seed` is
+ * set (SplitMix64: Steele, Lea & Flood 2014).  Copy the result to the device
+ * for kvq_config.signs.  KVQ_ERR_INVALID_ARG if host_out is NULL or
+ * head_dim < 1.
+ */
+kvq_status kvq_make_signs(uint64_t seed, int32_t head_dim, int8_t* host_out);
+
+/*
+ * Quantize ntok tokens of K and of V into the cache blocks starting at token
+ * t0 (the prefill / bulk path).  nsep+pchan post "Fix (nsep+pchan)" (norm +
+ * direction, per-channel scales, codes +-qmax); NSNQuant "Method" (NSN,
+ * Hadamard); Rotated Runtime Smooth symbol list (per-channel absmax over
+ * tokens, qmax = 2^(N-1)-1).
+ *   k, v   fp16 [B][H][ntok][head_dim], contiguous
+ *   t0     multiple of 128; ntok > 0 and a multiple of 128
+ * Per (b, h, block, tensor) one CTA reads the 128 x head_dim tile once and
+ * writes codes, per-token parameters and per-block channel scales/means.
+ * On success len = max(len, t0 + ntok).
+ * Errors: INVALID_ARG (null/misaligned pointers, t0 or ntok not multiples of
+ * 128, or a range that overlaps residual tokens that are still held, i.e.
+ * t0 + ntok > 128*floor(len/128) while len % 128 != 0); CAPACITY
+ * (t0 + ntok > capacity); UNSUPPORTED; CUDA.
+ */
+kvq_status kvq_quantize_block(const kvq_config* cfg, kvq_cache* cache,
+                              const uint16_t* k, const uint16_t* v,
+                              int64_t t0, int64_t ntok, void* stream);
+
+/*
+ * Append one token per (b, h) to the residual (NSNQuant "Implementation
+ * details": full-precision residual flushed into the quantized part when
+ * full).  k_new, v_new fp16 [B][H][head_dim].  The token goes to residual
+ * slot len % 128; when that slot is 127 the same launch quantizes the 128
+ * residual tokens into block floor(len/128) exactly as kvq_quantize_block
+ * would, which empties the residual.  On success len += 1.
+ * Errors: INVALID_ARG; CAPACITY (len + 1 > capacity); UNSUPPORTED; CUDA.
+ */
+kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache,
+                            const uint16_t* k_new, const uint16_t* v_new, void* stream);
+
+/* Workspace bytes kvq_decode_attention needs for this cache and q_heads
+   (partial softmax states of the sequence splits); 0 on invalid arguments.
+   The workspace must be zero-filled once when it is allocated: the decode
+   call leaves its counters at zero again when it completes. */
+size_t kvq_decode_workspace_bytes(const kvq_config* cfg, const kvq_cache* cache, int32_t q_heads);
+
+/*
+ * Decode attention of one query token per sequence over the cache:
+ *   out[b, j] = sum_{t < len} softmax_t(scale * q[b, j] . x_hat^K_t) x_hat^V_t
+ * with query head j reading kv head j / (q_heads / kv_heads).  Quantized
+ * tokens are read as packed codes plus their side parameters and are never
+ * expanded in memory (NSNQuant "Implementation details": the side products
+ * are folded into the attention kernel); residual tokens are attended at
+ * their fp16 values.  x_hat is the tensor kvq_dequantize rebuilds.
+ *   q     fp16 [B][q_heads][head_dim]; q_heads a multiple of kv_heads,
+ *         q_heads / kv_heads <= 8
+ *   scale softmax scale; <= 0 selects 1/sqrt(head_dim)
+ *   out   fp32 [B][q_heads][head_dim]; len == 0 gives zeros
+ *   ws    workspace of at least kvq_decode_workspace_bytes(), zero-filled
+ *         when first allocated; calls that share a workspace must not
+ *         overlap in time
+ * Errors: INVALID_ARG; WORKSPACE; UNSUPPORTED; CUDA.
+ */
+kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache,
+                                const uint16_t* q, int32_t q_heads, float scale,
+                                float* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Rebuild fp32 values of quantized tokens [t0, t0 + ntok) of K (tensor 0) or
+ * V (tensor 1): out fp32 [B][H][ntok][head_dim].  x_hat = norm * (q * sigma)
+ * (nsep); inverse rotation for HADAMARD; s1 * (s2 * sqrt(d) R^T (q * sigma) +
+ * o) for NSN (NSNQuant "Method": the side products rebuild the tensor).
+ * Errors: INVALID_ARG (t0, ntok not multiples of 128, or the range is not
+ * inside the quantized part); UNSUPPORTED; CUDA.
+ */
+kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t tensor,
+                          int64_t t0, int64_t ntok, float* out, void* stream);
+
+/*
+ * Read (and, if clear != 0, reset) the sticky device error word of the
+ * current device: bit 0 = a kernel gave up waiting for a TMA tile, bit 1 = a
+ * kernel gave up waiting on a barrier.  Kernels that give up write no
+ * results.  This word is the library's only device-global state.  HOST call;
+ * synchronizes the device.  Errors: INVALID_ARG (host_out NULL); CUDA.
+ */
+kvq_status kvq_read_device_errors(uint32_t* host_out, int32_t clear);
+
+/* Static description of a status code. */
+const char* kvq_status_string(kvq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H */

@@ -1,0 +1,403 @@
+// kvq_api.cu -- host side of libkvq: argument checks, shape arithmetic,
+// tensor-map set-up and kernel launches behind the C ABI of include/kvq.h.
+// This is the library's single translation unit; the kernels come in from
+// the .cuh files below.
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kvq.h"
+#include "kvq_decode_simple.cuh"
+#include "kvq_quant.cuh"
+
+namespace kvq {
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+
+struct ModeInfo {
+    int mode = -1;
+    bool had = false;
+};
+
+ModeInfo mode_of(uint32_t flags) {
+    ModeInfo m;
+    const uint32_t base = flags & ~uint32_t(KVQ_HADAMARD);
+    m.had = (flags & KVQ_HADAMARD) != 0;
+    if (base == (KVQ_NORM_SEP | KVQ_PER_CHANNEL)) m.mode = kNsep;
+    else if (flags == 0) m.mode = kNaive;
+    else if (base == (KVQ_NSN | KVQ_PER_CHANNEL)) m.mode = kNsn;
+    return m;
+}
+
+int row_bytes(int d, int bits) {
+    if ((d != 64 && d != 128) || bits < 2 || bits > 4) return 0;
+    return d * bits / 8;
+}
+
+// Status of a config; fills mode info.
+kvq_status check_cfg(const kvq_config* cfg, ModeInfo* mi) {
+    if (cfg == nullptr) return KVQ_ERR_INVALID_ARG;
+    if (cfg->reserved != 0) return KVQ_ERR_INVALID_ARG;
+    if (cfg->signs != nullptr && !aligned16(cfg->signs)) return KVQ_ERR_INVALID_ARG;
+    if (row_bytes(cfg->head_dim, cfg->bits) == 0) return KVQ_ERR_UNSUPPORTED;
+    *mi = mode_of(cfg->flags);
+    if (mi->mode < 0) return KVQ_ERR_UNSUPPORTED;
+    return KVQ_OK;
+}
+
+// Shape and pointer checks of a cache against a config.
+kvq_status check_cache(const kvq_config* cfg, const ModeInfo& mi, const kvq_cache* c) {
+    if (c == nullptr) return KVQ_ERR_INVALID_ARG;
+    if (c->batch < 1 || c->kv_heads < 1 || c->head_dim != cfg->head_dim) return KVQ_ERR_INVALID_ARG;
+    if (c->capacity < kT || c->capacity % kT != 0) return KVQ_ERR_INVALID_ARG;
+    if (c->len < 0 || c->len > c->capacity) return KVQ_ERR_INVALID_ARG;
+    if ((int64_t)c->batch * c->kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
+    for (int i = 0; i < 2; ++i) {
+        if (!ok_ptr(c->codes[i]) || !ok_ptr(c->tok[i]) || !ok_ptr(c->resid[i])) return KVQ_ERR_INVALID_ARG;
+        if (mi.mode != kNaive && !ok_ptr(c->chan[i])) return KVQ_ERR_INVALID_ARG;
+        if (mi.mode == kNsn && !ok_ptr(c->off[i])) return KVQ_ERR_INVALID_ARG;
+    }
+    return KVQ_OK;
+}
+
+kvq_status launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+float rsqd_of(int d) { return (float)(1.0 / std::sqrt((double)d)); }
+float sqd_of(int d) { return (float)std::sqrt((double)d); }
+
+// Compile-time dispatch over (head_dim, bits, mode, hadamard).
+template <int D, int BITS, typename Fn>
+kvq_status dispatch_mode(const ModeInfo& mi, Fn& fn) {
+    if (mi.mode == kNsep) return mi.had ? fn.template run<D, BITS, kNsep, true>() : fn.template run<D, BITS, kNsep, false>();
+    if (mi.mode == kNaive) return mi.had ? KVQ_ERR_UNSUPPORTED : fn.template run<D, BITS, kNaive, false>();
+    return mi.had ? fn.template run<D, BITS, kNsn, true>() : fn.template run<D, BITS, kNsn, false>();
+}
+
+template <typename Fn>
+kvq_status dispatch(int d, int bits, const ModeInfo& mi, Fn& fn) {
+    if (d == 64) {
+        if (bits == 2) return dispatch_mode<64, 2>(mi, fn);
+        if (bits == 3) return dispatch_mode<64, 3>(mi, fn);
+        if (bits == 4) return dispatch_mode<64, 4>(mi, fn);
+    } else if (d == 128) {
+        if (bits == 2) return dispatch_mode<128, 2>(mi, fn);
+        if (bits == 3) return dispatch_mode<128, 3>(mi, fn);
+        if (bits == 4) return dispatch_mode<128, 4>(mi, fn);
+    }
+    return KVQ_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------- TMA maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D view [rows][d] of fp16 rows; boxes of 64 channels x 128 rows with
+// 128-byte swizzle.
+bool make_row_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kT};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+QuantArgs quant_args(const kvq_config* cfg, const kvq_cache* c) {
+    QuantArgs a;
+    for (int i = 0; i < 2; ++i) {
+        a.codes[i] = c->codes[i];
+        a.tok[i] = reinterpret_cast<__half*>(c->tok[i]);
+        a.chan[i] = reinterpret_cast<__half*>(c->chan[i]);
+        a.off[i] = reinterpret_cast<__half*>(c->off[i]);
+    }
+    a.signs = cfg->signs;
+    a.H = c->kv_heads;
+    a.cap = c->capacity;
+    a.ntok = 0;
+    a.blk0 = 0;
+    a.rsqd = rsqd_of(cfg->head_dim);
+    a.sqd = sqd_of(cfg->head_dim);
+    return a;
+}
+
+// ---------------------------------------------------------------- launchers
+
+struct QuantLaunch {
+    QuantArgs a;
+    const void* k;
+    const void* v;
+    int bh;
+    int nblk;
+    cudaStream_t st;
+    template <int D, int BITS, int MODE, bool HAD>
+    kvq_status run() {
+        CUtensorMap mk, mv;
+        const uint64_t rows = (uint64_t)bh * (uint64_t)a.ntok;
+        if (!make_row_map(&mk, k, rows, D) || !make_row_map(&mv, v, rows, D)) return KVQ_ERR_CUDA;
+        constexpr int smem = quant_smem_bytes<D, MODE>();
+        static bool attr = false;
+        if (!attr) attr = set_smem(quantize_kernel<D, BITS, MODE, HAD>, smem);
+        if (!attr) return KVQ_ERR_CUDA;
+        quantize_kernel<D, BITS, MODE, HAD><<<dim3(nblk, bh, 2), kT, smem, st>>>(mk, mv, a);
+        return launch_status();
+    }
+};
+
+struct AppendLaunch {
+    AppendArgs a;
+    int bh;
+    cudaStream_t st;
+    template <int D, int BITS, int MODE, bool HAD>
+    kvq_status run() {
+        constexpr int smem = quant_smem_bytes<D, MODE>();
+        static bool attr = false;
+        if (!attr) attr = set_smem(append_kernel<D, BITS, MODE, HAD>, smem);
+        if (!attr) return KVQ_ERR_CUDA;
+        append_kernel<D, BITS, MODE, HAD><<<dim3(bh, 2), kT, a.slot == kT - 1 ? smem : 0, st>>>(a);
+        return launch_status();
+    }
+};
+
+struct DequantLaunch {
+    DequantArgs a;
+    int bh, nblk;
+    cudaStream_t st;
+    template <int D, int BITS, int MODE, bool HAD>
+    kvq_status run() {
+        dequantize_kernel<D, BITS, MODE, HAD><<<dim3(nblk, bh), kT, 0, st>>>(a);
+        return launch_status();
+    }
+};
+
+struct DecodeLaunch {
+    DecodeArgs a;
+    int bh;
+    cudaStream_t st;
+    template <int D, int BITS, int MODE, bool HAD>
+    kvq_status run() {
+        decode_split_kernel<D, BITS, MODE, HAD><<<dim3(a.nsplit, bh), kT, 0, st>>>(a);
+        kvq_status s = launch_status();
+        if (s != KVQ_OK) return s;
+        decode_combine_kernel<D, HAD><<<bh, kT, 0, st>>>(a);
+        return launch_status();
+    }
+};
+
+// Splits of the sequence for decode: enough CTAs to cover the GPU twice,
+// fixed per cache shape so the workspace size does not depend on len.
+int decode_splits(const kvq_cache* c) {
+    const int bh = c->batch * c->kv_heads;
+    const int nb = c->capacity / kT;
+    int ns = (296 + bh - 1) / bh;
+    if (ns > nb) ns = nb;
+    if (ns < 1) ns = 1;
+    return ns;
+}
+
+}  // namespace
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+int32_t kvq_row_bytes(int32_t head_dim, int32_t bits) { return row_bytes(head_dim, bits); }
+
+int32_t kvq_tok_params(uint32_t flags) {
+    const ModeInfo mi = mode_of(flags);
+    if (mi.mode < 0 || (mi.mode == kNaive && mi.had)) return -1;
+    return mi.mode == kNsn ? 2 : 1;
+}
+
+kvq_status kvq_make_signs(uint64_t seed, int32_t head_dim, int8_t* host_out) {
+    if (host_out == nullptr || head_dim < 1) return KVQ_ERR_INVALID_ARG;
+    uint64_t state = seed;
+    for (int32_t c = 0; c < head_dim; ++c) {
+        // SplitMix64 step (Steele, Lea & Flood 2014)
+        state += 0x9E3779B97F4A7C15ull;
+        uint64_t z = state;
+        z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+        z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+        z ^= z >> 31;
+        host_out[c] = (z >> 63) ? int8_t(-1) : int8_t(1);
+    }
+    return KVQ_OK;
+}
+
+kvq_status kvq_quantize_block(const kvq_config* cfg, kvq_cache* cache, const uint16_t* k, const uint16_t* v,
+                              int64_t t0, int64_t ntok, void* stream) {
+    ModeInfo mi;
+    kvq_status s = check_cfg(cfg, &mi);
+    if (s != KVQ_OK) return s;
+    if ((s = check_cache(cfg, mi, cache)) != KVQ_OK) return s;
+    if (!ok_ptr(k) || !ok_ptr(v)) return KVQ_ERR_INVALID_ARG;
+    if (t0 < 0 || ntok <= 0 || t0 % kT != 0 || ntok % kT != 0) return KVQ_ERR_INVALID_ARG;
+    if (t0 + ntok > cache->capacity) return KVQ_ERR_CAPACITY;
+    const int64_t held0 = (cache->len / kT) * kT;
+    if (cache->len % kT != 0 && t0 + ntok > held0) return KVQ_ERR_INVALID_ARG;
+    const int bh = cache->batch * cache->kv_heads;
+    if ((uint64_t)bh * (uint64_t)ntok >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
+    QuantLaunch L;
+    L.a = quant_args(cfg, cache);
+    L.a.ntok = (int)ntok;
+    L.a.blk0 = (int)(t0 / kT);
+    L.k = k;
+    L.v = v;
+    L.bh = bh;
+    L.nblk = (int)(ntok / kT);
+    L.st = static_cast<cudaStream_t>(stream);
+    if ((s = dispatch(cfg->head_dim, cfg->bits, mi, L)) != KVQ_OK) return s;
+    if (t0 + ntok > cache->len) cache->len = t0 + ntok;
+    return KVQ_OK;
+}
+
+kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache, const uint16_t* k_new, const uint16_t* v_new,
+                            void* stream) {
+    ModeInfo mi;
+    kvq_status s = check_cfg(cfg, &mi);
+    if (s != KVQ_OK) return s;
+    if ((s = check_cache(cfg, mi, cache)) != KVQ_OK) return s;
+    if (!ok_ptr(k_new) || !ok_ptr(v_new)) return KVQ_ERR_INVALID_ARG;
+    if (cache->len + 1 > cache->capacity) return KVQ_ERR_CAPACITY;
+    AppendLaunch L;
+    L.a.q = quant_args(cfg, cache);
+    for (int i = 0; i < 2; ++i) L.a.resid[i] = reinterpret_cast<__half*>(cache->resid[i]);
+    L.a.x_new[0] = reinterpret_cast<const __half*>(k_new);
+    L.a.x_new[1] = reinterpret_cast<const __half*>(v_new);
+    L.a.slot = (int)(cache->len % kT);
+    L.a.blk = (int)(cache->len / kT);
+    L.bh = cache->batch * cache->kv_heads;
+    L.st = static_cast<cudaStream_t>(stream);
+    if ((s = dispatch(cfg->head_dim, cfg->bits, mi, L)) != KVQ_OK) return s;
+    cache->len += 1;
+    return KVQ_OK;
+}
+
+size_t kvq_decode_workspace_bytes(const kvq_config* cfg, const kvq_cache* cache, int32_t q_heads) {
+    ModeInfo mi;
+    if (check_cfg(cfg, &mi) != KVQ_OK || check_cache(cfg, mi, cache) != KVQ_OK) return 0;
+    if (q_heads < cache->kv_heads || q_heads % cache->kv_heads != 0) return 0;
+    const int G = q_heads / cache->kv_heads;
+    if (G > kGMax) return 0;
+    const size_t bh = (size_t)cache->batch * cache->kv_heads;
+    return bh * (size_t)decode_splits(cache) * (size_t)G * (2 + 2 * (size_t)cfg->head_dim) * sizeof(float);
+}
+
+kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, const uint16_t* q, int32_t q_heads,
+                                float scale, float* out, void* ws, size_t ws_bytes, void* stream) {
+    ModeInfo mi;
+    kvq_status s = check_cfg(cfg, &mi);
+    if (s != KVQ_OK) return s;
+    if ((s = check_cache(cfg, mi, cache)) != KVQ_OK) return s;
+    if (!ok_ptr(q) || !ok_ptr(out)) return KVQ_ERR_INVALID_ARG;
+    if (q_heads < cache->kv_heads || q_heads % cache->kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+    const int G = q_heads / cache->kv_heads;
+    if (G > kGMax) return KVQ_ERR_UNSUPPORTED;
+    const size_t need = kvq_decode_workspace_bytes(cfg, cache, q_heads);
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < need) return KVQ_ERR_WORKSPACE;
+    DecodeLaunch L;
+    for (int i = 0; i < 2; ++i) {
+        L.a.codes[i] = cache->codes[i];
+        L.a.tok[i] = reinterpret_cast<const __half*>(cache->tok[i]);
+        L.a.chan[i] = reinterpret_cast<const __half*>(cache->chan[i]);
+        L.a.off[i] = reinterpret_cast<const __half*>(cache->off[i]);
+        L.a.resid[i] = reinterpret_cast<const __half*>(cache->resid[i]);
+    }
+    L.a.q = reinterpret_cast<const __half*>(q);
+    L.a.out = out;
+    L.a.part = static_cast<float*>(ws);
+    L.a.signs = cfg->signs;
+    L.a.H = cache->kv_heads;
+    L.a.G = G;
+    L.a.cap = cache->capacity;
+    L.a.nbq = (int)(cache->len / kT);
+    L.a.rlen = (int)(cache->len % kT);
+    L.a.nsplit = decode_splits(cache);
+    const int nbq1 = L.a.nbq > 0 ? L.a.nbq : 1;
+    L.a.bps = (nbq1 + L.a.nsplit - 1) / L.a.nsplit;
+    L.a.scale = scale > 0.0f ? scale : rsqd_of(cfg->head_dim);
+    L.a.rsqd = rsqd_of(cfg->head_dim);
+    L.a.sqd = sqd_of(cfg->head_dim);
+    L.bh = cache->batch * cache->kv_heads;
+    L.st = static_cast<cudaStream_t>(stream);
+    return dispatch(cfg->head_dim, cfg->bits, mi, L);
+}
+
+kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t tensor, int64_t t0, int64_t ntok,
+                          float* out, void* stream) {
+    ModeInfo mi;
+    kvq_status s = check_cfg(cfg, &mi);
+    if (s != KVQ_OK) return s;
+    if ((s = check_cache(cfg, mi, cache)) != KVQ_OK) return s;
+    if (tensor != 0 && tensor != 1) return KVQ_ERR_INVALID_ARG;
+    if (!ok_ptr(out)) return KVQ_ERR_INVALID_ARG;
+    if (t0 < 0 || ntok <= 0 || t0 % kT != 0 || ntok % kT != 0) return KVQ_ERR_INVALID_ARG;
+    if (t0 + ntok > (cache->len / kT) * kT) return KVQ_ERR_INVALID_ARG;
+    DequantLaunch L;
+    L.a.codes = cache->codes[tensor];
+    L.a.tok = reinterpret_cast<const __half*>(cache->tok[tensor]);
+    L.a.chan = reinterpret_cast<const __half*>(cache->chan[tensor]);
+    L.a.off = reinterpret_cast<const __half*>(cache->off[tensor]);
+    L.a.signs = cfg->signs;
+    L.a.out = out;
+    L.a.cap = cache->capacity;
+    L.a.ntok = (int)ntok;
+    L.a.blk0 = (int)(t0 / kT);
+    L.a.rsqd = rsqd_of(cfg->head_dim);
+    L.a.sqd = sqd_of(cfg->head_dim);
+    L.bh = cache->batch * cache->kv_heads;
+    L.nblk = (int)(ntok / kT);
+    L.st = static_cast<cudaStream_t>(stream);
+    return dispatch(cfg->head_dim, cfg->bits, mi, L);
+}
+
+kvq_status kvq_read_device_errors(uint32_t* host_out, int32_t clear) {
+    if (host_out == nullptr) return KVQ_ERR_INVALID_ARG;
+    if (cudaMemcpyFromSymbol(host_out, g_error_word, sizeof(uint32_t)) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (clear) {
+        const uint32_t zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(uint32_t)) != cudaSuccess) return KVQ_ERR_CUDA;
+    }
+    return KVQ_OK;
+}
+
+const char* kvq_status_string(kvq_status status) {
+    switch (status) {
+        case KVQ_OK: return "ok";
+        case KVQ_ERR_INVALID_ARG: return "invalid argument";
+        case KVQ_ERR_UNSUPPORTED: return "unsupported head_dim, bits or flag set";
+        case KVQ_ERR_CAPACITY: return "cache capacity exceeded";
+        case KVQ_ERR_WORKSPACE: return "decode workspace missing or too small";
+        case KVQ_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,250 @@
+// kvq_quant.cuh -- block quantizer, residual append/flush and dequantizer
+// kernels (sm_100a).  Included once, by kvq_api.cu.
+#pragma once
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+
+struct QuantArgs {
+    // per tensor (0 = K, 1 = V); layouts as in kvq.h
+    uint8_t* codes[2];
+    __half* tok[2];
+    __half* chan[2];
+    __half* off[2];
+    const int8_t* signs;
+    int H;           // kv heads
+    int cap;         // cache capacity (tokens)
+    int ntok;        // tokens in this call (multiple of 128)
+    int blk0;        // first destination block
+    float rsqd, sqd; // (float)(1/sqrt(d)), (float)sqrt(d)
+};
+
+// The fp16 input tile and (NSN only) the fp32 transpose buffer share the
+// first region.
+template <int D, int MODE>
+__host__ __device__ constexpr int quant_region_bytes() {
+    return MODE == kNsn ? kT * D * 4 : kT * D * 2;
+}
+
+template <int D, int MODE>
+__host__ __device__ constexpr int quant_smem_bytes() {
+    // 1024 B alignment slack + region + vec + wmax + sgn + mbarrier
+    return 1024 + quant_region_bytes<D, MODE>() + D * 4 + 4 * D * 4 + D * 4 + 64;
+}
+
+template <int D, int MODE>
+__device__ __forceinline__ QuantSmem<D> carve_quant_smem(uint8_t* base, uint64_t*& bar, uint8_t*& tile) {
+    uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023));
+    QuantSmem<D> sm;
+    tile = p;
+    sm.red = reinterpret_cast<float*>(p);
+    p += quant_region_bytes<D, MODE>();
+    sm.vec = reinterpret_cast<float*>(p);
+    p += D * 4;
+    sm.wmax = reinterpret_cast<uint32_t*>(p);
+    p += 4 * D * 4;
+    sm.sgn = reinterpret_cast<uint32_t*>(p);
+    p += D * 4;
+    bar = reinterpret_cast<uint64_t*>(p);
+    return sm;
+}
+
+template <int D, int BITS, int MODE, bool HAD>
+__device__ __forceinline__ QuantOut quant_out(const QuantArgs& a, int tensor, int bh, int blk) {
+    using L = RowLayout<D, BITS>;
+    const int ntk = (MODE == kNsn) ? 2 : 1;
+    const int nb = a.cap / kT;
+    QuantOut o;
+    // select with ternaries: a runtime index into the parameter arrays would
+    // copy them to local memory
+    const bool v = tensor != 0;
+    o.codes = (v ? a.codes[1] : a.codes[0]) + ((size_t)bh * a.cap + (size_t)blk * kT) * L::kBytes;
+    o.tok = (v ? a.tok[1] : a.tok[0]) + ((size_t)bh * a.cap + (size_t)blk * kT) * ntk;
+    o.chan = (MODE != kNaive) ? (v ? a.chan[1] : a.chan[0]) + ((size_t)bh * nb + blk) * D : nullptr;
+    o.off = (MODE == kNsn) ? (v ? a.off[1] : a.off[0]) + ((size_t)bh * nb + blk) * D : nullptr;
+    return o;
+}
+
+template <int D, bool HAD>
+__device__ __forceinline__ void load_signs(const QuantArgs& a, const QuantSmem<D>& sm, int t) {
+    if constexpr (HAD) {
+        if (t < D) sm.sgn[t] = (a.signs != nullptr && a.signs[t] < 0) ? 0x80000000u : 0u;
+    }
+}
+
+// One CTA = one 128-token block of one (tensor, batch, head).  grid:
+// x = block within the call, y = batch * H + head, z = tensor.  The tile is
+// brought in by TMA as 64-channel boxes with 128-byte swizzle, so that each
+// thread can then read its own token row from shared memory without bank
+// conflicts (chunk c of row t sits at chunk c ^ (t & 7)).
+template <int D, int BITS, int MODE, bool HAD>
+__global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ CUtensorMap map_k,
+                                                       const __grid_constant__ CUtensorMap map_v, QuantArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const int t = threadIdx.x;
+    const int blk = blockIdx.x, bh = blockIdx.y, tensor = blockIdx.z;
+    uint64_t* bar;
+    uint8_t* tile;
+    QuantSmem<D> sm = carve_quant_smem<D, MODE>(smem_raw, bar, tile);
+    constexpr uint32_t kTileBytes = kT * D * 2;
+
+    if (t == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (t == 0) {
+        mbar_expect_tx(bar, kTileBytes);
+        const int row0 = bh * a.ntok + blk * kT;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+            if (tensor == 0) tma_load_2d(tile + h * (kT * 128), &map_k, h * 64, row0, bar);
+            else tma_load_2d(tile + h * (kT * 128), &map_v, h * 64, row0, bar);
+        }
+    }
+    load_signs<D, HAD>(a, sm, t);
+    if (!mbar_wait(bar, 0, 1u << 24)) {
+        if (t == 0) report_error(kErrTmaTimeout);
+        // wait (bounded) for the copy in flight before the CTA's smem is released
+        mbar_wait(bar, 0, 1u << 24);
+        return;
+    }
+
+    float v[D];
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h) {
+        const uint8_t* rowp = tile + h * (kT * 128) + t * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(rowp + ((c ^ (t & 7)) << 4));
+            const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __half22float2(hp[i]);
+                v[h * 64 + c * 8 + 2 * i] = f.x;
+                v[h * 64 + c * 8 + 2 * i + 1] = f.y;
+            }
+        }
+    }
+    __syncthreads();  // the tile buffer is reused as the transpose buffer
+
+    const QuantOut out = quant_out<D, BITS, MODE, HAD>(a, tensor, bh, a.blk0 + blk);
+    quantize_rows<D, BITS, MODE, HAD>(v, t, sm, out, a.rsqd, a.sqd);
+}
+
+struct AppendArgs {
+    QuantArgs q;
+    __half* resid[2];
+    const __half* x_new[2];  // [B*H][D]
+    int slot;                // residual slot of the new token
+    int blk;                 // destination block when the slot is the last one
+};
+
+// One CTA per (batch*head, tensor).  The new token goes to its residual slot;
+// when that slot is the block's last, the CTA instead quantizes the 127 held
+// tokens plus the new one into block `blk` (same arithmetic as
+// quantize_kernel).
+template <int D, int BITS, int MODE, bool HAD>
+__global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
+    const int t = threadIdx.x;
+    const int bh = blockIdx.x, tensor = blockIdx.y;
+    const __half* xn = (tensor ? a.x_new[1] : a.x_new[0]) + (size_t)bh * D;
+    __half* res = (tensor ? a.resid[1] : a.resid[0]) + (size_t)bh * kT * D;
+    if (a.slot < kT - 1) {
+        if (t < D / 8)
+            reinterpret_cast<uint4*>(res + (size_t)a.slot * D)[t] = reinterpret_cast<const uint4*>(xn)[t];
+        return;
+    }
+    extern __shared__ uint8_t smem_raw[];
+    uint64_t* bar;
+    uint8_t* tile;
+    QuantSmem<D> sm = carve_quant_smem<D, MODE>(smem_raw, bar, tile);
+    load_signs<D, HAD>(a.q, sm, t);
+    const __half* src = (t == kT - 1) ? xn : res + (size_t)t * D;
+    float v[D];
+#pragma unroll
+    for (int k = 0; k < D / 8; ++k) {
+        const uint4 raw = reinterpret_cast<const uint4*>(src)[k];
+        const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(hp[i]);
+            v[8 * k + 2 * i] = f.x;
+            v[8 * k + 2 * i + 1] = f.y;
+        }
+    }
+    __syncthreads();
+    const QuantOut out = quant_out<D, BITS, MODE, HAD>(a.q, tensor, bh, a.blk);
+    quantize_rows<D, BITS, MODE, HAD>(v, t, sm, out, a.q.rsqd, a.q.sqd);
+}
+
+struct DequantArgs {
+    const uint8_t* codes;
+    const __half* tok;
+    const __half* chan;
+    const __half* off;
+    const int8_t* signs;
+    float* out;      // [B*H][ntok][D]
+    int cap, ntok, blk0;
+    float rsqd, sqd;
+};
+
+// One CTA = one block of one (batch, head); thread t rebuilds token t:
+//   w = q * sigma; nsep x = n * w, or s (.) (H w * (n rsqd)) under HADAMARD;
+//   naive x = w; NSN x = s1 * (b + o) with b = w * (s2 sqd), or
+//   s (.) (H w * s2) under HADAMARD.
+template <int D, int BITS, int MODE, bool HAD>
+__global__ void __launch_bounds__(128) dequantize_kernel(DequantArgs a) {
+    using L = RowLayout<D, BITS>;
+    const int t = threadIdx.x;
+    const int blk = a.blk0 + blockIdx.x, bh = blockIdx.y;
+    const int nb = a.cap / kT;
+    const int ntk = (MODE == kNsn) ? 2 : 1;
+    __shared__ float s_sig[D], s_off[D];
+    __shared__ uint32_t s_sgn[D];
+    if (t < D) {
+        if (MODE != kNaive) s_sig[t] = __half2float(a.chan[((size_t)bh * nb + blk) * D + t]);
+        if (MODE == kNsn) s_off[t] = __half2float(a.off[((size_t)bh * nb + blk) * D + t]);
+        s_sgn[t] = (HAD && a.signs != nullptr && a.signs[t] < 0) ? 0x80000000u : 0u;
+    }
+    __syncthreads();
+    const size_t tok_idx = (size_t)bh * a.cap + (size_t)blk * kT + t;
+    uint32_t w32[L::kWords];
+    load_words<L::kWords>(a.codes + tok_idx * L::kBytes, w32);
+    const __half* tp = a.tok + tok_idx * ntk;
+    float w[D];
+    const float tsig = (MODE == kNaive) ? __half2float(tp[0]) : 0.0f;
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+        const float q = (float)((int)code_at<D, BITS>(w32, c) - L::kOff);
+        w[c] = __fmul_rn(q, (MODE == kNaive) ? tsig : s_sig[c]);
+    }
+    if constexpr (HAD) fwht_reg<D>(w);
+    float* o = a.out + ((size_t)bh * a.ntok + (size_t)blockIdx.x * kT + t) * D;
+    if constexpr (MODE == kNsn) {
+        const float s1 = __half2float(tp[0]), s2 = __half2float(tp[1]);
+        const float kb = HAD ? s2 : __fmul_rn(s2, a.sqd);
+#pragma unroll
+        for (int c = 0; c < D; ++c) {
+            float b = __fmul_rn(w[c], kb);
+            if (HAD) b = __uint_as_float(__float_as_uint(b) ^ s_sgn[c]);
+            w[c] = __fmul_rn(s1, __fadd_rn(b, s_off[c]));
+        }
+    } else if constexpr (MODE == kNsep) {
+        const float n = __half2float(tp[0]);
+        if constexpr (HAD) {
+            const float kd = __fmul_rn(n, a.rsqd);
+#pragma unroll
+            for (int c = 0; c < D; ++c) w[c] = __uint_as_float(__float_as_uint(__fmul_rn(w[c], kd)) ^ s_sgn[c]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < D; ++c) w[c] = __fmul_rn(n, w[c]);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k)
+        reinterpret_cast<float4*>(o)[k] = make_float4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+}
+
+}  // namespace kvq

@@ -1,0 +1,116 @@
+"""Helpers shared by the GPU parity tests: run the same seeded inputs through
+the CUDA library (via the ctypes binding) and through the CPU oracle, and
+compare the results."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from kv_cache_bit_b200 import synth
+from tests.modes import f16bits, oracle_cfg
+
+T = 128
+
+
+def gpu_cfg(mode: str, d: int, bits: int):
+    from kv_cache_bit_b200 import kvq
+    names, seeded = synth.MODES[mode]
+    flags = 0
+    for n in names:
+        flags |= getattr(kvq, n)
+    signs = kvq.kvq_make_signs(synth.SIGN_SEED, d) if seeded else None
+    return kvq.Config(d, bits, flags, signs)
+
+
+def to_dev(a: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host16(t) -> np.ndarray:
+    """int16 device tensor holding fp16 bits -> uint16 numpy."""
+    return t.cpu().numpy().view(np.uint16)
+
+
+def gpu_prefill(mode, d, bits, K, V, cap=None, ntok=None):
+    """Quantize K, V (float16 [B, H, S, d]) into a fresh GPU cache."""
+    import torch
+    from kv_cache_bit_b200 import kvq
+    B, H, S, _ = K.shape
+    ntok = S if ntok is None else ntok
+    cfg = gpu_cfg(mode, d, bits)
+    cache = kvq.KVCache.allocate(cfg, B, H, cap or S)
+    if ntok:
+        kd = to_dev(f16bits(K[:, :, :ntok]).view(np.int16))
+        vd = to_dev(f16bits(V[:, :, :ntok]).view(np.int16))
+        kvq.kvq_quantize_block(cfg, cache, kd, vd, 0, ntok)
+    torch.cuda.synchronize()
+    return cfg, cache
+
+
+def oracle_prefill(mode, d, bits, K, V, cap=None, ntok=None, threads=8):
+    B, H, S, _ = K.shape
+    ntok = S if ntok is None else ntok
+    cfg = oracle_cfg(mode, d, bits)
+    ck = oracle.empty_cache(cfg, B, H, cap or S)
+    cv = oracle.empty_cache(cfg, B, H, cap or S)
+    if ntok:
+        oracle.quantize_into(cfg, f16bits(K[:, :, :ntok]), ck, 0, threads)
+        oracle.quantize_into(cfg, f16bits(V[:, :, :ntok]), cv, 0, threads)
+    return cfg, ck, cv
+
+
+def fp16_ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> int:
+    """Largest distance in fp16 ulps between two arrays of fp16 bit patterns."""
+    def key(x):
+        x = x.astype(np.int32)
+        return np.where(x & 0x8000, -(x & 0x7FFF), x)
+    if a_bits.size == 0:
+        return 0
+    return int(np.max(np.abs(key(a_bits) - key(b_bits))))
+
+
+def compare_cache(gcache, ck, cv, d, bits, nq, bh_slice=slice(None)):
+    """Codes bit-exact, side parameters within 1 fp16 ulp.  Returns a dict of
+    mismatch counts (codes that differ must be neighbours; each one counts as
+    a half-point case)."""
+    rb = oracle.row_bytes(d, bits)
+    res = {"code_mismatch": 0, "tok_ulp": 0, "chan_ulp": 0, "off_ulp": 0, "codes": 0}
+    nb = nq // T
+    for i, oc in enumerate((ck, cv)):
+        g_codes = gcache.codes[i].cpu().numpy()[bh_slice][:, :, :nq]
+        o_codes = oc["codes"][:, :, :nq]
+        if not np.array_equal(g_codes, o_codes):
+            gq, _ = oracle.unpack_rows(g_codes.reshape(-1, rb), d, bits)
+            oq, _ = oracle.unpack_rows(o_codes.reshape(-1, rb), d, bits)
+            diff = gq.astype(int) - oq.astype(int)
+            assert np.abs(diff).max() <= 1, "codes differ by more than one step"
+            res["code_mismatch"] += int(np.count_nonzero(diff))
+        res["codes"] += o_codes.size * 8 // bits
+        res["tok_ulp"] = max(res["tok_ulp"], fp16_ulp_diff(host16(gcache.tok[i])[bh_slice][:, :, :nq],
+                                                           oc["tok"][:, :, :nq]))
+        if oc["chan"] is not None:
+            res["chan_ulp"] = max(res["chan_ulp"], fp16_ulp_diff(host16(gcache.chan[i])[bh_slice][:, :, :nb],
+                                                                 oc["chan"][:, :, :nb]))
+        if oc["off"] is not None:
+            res["off_ulp"] = max(res["off_ulp"], fp16_ulp_diff(host16(gcache.off[i])[bh_slice][:, :, :nb],
+                                                               oc["off"][:, :, :nb]))
+    return res
+
+
+def assert_cache_parity(res, max_half_point_frac=1e-5):
+    assert res["tok_ulp"] <= 1 and res["chan_ulp"] <= 1 and res["off_ulp"] <= 1, res
+    assert res["code_mismatch"] <= max(1, int(max_half_point_frac * res["codes"])), res
+
+
+def gpu_decode(cfg, cache, q16: np.ndarray, scale: float = 0.0):
+    import torch
+    from kv_cache_bit_b200 import kvq
+    B, Hq, d = q16.shape
+    qd = to_dev(f16bits(q16).view(np.int16))
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device="cuda")
+    nbytes = kvq.kvq_decode_workspace_bytes(cfg, cache, Hq)
+    ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device="cuda")
+    kvq.kvq_decode_attention(cfg, cache, qd, Hq, scale, out, ws, nbytes)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
