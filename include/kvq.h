@@ -199,6 +199,31 @@ kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t
                           int64_t t0, int64_t ntok, float* out, void* stream);
 
 /*
+ * Decode attention that allocates nothing and needs no caller workspace.
+ * The pages have no counterpart to this call; it exists for callers that are
+ * handed only their input and output buffers and cannot allocate device
+ * memory: an operator plugin inside an inference engine that plans all
+ * device memory ahead of time, or code on a latency-critical path where
+ * cudaMalloc would synchronize the device.
+ * Same arguments, results and errors as kvq_decode_attention, minus the
+ * workspace.  The split-K partial results go to a scratch array of
+ * KVQ_NOALLOC_SCRATCH_BYTES (8 MiB) that the library holds in device memory
+ * on every GPU that loads it, until the process exits.  A call whose
+ * workspace need (kvq_decode_workspace_bytes) exceeds that size returns
+ * KVQ_ERR_WORKSPACE before enqueuing anything.
+ * The first call on a device looks up the array's device address on that
+ * device (it must be the current device); make that first call before any
+ * stream capture.  All calls on a device share the one array, which keeps the
+ * last call's contents: calls that overlap in time on the GPU (different
+ * streams, or different host threads) race and corrupt each other's results.
+ * The call never runs cudaMalloc, cudaFree or any allocating routine.
+ */
+#define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache* cache,
+                                        const uint16_t* q, int32_t q_heads, float scale,
+                                        float* out, void* stream);
+
+/*
  * Read (and, if clear != 0, reset) the sticky device error word of the
  * current device: bit 0 = a kernel gave up waiting for a TMA tile, bit 1 = a
  * kernel gave up waiting on a barrier.  Kernels that give up write no

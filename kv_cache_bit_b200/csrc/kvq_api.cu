@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "kvq.h"
 #include "kvq_decode_simple.cuh"
@@ -376,6 +377,59 @@ kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t
     L.nblk = (int)(ntok / kT);
     L.st = static_cast<cudaStream_t>(stream);
     return dispatch(cfg->head_dim, cfg->bits, mi, L);
+}
+
+}  // extern "C"
+
+namespace kvq {
+namespace {
+
+// Scratch of kvq_decode_attention_noalloc: a file-scope device array, so the
+// entry point needs neither an allocation nor a caller workspace.  Host code
+// must not pass `g_noalloc_scratch` itself to a kernel: on the host that name
+// is only a stand-in; the device address comes from cudaGetSymbolAddress.
+__device__ __align__(256) unsigned char g_noalloc_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device.  Returns nullptr if the lookup fails.
+void* noalloc_scratch_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+}  // namespace kvq
+
+extern "C" {
+
+kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache* cache, const uint16_t* q,
+                                        int32_t q_heads, float scale, float* out, void* stream) {
+    ModeInfo mi;
+    kvq_status s = check_cfg(cfg, &mi);
+    if (s != KVQ_OK) return s;
+    if ((s = check_cache(cfg, mi, cache)) != KVQ_OK) return s;
+    if (!ok_ptr(q) || !ok_ptr(out)) return KVQ_ERR_INVALID_ARG;
+    if (q_heads < cache->kv_heads || q_heads % cache->kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+    if (q_heads / cache->kv_heads > kGMax) return KVQ_ERR_UNSUPPORTED;
+    // sizes are checked before any CUDA call
+    const size_t need = kvq_decode_workspace_bytes(cfg, cache, q_heads);
+    if (need == 0 || need > (size_t)KVQ_NOALLOC_SCRATCH_BYTES) return KVQ_ERR_WORKSPACE;
+    void* ws = noalloc_scratch_ptr();
+    if (ws == nullptr) return KVQ_ERR_CUDA;
+    // The split kernel writes every partial it later reads, so no part of the
+    // shared scratch has to start at zero.
+    return kvq_decode_attention(cfg, cache, q, q_heads, scale, out, ws, (size_t)KVQ_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 kvq_status kvq_read_device_errors(uint32_t* host_out, int32_t clear) {

@@ -22,7 +22,8 @@ NORM_SEP, PER_CHANNEL, NSN, HADAMARD = KVQ_NORM_SEP, KVQ_PER_CHANNEL, KVQ_NSN, K
 BLOCK_TOKENS = 128
 
 EXPORTS = ["kvq_row_bytes", "kvq_tok_params", "kvq_make_signs", "kvq_quantize_block", "kvq_append_token",
-           "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_dequantize", "kvq_read_device_errors",
+           "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_dequantize",
+           "kvq_read_device_errors",
            "kvq_status_string"]
 
 
@@ -59,6 +60,9 @@ def _load():
     L.kvq_decode_attention.restype = ctypes.c_int
     L.kvq_decode_attention.argtypes = [ctypes.POINTER(kvq_config), ctypes.POINTER(kvq_cache), P, ctypes.c_int32,
                                        ctypes.c_float, P, P, ctypes.c_size_t, P]
+    L.kvq_decode_attention_noalloc.restype = ctypes.c_int
+    L.kvq_decode_attention_noalloc.argtypes = [ctypes.POINTER(kvq_config), ctypes.POINTER(kvq_cache), P,
+                                               ctypes.c_int32, ctypes.c_float, P, P]
     L.kvq_dequantize.restype = ctypes.c_int
     L.kvq_dequantize.argtypes = [ctypes.POINTER(kvq_config), ctypes.POINTER(kvq_cache), ctypes.c_int32,
                                  ctypes.c_int64, ctypes.c_int64, P, P]
@@ -134,6 +138,17 @@ def kvq_decode_attention(cfg: "Config", cache: "KVCache", q, q_heads: int, scale
                          stream=None):
     _check(lib.kvq_decode_attention(ctypes.byref(cfg.c), ctypes.byref(cache.c), _ptr(q), q_heads, scale,
                                     _ptr(out), _ptr(ws), ws_bytes, _stream(stream)), "kvq_decode_attention")
+
+
+def kvq_decode_attention_noalloc(cfg: "Config", cache: "KVCache", q, q_heads: int, scale: float, out,
+                                 stream=None):
+    """Decode attention with the library's own fixed device scratch (no
+    workspace argument, no allocation); see include/kvq.h."""
+    _check(lib.kvq_decode_attention_noalloc(ctypes.byref(cfg.c), ctypes.byref(cache.c), _ptr(q), q_heads, scale,
+                                            _ptr(out), _stream(stream)), "kvq_decode_attention_noalloc")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 def kvq_dequantize(cfg: "Config", cache: "KVCache", tensor: int, t0: int, ntok: int, out, stream=None):
