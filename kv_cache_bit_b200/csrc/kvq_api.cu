@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "kvq.h"
+#include "kvq_decode_mma.cuh"
 #include "kvq_decode_simple.cuh"
 #include "kvq_quant.cuh"
 
@@ -197,27 +198,49 @@ struct DequantLaunch {
     }
 };
 
+template <int D, int BITS, int MODE, bool HAD, int GP>
+kvq_status launch_decode_mma(DecodeArgs a, int bh, cudaStream_t st) {
+    constexpr int smem = mma_smem_bytes<D, BITS, MODE>();
+    static bool attr = false;
+    if (!attr) attr = set_smem(decode_mma_kernel<D, BITS, MODE, HAD, GP>, smem);
+    if (!attr) return KVQ_ERR_CUDA;
+    // every warp of a CTA gets the same number of blocks
+    a.bps = (a.bps + kNW - 1) / kNW * kNW;
+    decode_mma_kernel<D, BITS, MODE, HAD, GP><<<dim3(a.nsplit, bh), kNW * 32, smem, st>>>(a);
+    kvq_status s = launch_status();
+    if (s != KVQ_OK) return s;
+    decode_combine_kernel<D, HAD><<<bh, kT, 0, st>>>(a);
+    return launch_status();
+}
+
 struct DecodeLaunch {
     DecodeArgs a;
     int bh;
     cudaStream_t st;
     template <int D, int BITS, int MODE, bool HAD>
     kvq_status run() {
-        decode_split_kernel<D, BITS, MODE, HAD><<<dim3(a.nsplit, bh), kT, 0, st>>>(a);
-        kvq_status s = launch_status();
-        if (s != KVQ_OK) return s;
-        decode_combine_kernel<D, HAD><<<bh, kT, 0, st>>>(a);
-        return launch_status();
+        if constexpr (D == 128) {
+            // tensor-core path
+            if (a.G <= 4) return launch_decode_mma<D, BITS, MODE, HAD, 4>(a, bh, st);
+            return launch_decode_mma<D, BITS, MODE, HAD, 8>(a, bh, st);
+        } else {
+            decode_split_kernel<D, BITS, MODE, HAD><<<dim3(a.nsplit, bh), kT, 0, st>>>(a);
+            kvq_status s = launch_status();
+            if (s != KVQ_OK) return s;
+            decode_combine_kernel<D, HAD><<<bh, kT, 0, st>>>(a);
+            return launch_status();
+        }
     }
 };
 
-// Splits of the sequence for decode: enough CTAs to cover the GPU twice,
-// fixed per cache shape so the workspace size does not depend on len.
+// Splits of the sequence for decode: about six waves of CTAs on 148 SMs
+// (two resident per SM) with at least 8 blocks per split, fixed per cache
+// shape so that the workspace size does not depend on len.
 int decode_splits(const kvq_cache* c) {
     const int bh = c->batch * c->kv_heads;
     const int nb = c->capacity / kT;
-    int ns = (296 + bh - 1) / bh;
-    if (ns > nb) ns = nb;
+    int ns = (6 * 296 + bh - 1) / bh;
+    if (ns > nb / 8) ns = nb / 8;
     if (ns < 1) ns = 1;
     return ns;
 }
