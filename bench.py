@@ -202,6 +202,11 @@ def run_ours(args, rank: int, world: int):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     w = synth.WORKLOADS[WORKLOAD].scaled(seed=rank)
+    if args.batch:
+        w = w.scaled(B=args.batch)
+    if args.stream is not None:
+        w = w.scaled(stream=args.stream)
+    BITS = args.bits
     flags = flags_of(MODE)
     G = w.Hq // w.Hkv
     n_stream = w.stream
@@ -243,7 +248,7 @@ def run_ours(args, rank: int, world: int):
     step_bytes = accounting.quantize_bytes(w.d, BITS, flags, w.B, w.Hkv, w.S)
     dec_bytes = []
     for i in range(n_stream):
-        length = w.S + i + 1
+        length = w.S + i + 1  # the decode after append i sees this many tokens
         step_bytes += accounting.append_bytes(w.d, BITS, flags, w.B, w.Hkv, flush=(length % 128 == 0))
         db = accounting.decode_bytes(w.d, BITS, flags, w.B, w.Hkv, w.Hq, length)
         dec_bytes.append(db)
@@ -293,7 +298,8 @@ def run_ours(args, rank: int, world: int):
     value = world * step_bytes / (ms / 1e3) / 1e9
 
     # end to end through the public calls, host buffers, copies inside the region
-    e2e = run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, dev, step_bytes, world)
+    e2e = None if args.no_e2e else run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, dev,
+                                           step_bytes, world)
 
     if rank != 0:
         return 0
@@ -385,6 +391,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--batch", type=int, default=None, help="override the batch size (smaller profiling cases)")
+    ap.add_argument("--stream", type=int, default=None, help="override the number of streamed decode steps")
+    ap.add_argument("--bits", type=int, default=BITS, choices=[2, 3, 4])
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -288,14 +288,27 @@ __device__ __forceinline__ void mbar_inval(uint64_t* bar) {
 
 // ---------------------------------------------------------------- the kernel
 
-// GP: padded heads per kv head, 4 (G <= 4: one n-tile holds hi and lo of four
-// heads) or 8 (G <= 8: hi and lo n-tiles of eight heads).
+__device__ __forceinline__ uint32_t cvt_h2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// fp32 x -> (hi, lo) fp16 pair with hi = fp16(x), lo = fp16(x - hi); packed
+// with hi in the low half.
+__device__ __forceinline__ uint32_t split_h2(float x) {
+    const __half h = __float2half_rn(x);
+    return cvt_h2(__half2float(h), x - __half2float(h));
+}
+
+// Column layout of every n-tile (8 columns): column 2j + part holds part
+// (0 = hi, 1 = lo) of head 4n + j.  Thread (g, t) of a warp therefore owns
+// head 4n + t of every n-tile in the C fragments and sums its two columns.
 template <int D, int BITS, int MODE, bool HAD, int GP>
 __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "tensor-core decode is built for head dim 128");
     using SL = SlotLayout<D, BITS, MODE>;
-    constexpr int NTS = 2 * GP / 8;       // score n-tiles (1 or 2)
-    constexpr int NCOL = (GP == 4) ? 2 : 2;  // heads held per thread
+    constexpr int NT = GP / 4;  // n-tiles (heads per thread)
     constexpr bool PCH = MODE != kNaive;
     constexpr float kLog2e = 1.4426950408889634f;
     constexpr int QMAX = (1 << (BITS - 1)) - 1;
@@ -310,39 +323,44 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 
     uint8_t* ring = smem_raw;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kNW * kRing * SL::kStride);
-    __shared__ float s_q[kGMax][D];  // queries (original domain)
-    __shared__ float s_qt[kGMax][D]; // queries, rotated domain (== s_q without HADAMARD)
-    __shared__ float s_qscale[kGMax];
+    __shared__ float s_q[GP][D];   // queries (original domain)
+    __shared__ float s_qs[GP][D];  // rotated queries times the head's power-of-two scale
+    __shared__ float s_qscale[GP];
 
-    // ---- prologue: queries, rotation, per-head power-of-two scale
-    for (int i = tid; i < kGMax * D; i += kNW * 32) {
-        const int j = i / D, c = i % D;
-        float qv = 0.0f;
-        if (j < G) qv = __half2float(a.q[((size_t)b * a.H * G + (size_t)h * G + j) * D + c]);
-        s_q[j][c] = qv;
-        s_qt[j][c] = qv;
-    }
     if (tid < kNW * kRing) mbar_init(&bars[tid], 1);
     fence_mbar_init();
-    __syncthreads();
-    if (tid < kGMax) {
-        float r[D];
+    // ---- prologue: each warp rotates heads warp, warp + kNW, ... (lane owns 4 channels)
+    for (int j = warp; j < GP; j += kNW) {
+        float v[4];
 #pragma unroll
-        for (int c = 0; c < D; ++c) r[c] = s_q[tid][c];
-        if constexpr (HAD) {
-#pragma unroll
-            for (int c = 0; c < D; ++c)
-                if (a.signs != nullptr && a.signs[c] < 0) r[c] = -r[c];
-            fwht_reg<D>(r);
-#pragma unroll
-            for (int c = 0; c < D; ++c) s_qt[tid][c] = r[c];
+        for (int k = 0; k < 4; ++k) {
+            const int c = 4 * lane + k;
+            const float qv = (j < G) ? __half2float(a.q[((size_t)b * a.H * G + (size_t)h * G + j) * D + c]) : 0.0f;
+            s_q[j][c] = qv;
+            v[k] = (HAD && a.signs != nullptr && a.signs[c] < 0) ? -qv : qv;
         }
-        float amax = 0.0f;
+        if constexpr (HAD) {
+            float x0 = v[0] + v[1], x1 = v[0] - v[1], x2 = v[2] + v[3], x3 = v[2] - v[3];
+            v[0] = x0 + x2; v[2] = x0 - x2; v[1] = x1 + x3; v[3] = x1 - x3;
 #pragma unroll
-        for (int c = 0; c < D; ++c) amax = fmaxf(amax, fabsf(r[c]));
-        // |q'| <= amax * max(sigma) <= amax / qmax (1 + 2^-10); keep it <= 2^13
+            for (int m = 1; m < 32; m <<= 1) {
+                const bool upper = (lane & m) != 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
+                    v[k] = upper ? (o - v[k]) : (v[k] + o);
+                }
+            }
+        }
+        float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        // |q'| <= amax * max(sigma) <= amax / qmax (1 + 2^-10): keep it below 2^13
         const float bound = PCH ? amax * (1.001f / (float)QMAX) : amax;
-        s_qscale[tid] = bound > 0.0f ? pow2i(13 - ceil_log2(bound)) : 1.0f;
+        const float qsc = bound > 0.0f ? pow2i(13 - ceil_log2(bound)) : 1.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s_qs[j][4 * lane + k] = v[k] * qsc;
+        if (lane == 0) s_qscale[j] = qsc;
     }
     __syncthreads();
 
@@ -368,41 +386,27 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
         if (PCH) bulk_load(slot + SL::kChan, (ten ? a.chan[1] : a.chan[0]) + bi, D * 2, bar);
         if (MODE == kNsn) bulk_load(slot + SL::kOff, (ten ? a.off[1] : a.off[0]) + bi, D * 2, bar);
     };
-    int issued = min(kRing, nunits);  // units issued so far (same value in every lane)
+    int issued = min(kRing, nunits);
     if (lane == 0) {
         for (int u = 0; u < issued; ++u) issue(u);
     }
-    int waited = 0;  // units whose slot phase this warp has seen complete
+    int waited = 0;
 
-    // per-thread persistent state
-    // heads held by this thread in the score / value layouts
-    const int hbase = (GP == 4) ? 2 * (t & 1) : 2 * t;
-    float m_run[NCOL], l_run[NCOL];
+    // ---- persistent per-thread state: heads 4n + t, channels [16g, 16g + 16)
+    float m_run[NT], l_run[NT];
+    float acc[NT][16], acco[NT][16];
 #pragma unroll
-    for (int k = 0; k < NCOL; ++k) { m_run[k] = -INFINITY; l_run[k] = 0.0f; }
-    float acc[NTS][8][4];
+    for (int n = 0; n < NT; ++n) {
+        m_run[n] = -INFINITY;
+        l_run[n] = 0.0f;
 #pragma unroll
-    for (int n = 0; n < NTS; ++n)
+        for (int k = 0; k < 16; ++k) { acc[n][k] = 0.0f; acco[n][k] = 0.0f; }
+    }
+    float kcol[NT];  // 1 / (the head's power-of-two scale)
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[n][i][k] = 0.0f;
-    // NSN mean term: lane owns channels 4*lane .. 4*lane+3 for all heads
-    float acco[GP][4];
-#pragma unroll
-    for (int j = 0; j < GP; ++j)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acco[j][k] = 0.0f;
-    // rotated queries of the score column(s) this thread feeds, at its 32 channels
-    // (GP == 4: column g -> head g & 3, part g >> 2; GP == 8: head g, both parts)
-    const int qhead = (GP == 4) ? (g & 3) : g;
-    const bool qlo = (GP == 4) && (g >= 4);
-    const float* qt_row = &s_qt[qhead][32 * t];
-    const float qsc = s_qscale[qhead];
-    float qsc_col[NCOL];
-#pragma unroll
-    for (int k = 0; k < NCOL; ++k) qsc_col[k] = 1.0f / s_qscale[hbase + k];
-
+    for (int n = 0; n < NT; ++n) kcol[n] = 1.0f / s_qscale[4 * n + t];
+    // the B column this thread feeds in each n-tile: head 4n + g/2, part g%2
+    const bool blo = (g & 1) != 0;
     const float alpha2 = a.scale * kLog2e;
     bool ok = true;
 
@@ -410,101 +414,83 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
         const int uK = 2 * it, uV = 2 * it + 1;
         uint8_t* sk = my_ring + (uK % kRing) * SL::kStride;
         uint8_t* sv = my_ring + (uV % kRing) * SL::kStride;
-        // ---------------- K half
+        // ================= K half
         if (!mbar_wait(&my_bars[uK % kRing], (uK / kRing) & 1, 1u << 26)) { ok = false; break; }
         waited = uK + 1;
-        // B fragments: q' = qt * sigma^K * 2^e, as fp16 hi (and lo) parts
-        uint32_t bq[NTS][16];
+        // B fragments: q' = qs * sigma^K as (hi, lo) fp16 parts
+        uint32_t bq[NT][16];
         {
             const __half* sig = reinterpret_cast<const __half*>(sk + SL::kChan) + 32 * t;
 #pragma unroll
-            for (int p = 0; p < 16; ++p) {
-                const int ca = KUnpack<BITS>::ca(p), cb = KUnpack<BITS>::cb(p);
-                const float fa = qt_row[ca] * (PCH ? __half2float(sig[ca]) : 1.0f) * qsc;
-                const float fb = qt_row[cb] * (PCH ? __half2float(sig[cb]) : 1.0f) * qsc;
-                const __half ha = __float2half_rn(fa), hb = __float2half_rn(fb);
-                const float ra = fa - __half2float(ha), rb = fb - __half2float(hb);
-                if constexpr (GP == 4) {
-                    bq[0][p] = qlo ? pack_h2(ra, rb) : pack_h2(__half2float(ha), __half2float(hb));
-                } else {
-                    bq[0][p] = pack_h2(__half2float(ha), __half2float(hb));
-                    bq[1][p] = pack_h2(ra, rb);
+            for (int n = 0; n < NT; ++n) {
+                const float* qrow = &s_qs[4 * n + (g >> 1)][32 * t];
+#pragma unroll
+                for (int p = 0; p < 16; ++p) {
+                    const int ca = KUnpack<BITS>::ca(p), cb = KUnpack<BITS>::cb(p);
+                    const float fa = qrow[ca] * (PCH ? __half2float(sig[ca]) : 1.0f);
+                    const float fb = qrow[cb] * (PCH ? __half2float(sig[cb]) : 1.0f);
+                    const __half2 hh = __floats2half2_rn(fa, fb);
+                    if (blo) {
+                        const float2 hf = __half22float2(hh);
+                        bq[n][p] = cvt_h2(fa - hf.x, fb - hf.y);
+                    } else {
+                        bq[n][p] = *reinterpret_cast<const uint32_t*>(&hh);
+                    }
                 }
             }
         }
-        // scores for 8 m-tiles of 16 tokens
-        float sc[8][4];
+        // scores -> logits (log2 domain); thread holds tokens 16mt + g (+8)
+        const __half* tk = reinterpret_cast<const __half*>(sk + SL::kTok);
+        float qoK[NT];
+        if constexpr (MODE == kNsn) {
+            const __half* okp = reinterpret_cast<const __half*>(sk + SL::kOff) + 16 * g;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                float s = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) s += s_q[4 * n + t][16 * g + k] * __half2float(okp[k]);
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                qoK[n] = s;
+            }
+        }
+        float lg[NT][8][2];
+        float bmax[NT];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) bmax[n] = -INFINITY;
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-            float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t pa[16], pb[16];
             KUnpack<BITS>::run(sk + SL::kCodes + (16 * mt + g) * SL::kRB, t, pa);
             KUnpack<BITS>::run(sk + SL::kCodes + (16 * mt + g + 8) * SL::kRB, t, pb);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                mma16816(d0, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], bq[0][2 * s], bq[0][2 * s + 1]);
-                if constexpr (NTS == 2)
-                    mma16816(d1, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], bq[1][2 * s], bq[1][2 * s + 1]);
-            }
+            for (int n = 0; n < NT; ++n) {
+                // two independent accumulation chains over the 8 k-steps
+                float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                if constexpr (GP == 4) sc[mt][k] = d0[k] + __shfl_xor_sync(0xffffffffu, d0[k], 2);
-                else sc[mt][k] = d0[k] + d1[k];
-            }
-        }
-        // per-token K factors, logits (log2 domain)
-        const __half* tk = reinterpret_cast<const __half*>(sk + SL::kTok);
-        float qoK[NCOL];
-        if constexpr (MODE == kNsn) {
-            // q . o^K for this thread's heads (lanes own 4 channels each)
-            const __half* ok_ = reinterpret_cast<const __half*>(sk + SL::kOff);
-            float part[GP];
-#pragma unroll
-            for (int j = 0; j < GP; ++j) {
-                float s = 0.0f;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) s += s_q[j][4 * lane + k] * __half2float(ok_[4 * lane + k]);
-                part[j] = s;
-            }
-#pragma unroll
-            for (int j = 0; j < GP; ++j)
-#pragma unroll
-                for (int o = 16; o; o >>= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
-#pragma unroll
-            for (int k = 0; k < NCOL; ++k) {
-                float v = 0.0f;
-#pragma unroll
-                for (int j = 0; j < GP; ++j)
-                    if (j == hbase + k) v = part[j];
-                qoK[k] = v;
-            }
-        }
-        float bmax[NCOL] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int tok = 16 * mt + g + 8 * r;
-                float kap, add = 0.0f;
-                if constexpr (MODE == kNsn) {
-                    const __half2 s12 = reinterpret_cast<const __half2*>(tk)[tok];
-                    const float s1 = __low2float(s12), s2 = __high2float(s12);
-                    kap = s1 * s2 * (HAD ? 1.0f : a.sqd);
-                    add = s1;
-                } else {
-                    kap = __half2float(tk[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                for (int s = 0; s < 8; s += 2) {
+                    mma16816(d0, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], bq[n][2 * s], bq[n][2 * s + 1]);
+                    mma16816(d1, pa[2 * s + 2], pb[2 * s + 2], pa[2 * s + 3], pb[2 * s + 3], bq[n][2 * s + 2],
+                             bq[n][2 * s + 3]);
                 }
 #pragma unroll
-                for (int k = 0; k < NCOL; ++k) {
-                    float lg = sc[mt][2 * r + k] * (kap * qsc_col[k]);
-                    if constexpr (MODE == kNsn) lg += add * qoK[k];
-                    lg *= alpha2;
-                    sc[mt][2 * r + k] = lg;
-                    bmax[k] = fmaxf(bmax[k], lg);
+                for (int r = 0; r < 2; ++r) {
+                    const int tok = 16 * mt + g + 8 * r;
+                    const float sv_ = (d0[2 * r] + d0[2 * r + 1]) + (d1[2 * r] + d1[2 * r + 1]);
+                    float kap, add = 0.0f;
+                    if constexpr (MODE == kNsn) {
+                        const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tk)[tok]);
+                        kap = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
+                        add = s12.x * qoK[n];
+                    } else {
+                        kap = __half2float(tk[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                    }
+                    const float l2 = (sv_ * (kap * kcol[n]) + add) * alpha2;
+                    lg[n][mt][r] = l2;
+                    bmax[n] = fmaxf(bmax[n], l2);
                 }
             }
         }
-        // K slot consumed: reuse it for the unit kRing ahead
         __syncwarp();
         if (uK + kRing < nunits) {
             if (lane == 0) {
@@ -514,106 +500,90 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
             issued = uK + kRing + 1;
         }
 #pragma unroll
-        for (int k = 0; k < NCOL; ++k) {
+        for (int n = 0; n < NT; ++n)
 #pragma unroll
-            for (int o = 4; o < 32; o <<= 1) bmax[k] = fmaxf(bmax[k], __shfl_xor_sync(0xffffffffu, bmax[k], o));
-        }
-        // ---------------- V half
+            for (int o = 4; o < 32; o <<= 1) bmax[n] = fmaxf(bmax[n], __shfl_xor_sync(0xffffffffu, bmax[n], o));
+        // ================= V half
         if (!mbar_wait(&my_bars[uV % kRing], (uV / kRing) & 1, 1u << 26)) { ok = false; break; }
         waited = uV + 1;
         const __half* tv = reinterpret_cast<const __half*>(sv + SL::kTok);
-        // online softmax update
-        float corr[NCOL];
+        // online softmax: rescale when the running max moves
         bool changed = false;
+        float corr[NT];
 #pragma unroll
-        for (int k = 0; k < NCOL; ++k) {
-            const float mn = fmaxf(m_run[k], bmax[k]);
-            corr[k] = fast_exp2(m_run[k] - mn);  // 0 on the first block
-            changed |= (mn != m_run[k]);
-            m_run[k] = mn;
-            l_run[k] *= corr[k];
+        for (int n = 0; n < NT; ++n) {
+            const float mn = fmaxf(m_run[n], bmax[n]);
+            corr[n] = fast_exp2(m_run[n] - mn);
+            changed |= (mn != m_run[n]);
+            m_run[n] = mn;
+            l_run[n] *= corr[n];
         }
         if (__any_sync(0xffffffffu, changed)) {
 #pragma unroll
-            for (int n = 0; n < NTS; ++n)
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) acc[n][i][k] *= corr[k & 1];
-            if constexpr (MODE == kNsn) {
-                // correction of head j lives in lane t = (j / 2) mod 2 (GP 4) or j / 2 (GP 8)
-#pragma unroll
-                for (int j = 0; j < GP; ++j) {
-                    const int src = (GP == 4) ? ((j >> 1) & 1) : (j >> 1);
-                    const float cj = __shfl_sync(0xffffffffu, corr[j & 1], src);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) acco[j][k] *= cj;
+                for (int k = 0; k < 16; ++k) {
+                    acc[n][k] *= corr[n];
+                    if (MODE == kNsn) acco[n][k] *= corr[n];
                 }
-            }
         }
-        // nu per token and the block's power-of-two scale for P'
-        auto nu_of = [&](int tok, float& s1o) -> float {
-            if constexpr (MODE == kNsn) {
-                const __half2 s12 = reinterpret_cast<const __half2*>(tv)[tok];
-                s1o = __low2float(s12);
-                return __low2float(s12) * __high2float(s12) * (HAD ? 1.0f : a.sqd);
-            } else {
-                s1o = 0.0f;
-                return __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
-            }
-        };
-        float numax = 0.0f;
+        // power-of-two scale keeping p * nu * 2^f <= 2^13 in fp16 (p <= 1)
+        float numax;
+        {
+            // lane scans tokens 4 lane .. 4 lane + 3
+            float mx = 0.0f;
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                float s1o;
-                numax = fmaxf(numax, nu_of(16 * mt + g + 8 * r, s1o));
+            for (int k = 0; k < 4; ++k) {
+                const int tok = 4 * lane + k;
+                float v;
+                if constexpr (MODE == kNsn) {
+                    const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
+                    v = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
+                } else {
+                    v = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                }
+                mx = fmaxf(mx, v);
             }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            numax = mx;
         }
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) numax = fmaxf(numax, __shfl_xor_sync(0xffffffffu, numax, o));
         const int fexp = numax > 0.0f ? 13 - ceil_log2(numax) : 0;
         const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
-        // values: P' fragments via movmatrix, V codes transposed
-        float dv[NTS][8][4];
+        float dv[NT][8][4];
 #pragma unroll
-        for (int n = 0; n < NTS; ++n)
+        for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) dv[n][i][k] = 0.0f;
-        float lsum[NCOL] = {0.f, 0.f}, bsum[NCOL] = {0.f, 0.f};
+        float lsum[NT], bsum[NT];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-            uint32_t prow[NTS][2];
+            uint32_t bp[NT][2];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                float pv[NCOL], s1o;
-                const float nus = nu_of(16 * mt + g + 8 * r, s1o) * pscale;
-#pragma unroll
-                for (int k = 0; k < NCOL; ++k) {
-                    const float p = fast_exp2(sc[mt][2 * r + k] - m_run[k]);
-                    lsum[k] += p;
-                    if constexpr (MODE == kNsn) bsum[k] += p * s1o;
-                    pv[k] = p * nus;
-                }
-                const __half h0 = __float2half_rn(pv[0]), h1 = __float2half_rn(pv[1]);
-                const float l0 = pv[0] - __half2float(h0), l1 = pv[1] - __half2float(h1);
-                if constexpr (GP == 4) {
-                    prow[0][r] = (t >= 2) ? pack_h2(l0, l1) : pack_h2(__half2float(h0), __half2float(h1));
+                const int tok = 16 * mt + g + 8 * r;
+                float nu, s1o = 0.0f;
+                if constexpr (MODE == kNsn) {
+                    const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
+                    s1o = s12.x;
+                    nu = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
                 } else {
-                    prow[0][r] = pack_h2(__half2float(h0), __half2float(h1));
-                    prow[1][r] = pack_h2(l0, l1);
+                    nu = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                }
+                nu *= pscale;
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const float p = fast_exp2(lg[n][mt][r] - m_run[n]);
+                    lsum[n] += p;
+                    if constexpr (MODE == kNsn) bsum[n] += p * s1o;
+                    // row tok: (hi, lo) of head 4n + t in columns 2t, 2t + 1
+                    bp[n][r] = movmatrix_t(split_h2(p * nu));
                 }
             }
-            uint32_t bp[NTS][2];
-#pragma unroll
-            for (int n = 0; n < NTS; ++n) {
-                bp[n][0] = movmatrix_t(prow[n][0]);
-                bp[n][1] = movmatrix_t(prow[n][1]);
-            }
-            // V rows of this 16-token tile: (2t, 2t+1) and (2t+8, 2t+9)
             uint32_t va[16], vb[16];
             const uint8_t* vbase = sv + SL::kCodes + (16 * mt) * SL::kRB;
             VUnpack<BITS>::run(vbase + (2 * t) * SL::kRB, vbase + (2 * t + 1) * SL::kRB, g, va);
@@ -621,41 +591,38 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 #pragma unroll
             for (int tc = 0; tc < 8; ++tc) {
 #pragma unroll
-                for (int n = 0; n < NTS; ++n)
+                for (int n = 0; n < NT; ++n)
                     mma16816(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1], bp[n][0], bp[n][1]);
             }
         }
 #pragma unroll
-        for (int k = 0; k < NCOL; ++k) l_run[k] += lsum[k];
-        // block scale: acc[c][col] += dv * sigma^V_c * 2^-fexp
+        for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
+        // block epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f
         {
             const __half* sigv = reinterpret_cast<const __half*>(sv + SL::kChan) + 16 * g;
 #pragma unroll
             for (int tc = 0; tc < 8; ++tc) {
-                const float s0 = (PCH ? __half2float(sigv[2 * tc]) : 1.0f) * pinv;
-                const float s1_ = (PCH ? __half2float(sigv[2 * tc + 1]) : 1.0f) * pinv;
+                float s0 = pinv, s1_ = pinv;
+                if (PCH) {
+                    const float2 sg = __half22float2(reinterpret_cast<const __half2*>(sigv)[tc]);
+                    s0 *= sg.x;
+                    s1_ *= sg.y;
+                }
 #pragma unroll
-                for (int n = 0; n < NTS; ++n) {
-                    acc[n][tc][0] += dv[n][tc][0] * s0;
-                    acc[n][tc][1] += dv[n][tc][1] * s0;
-                    acc[n][tc][2] += dv[n][tc][2] * s1_;
-                    acc[n][tc][3] += dv[n][tc][3] * s1_;
+                for (int n = 0; n < NT; ++n) {
+                    acc[n][2 * tc] += (dv[n][tc][0] + dv[n][tc][1]) * s0;
+                    acc[n][2 * tc + 1] += (dv[n][tc][2] + dv[n][tc][3]) * s1_;
                 }
             }
         }
         if constexpr (MODE == kNsn) {
-            // beta_j = sum over the block of p * s1 (scores of head j live in lanes with t = hbase/2)
+            const __half* ov = reinterpret_cast<const __half*>(sv + SL::kOff) + 16 * g;
 #pragma unroll
-            for (int k = 0; k < NCOL; ++k)
+            for (int n = 0; n < NT; ++n) {
 #pragma unroll
-                for (int o = 4; o < 32; o <<= 1) bsum[k] += __shfl_xor_sync(0xffffffffu, bsum[k], o);
-            const __half* ov = reinterpret_cast<const __half*>(sv + SL::kOff);
+                for (int o = 4; o < 32; o <<= 1) bsum[n] += __shfl_xor_sync(0xffffffffu, bsum[n], o);
 #pragma unroll
-            for (int j = 0; j < GP; ++j) {
-                const int src = (GP == 4) ? ((j >> 1) & 1) : (j >> 1);
-                const float bj = __shfl_sync(0xffffffffu, bsum[j & 1], src);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) acco[j][k] += bj * __half2float(ov[4 * lane + k]);
+                for (int k = 0; k < 16; ++k) acco[n][k] += bsum[n] * __half2float(ov[k]);
             }
         }
         __syncwarp();
@@ -679,45 +646,28 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     }
 
     // ---- merge: warps -> shared memory -> one partial per CTA
-    // reduce l over the 8 row groups; combine hi + lo value columns
 #pragma unroll
-    for (int k = 0; k < NCOL; ++k)
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
-        for (int o = 4; o < 32; o <<= 1) l_run[k] += __shfl_xor_sync(0xffffffffu, l_run[k], o);
-    float accv[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            if constexpr (GP == 4) accv[i][k] = acc[0][i][k] + __shfl_xor_sync(0xffffffffu, acc[0][i][k], 2);
-            else accv[i][k] = acc[0][i][k] + acc[1][i][k];
-        }
+        for (int o = 4; o < 32; o <<= 1) l_run[n] += __shfl_xor_sync(0xffffffffu, l_run[n], o);
     __syncthreads();  // every warp is done with its ring; reuse it for the merge
     float* mw = reinterpret_cast<float*>(smem_raw);   // [kNW][kGMax] running max
     float* lw = mw + kNW * kGMax;                     // [kNW][kGMax] sums
     float* aw = lw + kNW * kGMax;                     // [kNW][kGMax][D] code-term accumulators
     float* ow = aw + kNW * kGMax * D;                 // [kNW][kGMax][D] original-domain accumulators
-    if (g == 0 && (GP == 8 || t < 2)) {
 #pragma unroll
-        for (int k = 0; k < NCOL; ++k) {
-            mw[warp * kGMax + hbase + k] = m_run[k];
-            lw[warp * kGMax + hbase + k] = l_run[k];
+    for (int n = 0; n < NT; ++n) {
+        const int head = 4 * n + t;
+        if (g == 0) {
+            mw[warp * kGMax + head] = m_run[n];
+            lw[warp * kGMax + head] = l_run[n];
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            aw[(warp * kGMax + head) * D + 16 * g + k] = acc[n][k];
+            ow[(warp * kGMax + head) * D + 16 * g + k] = (MODE == kNsn) ? acco[n][k] : 0.0f;
         }
     }
-    if (GP == 8 || t < 2) {
-#pragma unroll
-        for (int tc = 0; tc < 8; ++tc)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int c = 16 * g + 2 * tc + (k >> 1);
-                const int head = hbase + (k & 1);
-                aw[(warp * kGMax + head) * D + c] = accv[tc][k];
-            }
-    }
-#pragma unroll
-    for (int j = 0; j < kGMax; ++j)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) ow[(warp * kGMax + j) * D + 4 * lane + k] = (j < GP) ? acco[j < GP ? j : 0][k] : 0.0f;
     __syncthreads();
 
     // residual tokens (fp16), handled by the last split on CUDA cores
@@ -727,25 +677,36 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     float* rm = rl + kGMax * kT;       // [kGMax] residual max, [kGMax] sum
     if (do_res) {
         const __half* rk = a.resid[0] + (size_t)bh * kT * D;
-        for (int i = tid; i < kGMax * kT; i += kNW * 32) {
-            const int j = i / kT, tr = i % kT;
-            float s = -INFINITY;
-            if (j < G && tr < a.rlen) {
-                s = 0.0f;
-                for (int c = 0; c < D; ++c) s += s_q[j][c] * __half2float(rk[(size_t)tr * D + c]);
-                s *= alpha2;
+        // warp w scores tokens w, w + kNW, ...; lanes split the channels
+        for (int tr = warp; tr < kT; tr += kNW) {
+            float x[4];
+            if (tr < a.rlen) {
+                const float2 x01 = __half22float2(reinterpret_cast<const __half2*>(rk + (size_t)tr * D)[2 * lane]);
+                const float2 x23 = __half22float2(reinterpret_cast<const __half2*>(rk + (size_t)tr * D)[2 * lane + 1]);
+                x[0] = x01.x; x[1] = x01.y; x[2] = x23.x; x[3] = x23.y;
             }
-            rl[i] = s;
+            for (int j = 0; j < G; ++j) {
+                float s = -INFINITY;
+                if (tr < a.rlen) {
+                    s = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) s += s_q[j][4 * lane + k] * x[k];
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                    s *= alpha2;
+                }
+                if (lane == 0) rl[j * kT + tr] = s;
+            }
         }
         __syncthreads();
-        for (int j = warp; j < kGMax; j += kNW) {
+        for (int j = warp; j < G; j += kNW) {
             float mx = -INFINITY;
             for (int i = lane; i < kT; i += 32) mx = fmaxf(mx, rl[j * kT + i]);
 #pragma unroll
             for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             float sm = 0.0f;
             for (int i = lane; i < kT; i += 32) {
-                const float p = (mx == -INFINITY || rl[j * kT + i] == -INFINITY) ? 0.0f : fast_exp2(rl[j * kT + i] - mx);
+                const float p = (rl[j * kT + i] == -INFINITY) ? 0.0f : fast_exp2(rl[j * kT + i] - mx);
                 rl[j * kT + i] = p;
                 sm += p;
             }
