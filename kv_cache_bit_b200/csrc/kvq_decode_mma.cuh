@@ -33,7 +33,7 @@
 namespace kvq {
 
 constexpr int kNW = 4;    // consumer warps per CTA
-constexpr int kRing = 2;  // slots per warp
+constexpr int kRing = 3;  // slots per warp
 
 // ---------------------------------------------------------------- small PTX helpers
 
@@ -68,15 +68,14 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
     uint32_t r;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
     return r;
 }
 
 // D += A * B, m16n8k16, fp16 inputs, fp32 accumulators.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -257,16 +256,22 @@ struct VUnpack<3> {
 
 // ---------------------------------------------------------------- slot layout
 
+constexpr int kUT = 64;  // tokens per staging unit (half a block)
+
+// A unit is one tensor's half block: packed codes and per-token parameters of
+// 64 tokens; the first half also carries the block's channel scales and NSN
+// channel means.
 template <int D, int BITS, int MODE>
 struct SlotLayout {
     static constexpr int kRB = D * BITS / 8;
     static constexpr int kNtok = (MODE == kNsn) ? 2 : 1;
     static constexpr int kCodes = 0;
-    static constexpr int kTok = kT * kRB;
-    static constexpr int kChan = kTok + kT * kNtok * 2;
+    static constexpr int kTok = kUT * kRB;
+    static constexpr int kChan = kTok + kUT * kNtok * 2;
     static constexpr int kOff = kChan + ((MODE != kNaive) ? D * 2 : 0);
-    static constexpr int kBytes = kOff + ((MODE == kNsn) ? D * 2 : 0);
-    static constexpr int kStride = (kBytes + 127) / 128 * 128;
+    static constexpr int kBytesLo = kOff + ((MODE == kNsn) ? D * 2 : 0);  // first half
+    static constexpr int kBytesHi = kChan;                                 // second half
+    static constexpr int kStride = (kBytesLo + 127) / 128 * 128;
 };
 
 // Merge buffers reuse the ring after every warp is done with it.
@@ -285,6 +290,11 @@ __host__ __device__ constexpr int mma_smem_bytes() {
 __device__ __forceinline__ void mbar_inval(uint64_t* bar) {
     asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+
+// Token held by fragment row r (0..15) of a 16-token tile: rows 2k and 2k + 1
+// swap when k is odd.  Thread quads then read token rows of alternating
+// parity, which spreads the V-side loads over both halves of the banks.
+__device__ __forceinline__ int tile_tok(int r) { return r ^ ((r >> 1) & 1); }
 
 // ---------------------------------------------------------------- the kernel
 
@@ -364,33 +374,53 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     }
     __syncthreads();
 
-    // ---- this warp's blocks
+    // ---- this warp's blocks: units 4i + k = (K lo, K hi, V lo, V hi) of block i
     const int blk_begin = split * a.bps;
     const int blk_end = min(a.nbq, blk_begin + a.bps);
     const int nmine = blk_end > blk_begin + warp ? (blk_end - blk_begin - warp + kNW - 1) / kNW : 0;
-    const int nunits = 2 * nmine;
+    const int nunits = 4 * nmine;
     uint8_t* my_ring = ring + warp * kRing * SL::kStride;
     uint64_t* my_bars = bars + warp * kRing;
 
     auto issue = [&](int u) {
-        // unit u: block blk_begin + warp + kNW * (u / 2), tensor u % 2
-        const int blk = blk_begin + warp + kNW * (u >> 1);
-        const int ten = u & 1;
+        const int blk = blk_begin + warp + kNW * (u >> 2);
+        const int ten = (u >> 1) & 1;
+        const int half = u & 1;
         uint8_t* slot = my_ring + (u % kRing) * SL::kStride;
         uint64_t* bar = &my_bars[u % kRing];
-        const size_t row0 = (size_t)bh * a.cap + (size_t)blk * kT;
+        const size_t row0 = (size_t)bh * a.cap + (size_t)blk * kT + (size_t)half * kUT;
         const size_t bi = ((size_t)bh * nb_cap + blk) * D;
-        mbar_expect_tx(bar, SL::kBytes);
-        bulk_load(slot + SL::kCodes, (ten ? a.codes[1] : a.codes[0]) + row0 * SL::kRB, kT * SL::kRB, bar);
-        bulk_load(slot + SL::kTok, (ten ? a.tok[1] : a.tok[0]) + row0 * SL::kNtok, kT * SL::kNtok * 2, bar);
-        if (PCH) bulk_load(slot + SL::kChan, (ten ? a.chan[1] : a.chan[0]) + bi, D * 2, bar);
-        if (MODE == kNsn) bulk_load(slot + SL::kOff, (ten ? a.off[1] : a.off[0]) + bi, D * 2, bar);
+        mbar_expect_tx(bar, half ? SL::kBytesHi : SL::kBytesLo);
+        bulk_load(slot + SL::kCodes, (ten ? a.codes[1] : a.codes[0]) + row0 * SL::kRB, kUT * SL::kRB, bar);
+        bulk_load(slot + SL::kTok, (ten ? a.tok[1] : a.tok[0]) + row0 * SL::kNtok, kUT * SL::kNtok * 2, bar);
+        if (!half) {
+            if (PCH) bulk_load(slot + SL::kChan, (ten ? a.chan[1] : a.chan[0]) + bi, D * 2, bar);
+            if (MODE == kNsn) bulk_load(slot + SL::kOff, (ten ? a.off[1] : a.off[0]) + bi, D * 2, bar);
+        }
     };
     int issued = min(kRing, nunits);
     if (lane == 0) {
         for (int u = 0; u < issued; ++u) issue(u);
     }
     int waited = 0;
+    bool ok = true;
+    // wait for unit u; false on timeout
+    auto wait_unit = [&](int u) -> bool {
+        if (!mbar_wait(&my_bars[u % kRing], (u / kRing) & 1, 1u << 26)) return false;
+        waited = u + 1;
+        return true;
+    };
+    // unit u consumed: its slot takes unit u + kRing
+    auto release = [&](int u) {
+        __syncwarp();
+        if (u + kRing < nunits) {
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                issue(u + kRing);
+            }
+            issued = u + kRing + 1;
+        }
+    };
 
     // ---- persistent per-thread state: heads 4n + t, channels [16g, 16g + 16)
     float m_run[NT], l_run[NT];
@@ -408,133 +438,144 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     // the B column this thread feeds in each n-tile: head 4n + g/2, part g%2
     const bool blo = (g & 1) != 0;
     const float alpha2 = a.scale * kLog2e;
-    bool ok = true;
+    // token of fragment rows g and g + 8 inside a 16-token tile
+    const int tr0 = tile_tok(g), tr1 = 8 + tile_tok(g);
+    // V fragment rows 2t, 2t+1, 2t+8, 2t+9
+    const int vr0 = tile_tok(2 * t), vr1 = tile_tok(2 * t + 1);
 
     for (int it = 0; it < nmine; ++it) {
-        const int uK = 2 * it, uV = 2 * it + 1;
-        uint8_t* sk = my_ring + (uK % kRing) * SL::kStride;
-        uint8_t* sv = my_ring + (uV % kRing) * SL::kStride;
-        // ================= K half
-        if (!mbar_wait(&my_bars[uK % kRing], (uK / kRing) & 1, 1u << 26)) { ok = false; break; }
-        waited = uK + 1;
-        // B fragments: q' = qs * sigma^K as (hi, lo) fp16 parts
+        const int u0 = 4 * it;
+        // ================= K halves -> logits
         uint32_t bq[NT][16];
-        {
-            const __half* sig = reinterpret_cast<const __half*>(sk + SL::kChan) + 32 * t;
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const float* qrow = &s_qs[4 * n + (g >> 1)][32 * t];
-#pragma unroll
-                for (int p = 0; p < 16; ++p) {
-                    const int ca = KUnpack<BITS>::ca(p), cb = KUnpack<BITS>::cb(p);
-                    const float fa = qrow[ca] * (PCH ? __half2float(sig[ca]) : 1.0f);
-                    const float fb = qrow[cb] * (PCH ? __half2float(sig[cb]) : 1.0f);
-                    const __half2 hh = __floats2half2_rn(fa, fb);
-                    if (blo) {
-                        const float2 hf = __half22float2(hh);
-                        bq[n][p] = cvt_h2(fa - hf.x, fb - hf.y);
-                    } else {
-                        bq[n][p] = *reinterpret_cast<const uint32_t*>(&hh);
-                    }
-                }
-            }
-        }
-        // scores -> logits (log2 domain); thread holds tokens 16mt + g (+8)
-        const __half* tk = reinterpret_cast<const __half*>(sk + SL::kTok);
         float qoK[NT];
-        if constexpr (MODE == kNsn) {
-            const __half* okp = reinterpret_cast<const __half*>(sk + SL::kOff) + 16 * g;
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                float s = 0.0f;
-#pragma unroll
-                for (int k = 0; k < 16; ++k) s += s_q[4 * n + t][16 * g + k] * __half2float(okp[k]);
-#pragma unroll
-                for (int o = 4; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                qoK[n] = s;
-            }
-        }
         float lg[NT][8][2];
         float bmax[NT];
 #pragma unroll
         for (int n = 0; n < NT; ++n) bmax[n] = -INFINITY;
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            uint32_t pa[16], pb[16];
-            KUnpack<BITS>::run(sk + SL::kCodes + (16 * mt + g) * SL::kRB, t, pa);
-            KUnpack<BITS>::run(sk + SL::kCodes + (16 * mt + g + 8) * SL::kRB, t, pb);
+        for (int half = 0; half < 2; ++half) {
+            const int u = u0 + half;
+            if (!wait_unit(u)) { ok = false; break; }
+            uint8_t* sk = my_ring + (u % kRing) * SL::kStride;
+            if (half == 0) {
+                // B fragments: q' = qs * sigma^K as (hi, lo) fp16 parts
+                const __half* sig = reinterpret_cast<const __half*>(sk + SL::kChan) + 32 * t;
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                // two independent accumulation chains over the 8 k-steps
-                float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int n = 0; n < NT; ++n) {
+                    const float* qrow = &s_qs[4 * n + (g >> 1)][32 * t];
 #pragma unroll
-                for (int s = 0; s < 8; s += 2) {
-                    mma16816(d0, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], bq[n][2 * s], bq[n][2 * s + 1]);
-                    mma16816(d1, pa[2 * s + 2], pb[2 * s + 2], pa[2 * s + 3], pb[2 * s + 3], bq[n][2 * s + 2],
-                             bq[n][2 * s + 3]);
-                }
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int tok = 16 * mt + g + 8 * r;
-                    const float sv_ = (d0[2 * r] + d0[2 * r + 1]) + (d1[2 * r] + d1[2 * r + 1]);
-                    float kap, add = 0.0f;
-                    if constexpr (MODE == kNsn) {
-                        const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tk)[tok]);
-                        kap = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
-                        add = s12.x * qoK[n];
-                    } else {
-                        kap = __half2float(tk[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                    for (int p = 0; p < 16; ++p) {
+                        const int ca = KUnpack<BITS>::ca(p), cb = KUnpack<BITS>::cb(p);
+                        const float fa = qrow[ca] * (PCH ? __half2float(sig[ca]) : 1.0f);
+                        const float fb = qrow[cb] * (PCH ? __half2float(sig[cb]) : 1.0f);
+                        const __half2 hh = __floats2half2_rn(fa, fb);
+                        if (blo) {
+                            const float2 hf = __half22float2(hh);
+                            bq[n][p] = cvt_h2(fa - hf.x, fb - hf.y);
+                        } else {
+                            bq[n][p] = *reinterpret_cast<const uint32_t*>(&hh);
+                        }
                     }
-                    const float l2 = (sv_ * (kap * kcol[n]) + add) * alpha2;
-                    lg[n][mt][r] = l2;
-                    bmax[n] = fmaxf(bmax[n], l2);
+                }
+                if constexpr (MODE == kNsn) {
+                    const __half* okp = reinterpret_cast<const __half*>(sk + SL::kOff) + 16 * g;
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        float s = 0.0f;
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) s += s_q[4 * n + t][16 * g + k] * __half2float(okp[k]);
+#pragma unroll
+                        for (int o = 4; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                        qoK[n] = s;
+                    }
                 }
             }
-        }
-        __syncwarp();
-        if (uK + kRing < nunits) {
-            if (lane == 0) {
-                fence_proxy_async_smem();
-                issue(uK + kRing);
+            const __half* tk = reinterpret_cast<const __half*>(sk + SL::kTok);
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const int mt = 4 * half + m4;
+                uint32_t pa[16], pb[16];
+                KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr0) * SL::kRB, t, pa);
+                KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr1) * SL::kRB, t, pb);
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    // two independent accumulation chains over the 8 k-steps
+                    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int s = 0; s < 8; s += 2) {
+                        mma16816(d0, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], bq[n][2 * s],
+                                 bq[n][2 * s + 1]);
+                        mma16816(d1, pa[2 * s + 2], pb[2 * s + 2], pa[2 * s + 3], pb[2 * s + 3], bq[n][2 * s + 2],
+                                 bq[n][2 * s + 3]);
+                    }
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int tok = 16 * m4 + (r ? tr1 : tr0);
+                        const float sv_ = (d0[2 * r] + d0[2 * r + 1]) + (d1[2 * r] + d1[2 * r + 1]);
+                        float kap, add = 0.0f;
+                        if constexpr (MODE == kNsn) {
+                            const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tk)[tok]);
+                            kap = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
+                            add = s12.x * qoK[n];
+                        } else {
+                            kap = __half2float(tk[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                        }
+                        const float l2 = (sv_ * (kap * kcol[n]) + add) * alpha2;
+                        lg[n][mt][r] = l2;
+                        bmax[n] = fmaxf(bmax[n], l2);
+                    }
+                }
             }
-            issued = uK + kRing + 1;
+            release(u);
         }
+        if (!ok) break;
 #pragma unroll
         for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) bmax[n] = fmaxf(bmax[n], __shfl_xor_sync(0xffffffffu, bmax[n], o));
-        // ================= V half
-        if (!mbar_wait(&my_bars[uV % kRing], (uV / kRing) & 1, 1u << 26)) { ok = false; break; }
-        waited = uV + 1;
-        const __half* tv = reinterpret_cast<const __half*>(sv + SL::kTok);
         // online softmax: rescale when the running max moves
-        bool changed = false;
-        float corr[NT];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const float mn = fmaxf(m_run[n], bmax[n]);
-            corr[n] = fast_exp2(m_run[n] - mn);
-            changed |= (mn != m_run[n]);
-            m_run[n] = mn;
-            l_run[n] *= corr[n];
-        }
-        if (__any_sync(0xffffffffu, changed)) {
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    acc[n][k] *= corr[n];
-                    if (MODE == kNsn) acco[n][k] *= corr[n];
-                }
-        }
-        // power-of-two scale keeping p * nu * 2^f <= 2^13 in fp16 (p <= 1)
-        float numax;
         {
-            // lane scans tokens 4 lane .. 4 lane + 3
-            float mx = 0.0f;
+            bool changed = false;
+            float corr[NT];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int tok = 4 * lane + k;
+            for (int n = 0; n < NT; ++n) {
+                const float mn = fmaxf(m_run[n], bmax[n]);
+                corr[n] = fast_exp2(m_run[n] - mn);
+                changed |= (mn != m_run[n]);
+                m_run[n] = mn;
+                l_run[n] *= corr[n];
+            }
+            if (__any_sync(0xffffffffu, changed)) {
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        acc[n][k] *= corr[n];
+                        if (MODE == kNsn) acco[n][k] *= corr[n];
+                    }
+            }
+        }
+        // ================= V halves
+        __half2 sigv[8], offv[8];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int u = u0 + 2 + half;
+            if (!wait_unit(u)) { ok = false; break; }
+            uint8_t* sv = my_ring + (u % kRing) * SL::kStride;
+            if (half == 0) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    sigv[k] = PCH ? reinterpret_cast<const __half2*>(sv + SL::kChan)[8 * g + k] : __floats2half2_rn(1.f, 1.f);
+                    offv[k] = (MODE == kNsn) ? reinterpret_cast<const __half2*>(sv + SL::kOff)[8 * g + k]
+                                             : __floats2half2_rn(0.f, 0.f);
+                }
+            }
+            const __half* tv = reinterpret_cast<const __half*>(sv + SL::kTok);
+            // power-of-two scale keeping p * nu * 2^f <= 2^13 in fp16 (p <= 1)
+            float numax = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int tok = 2 * lane + k;
                 float v;
                 if constexpr (MODE == kNsn) {
                     const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
@@ -542,97 +583,87 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                 } else {
                     v = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
                 }
-                mx = fmaxf(mx, v);
+                numax = fmaxf(numax, v);
             }
 #pragma unroll
-            for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            numax = mx;
-        }
-        const int fexp = numax > 0.0f ? 13 - ceil_log2(numax) : 0;
-        const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
-        float dv[NT][8][4];
+            for (int o = 16; o; o >>= 1) numax = fmaxf(numax, __shfl_xor_sync(0xffffffffu, numax, o));
+            const int fexp = numax > 0.0f ? 13 - ceil_log2(numax) : 0;
+            const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
+            float dv[NT][8][4];
 #pragma unroll
-        for (int n = 0; n < NT; ++n)
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int k = 0; k < 4; ++k) dv[n][i][k] = 0.0f;
-        float lsum[NT], bsum[NT];
+                    for (int k = 0; k < 4; ++k) dv[n][i][k] = 0.0f;
+            float lsum[NT], bsum[NT];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
+            for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            uint32_t bp[NT][2];
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const int mt = 4 * half + m4;
+                uint32_t bp[NT][2];
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int tok = 16 * mt + g + 8 * r;
-                float nu, s1o = 0.0f;
-                if constexpr (MODE == kNsn) {
-                    const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
-                    s1o = s12.x;
-                    nu = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
-                } else {
-                    nu = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                for (int r = 0; r < 2; ++r) {
+                    const int tok = 16 * m4 + (r ? tr1 : tr0);
+                    float nu, s1o = 0.0f;
+                    if constexpr (MODE == kNsn) {
+                        const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
+                        s1o = s12.x;
+                        nu = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
+                    } else {
+                        nu = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                    }
+                    nu *= pscale;
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        const float p = fast_exp2(lg[n][mt][r] - m_run[n]);
+                        lsum[n] += p;
+                        if constexpr (MODE == kNsn) bsum[n] += p * s1o;
+                        // row tok: (hi, lo) of head 4n + t in columns 2t, 2t + 1
+                        bp[n][r] = movmatrix_t(split_h2(p * nu));
+                    }
                 }
-                nu *= pscale;
+                uint32_t va[16], vb[16];
+                const uint8_t* vbase = sv + SL::kCodes + (16 * m4) * SL::kRB;
+                VUnpack<BITS>::run(vbase + vr0 * SL::kRB, vbase + vr1 * SL::kRB, g, va);
+                VUnpack<BITS>::run(vbase + (8 + vr0) * SL::kRB, vbase + (8 + vr1) * SL::kRB, g, vb);
 #pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const float p = fast_exp2(lg[n][mt][r] - m_run[n]);
-                    lsum[n] += p;
-                    if constexpr (MODE == kNsn) bsum[n] += p * s1o;
-                    // row tok: (hi, lo) of head 4n + t in columns 2t, 2t + 1
-                    bp[n][r] = movmatrix_t(split_h2(p * nu));
+                for (int tc = 0; tc < 8; ++tc) {
+#pragma unroll
+                    for (int n = 0; n < NT; ++n)
+                        mma16816(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1], bp[n][0], bp[n][1]);
                 }
             }
-            uint32_t va[16], vb[16];
-            const uint8_t* vbase = sv + SL::kCodes + (16 * mt) * SL::kRB;
-            VUnpack<BITS>::run(vbase + (2 * t) * SL::kRB, vbase + (2 * t + 1) * SL::kRB, g, va);
-            VUnpack<BITS>::run(vbase + (2 * t + 8) * SL::kRB, vbase + (2 * t + 9) * SL::kRB, g, vb);
+#pragma unroll
+            for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
+            // unit epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f
 #pragma unroll
             for (int tc = 0; tc < 8; ++tc) {
-#pragma unroll
-                for (int n = 0; n < NT; ++n)
-                    mma16816(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1], bp[n][0], bp[n][1]);
-            }
-        }
-#pragma unroll
-        for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
-        // block epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f
-        {
-            const __half* sigv = reinterpret_cast<const __half*>(sv + SL::kChan) + 16 * g;
-#pragma unroll
-            for (int tc = 0; tc < 8; ++tc) {
-                float s0 = pinv, s1_ = pinv;
-                if (PCH) {
-                    const float2 sg = __half22float2(reinterpret_cast<const __half2*>(sigv)[tc]);
-                    s0 *= sg.x;
-                    s1_ *= sg.y;
-                }
+                const float2 sg = __half22float2(sigv[tc]);
+                const float s0 = sg.x * pinv, s1_ = sg.y * pinv;
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     acc[n][2 * tc] += (dv[n][tc][0] + dv[n][tc][1]) * s0;
                     acc[n][2 * tc + 1] += (dv[n][tc][2] + dv[n][tc][3]) * s1_;
                 }
             }
-        }
-        if constexpr (MODE == kNsn) {
-            const __half* ov = reinterpret_cast<const __half*>(sv + SL::kOff) + 16 * g;
+            if constexpr (MODE == kNsn) {
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
+                for (int n = 0; n < NT; ++n) {
 #pragma unroll
-                for (int o = 4; o < 32; o <<= 1) bsum[n] += __shfl_xor_sync(0xffffffffu, bsum[n], o);
+                    for (int o = 4; o < 32; o <<= 1) bsum[n] += __shfl_xor_sync(0xffffffffu, bsum[n], o);
 #pragma unroll
-                for (int k = 0; k < 16; ++k) acco[n][k] += bsum[n] * __half2float(ov[k]);
+                    for (int k = 0; k < 8; ++k) {
+                        const float2 ov = __half22float2(offv[k]);
+                        acco[n][2 * k] += bsum[n] * ov.x;
+                        acco[n][2 * k + 1] += bsum[n] * ov.y;
+                    }
+                }
             }
+            release(u);
         }
-        __syncwarp();
-        if (uV + kRing < nunits) {
-            if (lane == 0) {
-                fence_proxy_async_smem();
-                issue(uV + kRing);
-            }
-            issued = uV + kRing + 1;
-        }
+        if (!ok) break;
     }
     if (!ok) {
         // give the copies still in flight a bounded time to land before the
