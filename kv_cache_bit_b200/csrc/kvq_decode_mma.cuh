@@ -333,8 +333,12 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 
     uint8_t* ring = smem_raw;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kNW * kRing * SL::kStride);
-    __shared__ float s_q[GP][D];   // queries (original domain)
-    __shared__ float s_qs[GP][D];  // rotated queries times the head's power-of-two scale
+    __shared__ float s_q[GP][D];  // queries (original domain)
+    // rotated queries times the head's power-of-two scale; element c of head j
+    // at j * kQS + c + c / 32, so the four 32-channel slices of four heads fall
+    // in distinct banks
+    constexpr int kQS = D + 4;
+    __shared__ float s_qs[GP * kQS];
     __shared__ float s_qscale[GP];
 
     if (tid < kNW * kRing) mbar_init(&bars[tid], 1);
@@ -369,12 +373,15 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
         const float bound = PCH ? amax * (1.001f / (float)QMAX) : amax;
         const float qsc = bound > 0.0f ? pow2i(13 - ceil_log2(bound)) : 1.0f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) s_qs[j][4 * lane + k] = v[k] * qsc;
+        for (int k = 0; k < 4; ++k) {
+            const int c = 4 * lane + k;
+            s_qs[j * kQS + c + (c >> 5)] = v[k] * qsc;
+        }
         if (lane == 0) s_qscale[j] = qsc;
     }
     __syncthreads();
 
-    // ---- this warp's blocks: units 4i + k = (K lo, K hi, V lo, V hi) of block i
+    // ---- this warp's blocks: units 4i + k = (K lo, V lo, K hi, V hi) of block i
     const int blk_begin = split * a.bps;
     const int blk_end = min(a.nbq, blk_begin + a.bps);
     const int nmine = blk_end > blk_begin + warp ? (blk_end - blk_begin - warp + kNW - 1) / kNW : 0;
@@ -384,8 +391,8 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 
     auto issue = [&](int u) {
         const int blk = blk_begin + warp + kNW * (u >> 2);
-        const int ten = (u >> 1) & 1;
-        const int half = u & 1;
+        const int ten = u & 1;
+        const int half = (u >> 1) & 1;
         uint8_t* slot = my_ring + (u % kRing) * SL::kStride;
         uint64_t* bar = &my_bars[u % kRing];
         const size_t row0 = (size_t)bh * a.cap + (size_t)blk * kT + (size_t)half * kUT;
@@ -404,7 +411,6 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     }
     int waited = 0;
     bool ok = true;
-    // wait for unit u; false on timeout
     auto wait_unit = [&](int u) -> bool {
         if (!mbar_wait(&my_bars[u % kRing], (u / kRing) & 1, 1u << 26)) return false;
         waited = u + 1;
@@ -423,11 +429,15 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     };
 
     // ---- persistent per-thread state: heads 4n + t, channels [16g, 16g + 16)
-    float m_run[NT], l_run[NT];
+    // Softmax weights are taken against a reference max m_ref that only moves
+    // when a tile's logit exceeds it by more than kTau (log2 units), so that
+    // p <= 2^kTau and most tiles need no rescale.
+    constexpr float kTau = 8.0f;
+    float m_ref[NT], l_run[NT];
     float acc[NT][16], acco[NT][16];
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-        m_run[n] = -INFINITY;
+        m_ref[n] = -INFINITY;
         l_run[n] = 0.0f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) { acc[n][k] = 0.0f; acco[n][k] = 0.0f; }
@@ -443,26 +453,21 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     // V fragment rows 2t, 2t+1, 2t+8, 2t+9
     const int vr0 = tile_tok(2 * t), vr1 = tile_tok(2 * t + 1);
 
+    uint32_t bq[NT][16];
+    float qoK[NT];
+    __half2 sigv[8], offv[8];
     for (int it = 0; it < nmine; ++it) {
-        const int u0 = 4 * it;
-        // ================= K halves -> logits
-        uint32_t bq[NT][16];
-        float qoK[NT];
-        float lg[NT][8][2];
-        float bmax[NT];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) bmax[n] = -INFINITY;
-#pragma unroll
+#pragma unroll 1
         for (int half = 0; half < 2; ++half) {
-            const int u = u0 + half;
-            if (!wait_unit(u)) { ok = false; break; }
-            uint8_t* sk = my_ring + (u % kRing) * SL::kStride;
+            const int uk = 4 * it + 2 * half, uv = uk + 1;
+            if (!wait_unit(uk)) { ok = false; break; }
+            uint8_t* sk = my_ring + (uk % kRing) * SL::kStride;
             if (half == 0) {
                 // B fragments: q' = qs * sigma^K as (hi, lo) fp16 parts
                 const __half* sig = reinterpret_cast<const __half*>(sk + SL::kChan) + 32 * t;
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
-                    const float* qrow = &s_qs[4 * n + (g >> 1)][32 * t];
+                    const float* qrow = &s_qs[(4 * n + (g >> 1)) * kQS + 33 * t];
 #pragma unroll
                     for (int p = 0; p < 16; ++p) {
                         const int ca = KUnpack<BITS>::ca(p), cb = KUnpack<BITS>::cb(p);
@@ -490,16 +495,57 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                     }
                 }
             }
+            if (!wait_unit(uv)) { ok = false; break; }
+            uint8_t* sv = my_ring + (uv % kRing) * SL::kStride;
+            if (half == 0) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    sigv[k] = PCH ? reinterpret_cast<const __half2*>(sv + SL::kChan)[8 * g + k]
+                                  : __floats2half2_rn(1.f, 1.f);
+                    offv[k] = (MODE == kNsn) ? reinterpret_cast<const __half2*>(sv + SL::kOff)[8 * g + k]
+                                             : __floats2half2_rn(0.f, 0.f);
+                }
+            }
             const __half* tk = reinterpret_cast<const __half*>(sk + SL::kTok);
+            const __half* tv = reinterpret_cast<const __half*>(sv + SL::kTok);
+            // power-of-two scale keeping p * nu * 2^f <= 2^13 in fp16 (p <= 2^kTau)
+            float numax = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int tok = 2 * lane + k;
+                float v;
+                if constexpr (MODE == kNsn) {
+                    const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
+                    v = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
+                } else {
+                    v = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                }
+                numax = fmaxf(numax, v);
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) numax = fmaxf(numax, __shfl_xor_sync(0xffffffffu, numax, o));
+            const int fexp = numax > 0.0f ? 13 - (int)kTau - ceil_log2(numax) : 0;
+            const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
+            float dv[NT][8][4];
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) dv[n][i][k] = 0.0f;
+            float lsum[NT], bsum[NT];
+#pragma unroll
+            for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
 #pragma unroll
             for (int m4 = 0; m4 < 4; ++m4) {
-                const int mt = 4 * half + m4;
+                // ---- scores of the tile's 16 tokens
                 uint32_t pa[16], pb[16];
                 KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr0) * SL::kRB, t, pa);
                 KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr1) * SL::kRB, t, pb);
+                float l2[NT][2];
+                bool over = false;
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
-                    // two independent accumulation chains over the 8 k-steps
                     float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int s = 0; s < 8; s += 2) {
@@ -520,88 +566,35 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                         } else {
                             kap = __half2float(tk[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
                         }
-                        const float l2 = (sv_ * (kap * kcol[n]) + add) * alpha2;
-                        lg[n][mt][r] = l2;
-                        bmax[n] = fmaxf(bmax[n], l2);
+                        l2[n][r] = (sv_ * (kap * kcol[n]) + add) * alpha2;
+                        over |= l2[n][r] > m_ref[n] + kTau;
                     }
                 }
-            }
-            release(u);
-        }
-        if (!ok) break;
+                // ---- rare: move the reference max up and rescale what was accumulated
+                if (__any_sync(0xffffffffu, over)) {
 #pragma unroll
-        for (int n = 0; n < NT; ++n)
+                    for (int n = 0; n < NT; ++n) {
+                        float mx = fmaxf(l2[n][0], l2[n][1]);
 #pragma unroll
-            for (int o = 4; o < 32; o <<= 1) bmax[n] = fmaxf(bmax[n], __shfl_xor_sync(0xffffffffu, bmax[n], o));
-        // online softmax: rescale when the running max moves
-        {
-            bool changed = false;
-            float corr[NT];
+                        for (int o = 4; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                        const float mn = fmaxf(m_ref[n], mx);
+                        const float corr = fast_exp2(m_ref[n] - mn);
+                        m_ref[n] = mn;
+                        l_run[n] *= corr;
+                        lsum[n] *= corr;
+                        bsum[n] *= corr;
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const float mn = fmaxf(m_run[n], bmax[n]);
-                corr[n] = fast_exp2(m_run[n] - mn);
-                changed |= (mn != m_run[n]);
-                m_run[n] = mn;
-                l_run[n] *= corr[n];
-            }
-            if (__any_sync(0xffffffffu, changed)) {
+                        for (int k = 0; k < 16; ++k) {
+                            acc[n][k] *= corr;
+                            if (MODE == kNsn) acco[n][k] *= corr;
+                        }
 #pragma unroll
-                for (int n = 0; n < NT; ++n)
+                        for (int i = 0; i < 8; ++i)
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        acc[n][k] *= corr[n];
-                        if (MODE == kNsn) acco[n][k] *= corr[n];
+                            for (int k = 0; k < 4; ++k) dv[n][i][k] *= corr;
                     }
-            }
-        }
-        // ================= V halves
-        __half2 sigv[8], offv[8];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int u = u0 + 2 + half;
-            if (!wait_unit(u)) { ok = false; break; }
-            uint8_t* sv = my_ring + (u % kRing) * SL::kStride;
-            if (half == 0) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    sigv[k] = PCH ? reinterpret_cast<const __half2*>(sv + SL::kChan)[8 * g + k] : __floats2half2_rn(1.f, 1.f);
-                    offv[k] = (MODE == kNsn) ? reinterpret_cast<const __half2*>(sv + SL::kOff)[8 * g + k]
-                                             : __floats2half2_rn(0.f, 0.f);
                 }
-            }
-            const __half* tv = reinterpret_cast<const __half*>(sv + SL::kTok);
-            // power-of-two scale keeping p * nu * 2^f <= 2^13 in fp16 (p <= 1)
-            float numax = 0.0f;
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int tok = 2 * lane + k;
-                float v;
-                if constexpr (MODE == kNsn) {
-                    const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
-                    v = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
-                } else {
-                    v = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
-                }
-                numax = fmaxf(numax, v);
-            }
-#pragma unroll
-            for (int o = 16; o; o >>= 1) numax = fmaxf(numax, __shfl_xor_sync(0xffffffffu, numax, o));
-            const int fexp = numax > 0.0f ? 13 - ceil_log2(numax) : 0;
-            const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
-            float dv[NT][8][4];
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) dv[n][i][k] = 0.0f;
-            float lsum[NT], bsum[NT];
-#pragma unroll
-            for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
-#pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-                const int mt = 4 * half + m4;
+                // ---- P' = p * nu (scaled), as (hi, lo) rows, moved into the B layout
                 uint32_t bp[NT][2];
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
@@ -617,13 +610,13 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                     nu *= pscale;
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
-                        const float p = fast_exp2(lg[n][mt][r] - m_run[n]);
+                        const float p = fast_exp2(l2[n][r] - m_ref[n]);
                         lsum[n] += p;
                         if constexpr (MODE == kNsn) bsum[n] += p * s1o;
-                        // row tok: (hi, lo) of head 4n + t in columns 2t, 2t + 1
                         bp[n][r] = movmatrix_t(split_h2(p * nu));
                     }
                 }
+                // ---- values
                 uint32_t va[16], vb[16];
                 const uint8_t* vbase = sv + SL::kCodes + (16 * m4) * SL::kRB;
                 VUnpack<BITS>::run(vbase + vr0 * SL::kRB, vbase + vr1 * SL::kRB, g, va);
@@ -635,6 +628,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                         mma16816(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1], bp[n][0], bp[n][1]);
                 }
             }
+            release(uk);
 #pragma unroll
             for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
             // unit epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f
@@ -661,10 +655,13 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                     }
                 }
             }
-            release(u);
+            release(uv);
         }
         if (!ok) break;
     }
+    float m_run[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) m_run[n] = m_ref[n];
     if (!ok) {
         // give the copies still in flight a bounded time to land before the
         // shared memory is reused; the results of this call are void
