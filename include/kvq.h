@@ -207,7 +207,7 @@ kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t
  * cudaMalloc would synchronize the device.
  * Same arguments, results and errors as kvq_decode_attention, minus the
  * workspace.  The split-K partial results go to a scratch array of
- * KVQ_NOALLOC_SCRATCH_BYTES (8 MiB) that the library holds in device memory
+ * KVQ_NOALLOC_SCRATCH_BYTES (32 MiB) that the library holds in device memory
  * on every GPU that loads it, until the process exits.  A call whose
  * workspace need (kvq_decode_workspace_bytes) exceeds that size returns
  * KVQ_ERR_WORKSPACE before enqueuing anything.
@@ -218,7 +218,7 @@ kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t
  * streams, or different host threads) race and corrupt each other's results.
  * The call never runs cudaMalloc, cudaFree or any allocating routine.
  */
-#define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define KVQ_NOALLOC_SCRATCH_BYTES (32u << 20)
 kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache* cache,
                                         const uint16_t* q, int32_t q_heads, float scale,
                                         float* out, void* stream);

@@ -126,9 +126,13 @@ bool make_row_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dynamic shared memory size, and the largest shared-memory carveout so that
+// the residency the occupancy calculator reports is the one the launch gets.
 template <typename K>
 bool set_smem(K kernel, int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
+           cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared) == cudaSuccess;
 }
 
 QuantArgs quant_args(const kvq_config* cfg, const kvq_cache* c) {
@@ -200,16 +204,44 @@ struct DequantLaunch {
 
 template <int D, int BITS, int MODE, bool HAD, int GP>
 kvq_status launch_decode_mma(DecodeArgs a, int bh, cudaStream_t st) {
-    constexpr int smem = mma_smem_bytes<D, BITS, MODE>();
+    constexpr int smem = mma_smem_bytes<D, BITS, MODE, GP>();
+    auto kern = decode_mma_kernel<D, BITS, MODE, HAD, GP>;
     static bool attr = false;
-    if (!attr) attr = set_smem(decode_mma_kernel<D, BITS, MODE, HAD, GP>, smem);
+    if (!attr) attr = set_smem(kern, smem);
     if (!attr) return KVQ_ERR_CUDA;
-    // every warp of a CTA gets the same number of blocks
-    a.bps = (a.bps + kNW - 1) / kNW * kNW;
-    decode_mma_kernel<D, BITS, MODE, HAD, GP><<<dim3(a.nsplit, bh), kNW * 32, smem, st>>>(a);
-    kvq_status s = launch_status();
-    if (s != KVQ_OK) return s;
-    decode_combine_kernel<D, HAD><<<bh, kT, 0, st>>>(a);
+    int dev = 0, sms = 0, occ = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kNW * 32, smem) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    int grid = sms * (occ > 0 ? occ : 1);
+    if (grid > kMaxCTAs) grid = kMaxCTAs;
+    a.nwarps = (long long)grid * kNW;
+    a.work = (long long)bh * a.nbq;
+    if (a.work >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+    if (a.work > 0) {
+        kern<<<grid, kNW * 32, smem, st>>>(a);
+        kvq_status s = launch_status();
+        if (s != KVQ_OK) return s;
+    }
+    // the combine kernel is a programmatic dependent of the decode kernel:
+    // its residual phase overlaps the decode kernel's tail
+    auto comb = decode_combine_mma_kernel<D, HAD, GP>;
+    constexpr int csmem = combine_smem_bytes<D>();
+    static bool cattr = false;
+    if (!cattr) cattr = set_smem(comb, csmem);
+    if (!cattr) return KVQ_ERR_CUDA;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(bh);
+    lc.blockDim = dim3(128);
+    lc.dynamicSmemBytes = csmem;
+    lc.stream = st;
+    cudaLaunchAttribute la[1];
+    la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    la[0].val.programmaticStreamSerializationAllowed = a.work > 0 ? 1 : 0;
+    lc.attrs = la;
+    lc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&lc, comb, a) != cudaSuccess) return KVQ_ERR_CUDA;
     return launch_status();
 }
 
@@ -331,6 +363,10 @@ size_t kvq_decode_workspace_bytes(const kvq_config* cfg, const kvq_cache* cache,
     const int G = q_heads / cache->kv_heads;
     if (G > kGMax) return 0;
     const size_t bh = (size_t)cache->batch * cache->kv_heads;
+    // tensor-core path: one partial per (warp, pair) segment, kNW slots per
+    // (CTA, pair) meeting; those are bounded by (largest persistent grid) + (pairs)
+    if (cfg->head_dim == 128)
+        return (size_t)kNW * ((size_t)kMaxCTAs + bh) * (size_t)G * part_stride<128>() * sizeof(float);
     return bh * (size_t)decode_splits(cache) * (size_t)G * (2 + 2 * (size_t)cfg->head_dim) * sizeof(float);
 }
 

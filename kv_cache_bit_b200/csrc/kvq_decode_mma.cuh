@@ -1,14 +1,17 @@
 // kvq_decode_mma.cuh -- decode attention over the packed cache on the tensor
 // cores (head dim 128).  Included once, by kvq_api.cu.
 //
-// Work: grid (split, batch*kv-head); a CTA of kNW warps covers a contiguous
-// range of 128-token blocks of one (batch, kv head); warp w takes blocks
-// w, w + kNW, ... of the range, each warp an independent online-softmax
-// partial.  Each warp owns a ring of kRing shared-memory slots; a slot holds
-// one tensor's half of a block (packed codes, per-token parameters, channel
-// scales and NSN means), brought in by 1-D bulk copies (no multicast) that
-// complete on the slot's mbarrier.  The order of slots is K(b0), V(b0),
-// K(b1), V(b1), ...
+// Work: a persistent grid.  The quantized blocks of all (batch, kv head)
+// pairs are laid end to end and split into equal contiguous ranges, one per
+// CTA; warp w of a CTA takes blocks w, w + kNW, ... of the range (so the
+// warps of a CTA stream neighbouring blocks) through its own ring of kRing
+// shared-memory slots, and writes one partial softmax state per pair segment
+// it covers.  A
+// slot holds one tensor's half block (packed codes, per-token parameters,
+// and on the first half the channel scales and NSN means), brought in by 1-D
+// bulk copies (no multicast) that complete on the slot's mbarrier.  Per block
+// the unit order is K lo, V lo, K hi, V hi.  decode_combine_mma_kernel then
+// merges the partials of each pair with its fp16 residual tokens.
 //
 // Per block (all G query heads of the kv head at once, G <= 8):
 //   scores  S[tok][col] = sum_c code[tok][c] * q'[c][col] with
@@ -99,6 +102,20 @@ __device__ __forceinline__ int ceil_log2(float x) {
     const int e = int((b >> 23) & 0xFF) - 127;
     return (b & 0x7FFFFF) ? e + 1 : e;
 }
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Programmatic dependent launch: the decode kernel lets the combine kernel
+// be scheduled early; the combine kernel does its residual work and then
+// waits here until the decode kernel has finished and its partials are
+// visible.  Without the launch attribute the wait returns at once.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 constexpr uint32_t kMagic = 0x64006400u;  // fp16x2 1024.0, 1024.0
 
@@ -257,6 +274,7 @@ struct VUnpack<3> {
 // ---------------------------------------------------------------- slot layout
 
 constexpr int kUT = 64;  // tokens per staging unit (half a block)
+constexpr int kMaxCTAs = 4 * 148;  // cap of the persistent grid
 
 // A unit is one tensor's half block: packed codes and per-token parameters of
 // 64 tokens; the first half also carries the block's channel scales and NSN
@@ -274,17 +292,26 @@ struct SlotLayout {
     static constexpr int kStride = (kBytesLo + 127) / 128 * 128;
 };
 
-// Merge buffers reuse the ring after every warp is done with it.
-template <int D>
-__host__ __device__ constexpr int mma_merge_bytes() {
-    return (2 * kNW * kGMax + 2 * kNW * kGMax * D + kGMax * kT + 2 * kGMax) * 4;
-}
+constexpr int kQS = 128 + 4;  // row stride of the skewed rotated-query table
 
-template <int D, int BITS, int MODE>
+// Partial record of one (segment, head): [m, l, 0, 0, acc[D], acc_o[D]]; the
+// two pad floats keep acc and acc_o 16-byte aligned for vector stores.
+template <int D>
+__host__ __device__ constexpr int part_stride() { return 4 + 2 * D; }
+
+template <int D, int BITS, int MODE, int GP>
+struct MmaSmem {
+    static constexpr int kRing0 = 0;
+    static constexpr int kBars = kNW * kRing * SlotLayout<D, BITS, MODE>::kStride;
+    static constexpr int kQ = kBars + kNW * kRing * 8;        // per warp: q [GP][D] fp32
+    static constexpr int kQs = kQ + kNW * GP * D * 4;         // per warp: skewed scaled rotated q [GP][kQS]
+    static constexpr int kQsc = kQs + kNW * GP * kQS * 4;     // per warp: [GP] scales
+    static constexpr int kBytes = kQsc + kNW * GP * 4 + 128;
+};
+
+template <int D, int BITS, int MODE, int GP>
 __host__ __device__ constexpr int mma_smem_bytes() {
-    constexpr int ring = kNW * kRing * SlotLayout<D, BITS, MODE>::kStride + kNW * kRing * 8;
-    constexpr int merge = mma_merge_bytes<D>();
-    return (ring > merge ? ring : merge) + 128;
+    return MmaSmem<D, BITS, MODE, GP>::kBytes;
 }
 
 __device__ __forceinline__ void mbar_inval(uint64_t* bar) {
@@ -295,6 +322,26 @@ __device__ __forceinline__ void mbar_inval(uint64_t* bar) {
 // swap when k is odd.  Thread quads then read token rows of alternating
 // parity, which spreads the V-side loads over both halves of the banks.
 __device__ __forceinline__ int tile_tok(int r) { return r ^ ((r >> 1) & 1); }
+
+// Split of `work` blocks over nctas CTAs: the first r CTAs take q + 1 blocks,
+// the others q (q = work / nctas, r = work % nctas; work < 2^31).
+struct CtaSplit {
+    int q, r;
+    __host__ __device__ CtaSplit(long long work, long long nctas)
+        : q((int)(work / nctas)), r((int)(work % nctas)) {}
+    __host__ __device__ int start(int c) const { return c * q + min(c, r); }
+    // CTA holding block x
+    __host__ __device__ int cta_of(int x) const {
+        const int big = r * (q + 1);
+        return x < big ? x / (q + 1) : r + (x - big) / q;
+    }
+};
+
+// Partial slot of warp w of CTA c for pair p: CTA ranges are contiguous and
+// ordered, so c + p is unique per (CTA, pair) that meet; slots < kNW * (nctas + pairs).
+__host__ __device__ __forceinline__ long long part_slot(long long c, int w, long long p) {
+    return (c + p) * kNW + w;
+}
 
 // ---------------------------------------------------------------- the kernel
 
@@ -314,89 +361,56 @@ __device__ __forceinline__ uint32_t split_h2(float x) {
 // Column layout of every n-tile (8 columns): column 2j + part holds part
 // (0 = hi, 1 = lo) of head 4n + j.  Thread (g, t) of a warp therefore owns
 // head 4n + t of every n-tile in the C fragments and sums its two columns.
+// Partial state of a (warp, pair) segment goes to slot part_slot() of a.part:
+// [m (log2 units), l, pad, pad, acc[D] (rotated domain), acc_o[D] (original
+// domain)] per head (part_stride floats).
 template <int D, int BITS, int MODE, bool HAD, int GP>
 __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "tensor-core decode is built for head dim 128");
     using SL = SlotLayout<D, BITS, MODE>;
+    using SM = MmaSmem<D, BITS, MODE, GP>;
     constexpr int NT = GP / 4;  // n-tiles (heads per thread)
     constexpr bool PCH = MODE != kNaive;
     constexpr float kLog2e = 1.4426950408889634f;
     constexpr int QMAX = (1 << (BITS - 1)) - 1;
+    constexpr float kTau = 8.0f;  // reference-max slack (log2 units): p <= 2^kTau
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
+    grid_dep_launch();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int split = blockIdx.x, bh = blockIdx.y;
     const int G = a.G;
-    const int b = bh / a.H, h = bh % a.H;
+    const int nbq = a.nbq;
     const int nb_cap = a.cap / kT;
-
-    uint8_t* ring = smem_raw;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kNW * kRing * SL::kStride);
-    __shared__ float s_q[GP][D];  // queries (original domain)
-    // rotated queries times the head's power-of-two scale; element c of head j
-    // at j * kQS + c + c / 32, so the four 32-channel slices of four heads fall
-    // in distinct banks
-    constexpr int kQS = D + 4;
-    __shared__ float s_qs[GP * kQS];
-    __shared__ float s_qscale[GP];
-
-    if (tid < kNW * kRing) mbar_init(&bars[tid], 1);
-    fence_mbar_init();
-    // ---- prologue: each warp rotates heads warp, warp + kNW, ... (lane owns 4 channels)
-    for (int j = warp; j < GP; j += kNW) {
-        float v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int c = 4 * lane + k;
-            const float qv = (j < G) ? __half2float(a.q[((size_t)b * a.H * G + (size_t)h * G + j) * D + c]) : 0.0f;
-            s_q[j][c] = qv;
-            v[k] = (HAD && a.signs != nullptr && a.signs[c] < 0) ? -qv : qv;
-        }
-        if constexpr (HAD) {
-            float x0 = v[0] + v[1], x1 = v[0] - v[1], x2 = v[2] + v[3], x3 = v[2] - v[3];
-            v[0] = x0 + x2; v[2] = x0 - x2; v[1] = x1 + x3; v[3] = x1 - x3;
-#pragma unroll
-            for (int m = 1; m < 32; m <<= 1) {
-                const bool upper = (lane & m) != 0;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
-                    v[k] = upper ? (o - v[k]) : (v[k] + o);
-                }
-            }
-        }
-        float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-#pragma unroll
-        for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        // |q'| <= amax * max(sigma) <= amax / qmax (1 + 2^-10): keep it below 2^13
-        const float bound = PCH ? amax * (1.001f / (float)QMAX) : amax;
-        const float qsc = bound > 0.0f ? pow2i(13 - ceil_log2(bound)) : 1.0f;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int c = 4 * lane + k;
-            s_qs[j * kQS + c + (c >> 5)] = v[k] * qsc;
-        }
-        if (lane == 0) s_qscale[j] = qsc;
-    }
-    __syncthreads();
-
-    // ---- this warp's blocks: units 4i + k = (K lo, V lo, K hi, V hi) of block i
-    const int blk_begin = split * a.bps;
-    const int blk_end = min(a.nbq, blk_begin + a.bps);
-    const int nmine = blk_end > blk_begin + warp ? (blk_end - blk_begin - warp + kNW - 1) / kNW : 0;
+    const int cta = blockIdx.x;
+    const CtaSplit split(a.work, a.nwarps / kNW);
+    const int c0 = split.start(cta), c1 = split.start(cta + 1);
+    const int w0 = c0 + warp;  // this warp's blocks: w0, w0 + kNW, ... < c1
+    const int nmine = w0 < c1 ? (c1 - w0 + kNW - 1) / kNW : 0;
     const int nunits = 4 * nmine;
-    uint8_t* my_ring = ring + warp * kRing * SL::kStride;
-    uint64_t* my_bars = bars + warp * kRing;
 
+    uint8_t* my_ring = smem_raw + SM::kRing0 + warp * kRing * SL::kStride;
+    uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem_raw + SM::kBars) + warp * kRing;
+    float* wq = reinterpret_cast<float*>(smem_raw + SM::kQ) + warp * GP * D;       // [GP][D]
+    float* wqs = reinterpret_cast<float*>(smem_raw + SM::kQs) + warp * GP * kQS;    // [GP][kQS]
+    float* wqsc = reinterpret_cast<float*>(smem_raw + SM::kQsc) + warp * GP;        // [GP]
+
+    if (lane < kRing) mbar_init(&my_bars[lane], 1);
+    fence_mbar_init();
+    __syncwarp();
+
+    // The units are issued strictly in order; the block of the next unit to
+    // issue is kept as a (pair, block) cursor instead of dividing per unit.
+    int iss_pair = nmine > 0 ? w0 / nbq : 0;
+    int iss_blk = nmine > 0 ? w0 - iss_pair * nbq : 0;
     auto issue = [&](int u) {
-        const int blk = blk_begin + warp + kNW * (u >> 2);
+        const int pair = iss_pair, blk = iss_blk;
         const int ten = u & 1;
         const int half = (u >> 1) & 1;
         uint8_t* slot = my_ring + (u % kRing) * SL::kStride;
         uint64_t* bar = &my_bars[u % kRing];
-        const size_t row0 = (size_t)bh * a.cap + (size_t)blk * kT + (size_t)half * kUT;
-        const size_t bi = ((size_t)bh * nb_cap + blk) * D;
+        const size_t row0 = (size_t)pair * a.cap + (size_t)blk * kT + (size_t)half * kUT;
+        const size_t bi = ((size_t)pair * nb_cap + blk) * D;
         mbar_expect_tx(bar, half ? SL::kBytesHi : SL::kBytesLo);
         bulk_load(slot + SL::kCodes, (ten ? a.codes[1] : a.codes[0]) + row0 * SL::kRB, kUT * SL::kRB, bar);
         bulk_load(slot + SL::kTok, (ten ? a.tok[1] : a.tok[0]) + row0 * SL::kNtok, kUT * SL::kNtok * 2, bar);
@@ -405,9 +419,17 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
             if (MODE == kNsn) bulk_load(slot + SL::kOff, (ten ? a.off[1] : a.off[0]) + bi, D * 2, bar);
         }
     };
+    // advance the cursor past unit u (every lane keeps the same cursor)
+    auto advance = [&](int u) {
+        if ((u & 3) == 3) {
+            iss_blk += kNW;
+            while (iss_blk >= nbq) { iss_blk -= nbq; ++iss_pair; }
+        }
+    };
     int issued = min(kRing, nunits);
-    if (lane == 0) {
-        for (int u = 0; u < issued; ++u) issue(u);
+    for (int u = 0; u < issued; ++u) {
+        if (lane == 0) issue(u);
+        advance(u);
     }
     int waited = 0;
     bool ok = true;
@@ -424,353 +446,550 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                 fence_proxy_async_smem();
                 issue(u + kRing);
             }
+            advance(u + kRing);
             issued = u + kRing + 1;
         }
     };
 
-    // ---- persistent per-thread state: heads 4n + t, channels [16g, 16g + 16)
-    // Softmax weights are taken against a reference max m_ref that only moves
-    // when a tile's logit exceeds it by more than kTau (log2 units), so that
-    // p <= 2^kTau and most tiles need no rescale.
-    constexpr float kTau = 8.0f;
-    float m_ref[NT], l_run[NT];
-    float acc[NT][16], acco[NT][16];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        m_ref[n] = -INFINITY;
-        l_run[n] = 0.0f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) { acc[n][k] = 0.0f; acco[n][k] = 0.0f; }
-    }
-    float kcol[NT];  // 1 / (the head's power-of-two scale)
-#pragma unroll
-    for (int n = 0; n < NT; ++n) kcol[n] = 1.0f / s_qscale[4 * n + t];
-    // the B column this thread feeds in each n-tile: head 4n + g/2, part g%2
-    const bool blo = (g & 1) != 0;
     const float alpha2 = a.scale * kLog2e;
-    // token of fragment rows g and g + 8 inside a 16-token tile
+    const bool blo = (g & 1) != 0;  // B column of this thread: head 4n + g/2, part g%2
     const int tr0 = tile_tok(g), tr1 = 8 + tile_tok(g);
-    // V fragment rows 2t, 2t+1, 2t+8, 2t+9
     const int vr0 = tile_tok(2 * t), vr1 = tile_tok(2 * t + 1);
 
-    uint32_t bq[NT][16];
-    float qoK[NT];
-    __half2 sigv[8], offv[8];
-    for (int it = 0; it < nmine; ++it) {
+    int pos = 0;
+    while (pos < nmine && ok) {
+        const int x0 = w0 + pos * kNW;
+        const int pair = x0 / nbq;
+        // blocks of this warp inside the pair: x0, x0 + kNW, ... < (pair + 1) * nbq
+        const int seg = min(nmine - pos, ((pair + 1) * nbq - x0 + kNW - 1) / kNW);
+        const int b = pair / a.H, h = pair % a.H;
+        // ---- segment prologue: this pair's queries, rotated and scaled (lane owns 4 channels)
+#pragma unroll
+        for (int j = 0; j < GP; ++j) {
+            float v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int c = 4 * lane + k;
+                const float qv =
+                    (j < G) ? __half2float(a.q[((size_t)b * a.H * G + (size_t)h * G + j) * D + c]) : 0.0f;
+                wq[j * D + c] = qv;
+                v[k] = (HAD && a.signs != nullptr && a.signs[c] < 0) ? -qv : qv;
+            }
+            if constexpr (HAD) {
+                const float x0_ = v[0] + v[1], x1_ = v[0] - v[1], x2_ = v[2] + v[3], x3_ = v[2] - v[3];
+                v[0] = x0_ + x2_; v[2] = x0_ - x2_; v[1] = x1_ + x3_; v[3] = x1_ - x3_;
+#pragma unroll
+                for (int m = 1; m < 32; m <<= 1) {
+                    const bool upper = (lane & m) != 0;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
+                        v[k] = upper ? (o - v[k]) : (v[k] + o);
+                    }
+                }
+            }
+            float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+            for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            // |q'| <= amax * max(sigma) <= amax / qmax (1 + 2^-10): keep it below 2^13
+            const float bound = PCH ? amax * (1.001f / (float)QMAX) : amax;
+            const float qsc = bound > 0.0f ? pow2i(13 - ceil_log2(bound)) : 1.0f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int c = 4 * lane + k;
+                wqs[j * kQS + c + (c >> 5)] = v[k] * qsc;
+            }
+            if (lane == 0) wqsc[j] = qsc;
+        }
+        __syncwarp();
+
+        // ---- per-thread state of the segment: heads 4n + t, channels [16g, 16g + 16)
+        float m_ref[NT], l_run[NT], kcol[NT];
+        float acc[NT][16], acco[NT][16];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            m_ref[n] = -INFINITY;
+            l_run[n] = 0.0f;
+            kcol[n] = 1.0f / wqsc[4 * n + t];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) { acc[n][k] = 0.0f; acco[n][k] = 0.0f; }
+        }
+        uint32_t bq[NT][16];
+        float qoK[NT];
+        __half2 sigv[8], offv[8];
+
+        for (int it = pos; it < pos + seg; ++it) {
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            const int uk = 4 * it + 2 * half, uv = uk + 1;
-            if (!wait_unit(uk)) { ok = false; break; }
-            uint8_t* sk = my_ring + (uk % kRing) * SL::kStride;
-            if (half == 0) {
-                // B fragments: q' = qs * sigma^K as (hi, lo) fp16 parts
-                const __half* sig = reinterpret_cast<const __half*>(sk + SL::kChan) + 32 * t;
+            for (int half = 0; half < 2; ++half) {
+                const int uk = 4 * it + 2 * half, uv = uk + 1;
+                if (!wait_unit(uk)) { ok = false; break; }
+                uint8_t* sk = my_ring + (uk % kRing) * SL::kStride;
+                if (half == 0) {
+                    // B fragments: q' = qs * sigma^K as (hi, lo) fp16 parts
+                    const __half* sig = reinterpret_cast<const __half*>(sk + SL::kChan) + 32 * t;
 #pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const float* qrow = &s_qs[(4 * n + (g >> 1)) * kQS + 33 * t];
+                    for (int n = 0; n < NT; ++n) {
+                        const float* qrow = &wqs[(4 * n + (g >> 1)) * kQS + 33 * t];
 #pragma unroll
-                    for (int p = 0; p < 16; ++p) {
-                        const int ca = KUnpack<BITS>::ca(p), cb = KUnpack<BITS>::cb(p);
-                        const float fa = qrow[ca] * (PCH ? __half2float(sig[ca]) : 1.0f);
-                        const float fb = qrow[cb] * (PCH ? __half2float(sig[cb]) : 1.0f);
-                        const __half2 hh = __floats2half2_rn(fa, fb);
-                        if (blo) {
-                            const float2 hf = __half22float2(hh);
-                            bq[n][p] = cvt_h2(fa - hf.x, fb - hf.y);
-                        } else {
-                            bq[n][p] = *reinterpret_cast<const uint32_t*>(&hh);
+                        for (int p = 0; p < 16; ++p) {
+                            const int ca = KUnpack<BITS>::ca(p), cb = KUnpack<BITS>::cb(p);
+                            const float fa = qrow[ca] * (PCH ? __half2float(sig[ca]) : 1.0f);
+                            const float fb = qrow[cb] * (PCH ? __half2float(sig[cb]) : 1.0f);
+                            const __half2 hh = __floats2half2_rn(fa, fb);
+                            if (blo) {
+                                const float2 hf = __half22float2(hh);
+                                bq[n][p] = cvt_h2(fa - hf.x, fb - hf.y);
+                            } else {
+                                bq[n][p] = *reinterpret_cast<const uint32_t*>(&hh);
+                            }
+                        }
+                    }
+                    if constexpr (MODE == kNsn) {
+                        // q . o^K for head 4n + t: lanes (g) split the channels
+                        const __half2* okp = reinterpret_cast<const __half2*>(sk + SL::kOff) + 8 * g;
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) {
+                            const float* qh = &wq[(4 * n + t) * D + 16 * g];
+                            float s = 0.0f;
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                const float2 o2 = __half22float2(okp[k]);
+                                s += qh[2 * k] * o2.x + qh[2 * k + 1] * o2.y;
+                            }
+#pragma unroll
+                            for (int o = 4; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                            qoK[n] = s;
                         }
                     }
                 }
-                if constexpr (MODE == kNsn) {
-                    const __half* okp = reinterpret_cast<const __half*>(sk + SL::kOff) + 16 * g;
+                if (!wait_unit(uv)) { ok = false; break; }
+                uint8_t* sv = my_ring + (uv % kRing) * SL::kStride;
+                if (half == 0) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        sigv[k] = PCH ? reinterpret_cast<const __half2*>(sv + SL::kChan)[8 * g + k]
+                                      : __floats2half2_rn(1.f, 1.f);
+                        offv[k] = (MODE == kNsn) ? reinterpret_cast<const __half2*>(sv + SL::kOff)[8 * g + k]
+                                                 : __floats2half2_rn(0.f, 0.f);
+                    }
+                }
+                const __half* tk = reinterpret_cast<const __half*>(sk + SL::kTok);
+                const __half* tv = reinterpret_cast<const __half*>(sv + SL::kTok);
+                // power-of-two scale keeping p * nu * 2^f <= 2^13 in fp16 (p <= 2^kTau)
+                float numax = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int tok = 2 * lane + k;
+                    float v;
+                    if constexpr (MODE == kNsn) {
+                        const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
+                        v = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
+                    } else {
+                        v = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                    }
+                    numax = fmaxf(numax, v);
+                }
+#pragma unroll
+                for (int o = 16; o; o >>= 1) numax = fmaxf(numax, __shfl_xor_sync(0xffffffffu, numax, o));
+                const int fexp = numax > 0.0f ? 13 - (int)kTau - ceil_log2(numax) : 0;
+                const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
+                float dv[NT][8][4];
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) dv[n][i][k] = 0.0f;
+                float lsum[NT], bsum[NT];
+#pragma unroll
+                for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+                    // ---- scores of the tile's 16 tokens
+                    uint32_t pa[16], pb[16];
+                    KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr0) * SL::kRB, t, pa);
+                    KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr1) * SL::kRB, t, pb);
+                    float l2[NT][2];
+                    bool over = false;
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
-                        float s = 0.0f;
+                        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) s += s_q[4 * n + t][16 * g + k] * __half2float(okp[k]);
+                        for (int s = 0; s < 8; s += 2) {
+                            mma16816(d0, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], bq[n][2 * s],
+                                     bq[n][2 * s + 1]);
+                            mma16816(d1, pa[2 * s + 2], pb[2 * s + 2], pa[2 * s + 3], pb[2 * s + 3],
+                                     bq[n][2 * s + 2], bq[n][2 * s + 3]);
+                        }
 #pragma unroll
-                        for (int o = 4; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                        qoK[n] = s;
+                        for (int r = 0; r < 2; ++r) {
+                            const int tok = 16 * m4 + (r ? tr1 : tr0);
+                            const float sv_ = (d0[2 * r] + d0[2 * r + 1]) + (d1[2 * r] + d1[2 * r + 1]);
+                            float kap, add = 0.0f;
+                            if constexpr (MODE == kNsn) {
+                                const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tk)[tok]);
+                                kap = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
+                                add = s12.x * qoK[n];
+                            } else {
+                                kap = __half2float(tk[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                            }
+                            l2[n][r] = (sv_ * (kap * kcol[n]) + add) * alpha2;
+                            over |= l2[n][r] > m_ref[n] + kTau;
+                        }
                     }
-                }
-            }
-            if (!wait_unit(uv)) { ok = false; break; }
-            uint8_t* sv = my_ring + (uv % kRing) * SL::kStride;
-            if (half == 0) {
+                    // ---- rare: move the reference max up and rescale what was accumulated
+                    if (__any_sync(0xffffffffu, over)) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    sigv[k] = PCH ? reinterpret_cast<const __half2*>(sv + SL::kChan)[8 * g + k]
-                                  : __floats2half2_rn(1.f, 1.f);
-                    offv[k] = (MODE == kNsn) ? reinterpret_cast<const __half2*>(sv + SL::kOff)[8 * g + k]
-                                             : __floats2half2_rn(0.f, 0.f);
-                }
-            }
-            const __half* tk = reinterpret_cast<const __half*>(sk + SL::kTok);
-            const __half* tv = reinterpret_cast<const __half*>(sv + SL::kTok);
-            // power-of-two scale keeping p * nu * 2^f <= 2^13 in fp16 (p <= 2^kTau)
-            float numax = 0.0f;
+                        for (int n = 0; n < NT; ++n) {
+                            float mx = fmaxf(l2[n][0], l2[n][1]);
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int tok = 2 * lane + k;
-                float v;
-                if constexpr (MODE == kNsn) {
-                    const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
-                    v = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
-                } else {
-                    v = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
-                }
-                numax = fmaxf(numax, v);
-            }
+                            for (int o = 4; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                            const float mn = fmaxf(m_ref[n], mx);
+                            const float corr = fast_exp2(m_ref[n] - mn);
+                            m_ref[n] = mn;
+                            l_run[n] *= corr;
+                            lsum[n] *= corr;
+                            bsum[n] *= corr;
 #pragma unroll
-            for (int o = 16; o; o >>= 1) numax = fmaxf(numax, __shfl_xor_sync(0xffffffffu, numax, o));
-            const int fexp = numax > 0.0f ? 13 - (int)kTau - ceil_log2(numax) : 0;
-            const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
-            float dv[NT][8][4];
+                            for (int k = 0; k < 16; ++k) {
+                                acc[n][k] *= corr;
+                                if (MODE == kNsn) acco[n][k] *= corr;
+                            }
 #pragma unroll
-            for (int n = 0; n < NT; ++n)
+                            for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) dv[n][i][k] = 0.0f;
-            float lsum[NT], bsum[NT];
-#pragma unroll
-            for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
-#pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-                // ---- scores of the tile's 16 tokens
-                uint32_t pa[16], pb[16];
-                KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr0) * SL::kRB, t, pa);
-                KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr1) * SL::kRB, t, pb);
-                float l2[NT][2];
-                bool over = false;
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int s = 0; s < 8; s += 2) {
-                        mma16816(d0, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], bq[n][2 * s],
-                                 bq[n][2 * s + 1]);
-                        mma16816(d1, pa[2 * s + 2], pb[2 * s + 2], pa[2 * s + 3], pb[2 * s + 3], bq[n][2 * s + 2],
-                                 bq[n][2 * s + 3]);
+                                for (int k = 0; k < 4; ++k) dv[n][i][k] *= corr;
+                        }
                     }
+                    // ---- P' = p * nu (scaled), as (hi, lo) rows, moved into the B layout
+                    uint32_t bp[NT][2];
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
                         const int tok = 16 * m4 + (r ? tr1 : tr0);
-                        const float sv_ = (d0[2 * r] + d0[2 * r + 1]) + (d1[2 * r] + d1[2 * r + 1]);
-                        float kap, add = 0.0f;
+                        float nu, s1o = 0.0f;
                         if constexpr (MODE == kNsn) {
-                            const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tk)[tok]);
-                            kap = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
-                            add = s12.x * qoK[n];
+                            const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
+                            s1o = s12.x;
+                            nu = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
                         } else {
-                            kap = __half2float(tk[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                            nu = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
                         }
-                        l2[n][r] = (sv_ * (kap * kcol[n]) + add) * alpha2;
-                        over |= l2[n][r] > m_ref[n] + kTau;
-                    }
-                }
-                // ---- rare: move the reference max up and rescale what was accumulated
-                if (__any_sync(0xffffffffu, over)) {
+                        nu *= pscale;
 #pragma unroll
-                    for (int n = 0; n < NT; ++n) {
-                        float mx = fmaxf(l2[n][0], l2[n][1]);
-#pragma unroll
-                        for (int o = 4; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                        const float mn = fmaxf(m_ref[n], mx);
-                        const float corr = fast_exp2(m_ref[n] - mn);
-                        m_ref[n] = mn;
-                        l_run[n] *= corr;
-                        lsum[n] *= corr;
-                        bsum[n] *= corr;
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            acc[n][k] *= corr;
-                            if (MODE == kNsn) acco[n][k] *= corr;
+                        for (int n = 0; n < NT; ++n) {
+                            const float p = fast_exp2(l2[n][r] - m_ref[n]);
+                            lsum[n] += p;
+                            if constexpr (MODE == kNsn) bsum[n] += p * s1o;
+                            bp[n][r] = movmatrix_t(split_h2(p * nu));
                         }
+                    }
+                    // ---- values
+                    uint32_t va[16], vb[16];
+                    const uint8_t* vbase = sv + SL::kCodes + (16 * m4) * SL::kRB;
+                    VUnpack<BITS>::run(vbase + vr0 * SL::kRB, vbase + vr1 * SL::kRB, g, va);
+                    VUnpack<BITS>::run(vbase + (8 + vr0) * SL::kRB, vbase + (8 + vr1) * SL::kRB, g, vb);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
+                    for (int tc = 0; tc < 8; ++tc) {
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) dv[n][i][k] *= corr;
+                        for (int n = 0; n < NT; ++n)
+                            mma16816(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1], bp[n][0],
+                                     bp[n][1]);
                     }
                 }
-                // ---- P' = p * nu (scaled), as (hi, lo) rows, moved into the B layout
-                uint32_t bp[NT][2];
+                release(uk);
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int tok = 16 * m4 + (r ? tr1 : tr0);
-                    float nu, s1o = 0.0f;
-                    if constexpr (MODE == kNsn) {
-                        const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
-                        s1o = s12.x;
-                        nu = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
-                    } else {
-                        nu = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
-                    }
-                    nu *= pscale;
-#pragma unroll
-                    for (int n = 0; n < NT; ++n) {
-                        const float p = fast_exp2(l2[n][r] - m_ref[n]);
-                        lsum[n] += p;
-                        if constexpr (MODE == kNsn) bsum[n] += p * s1o;
-                        bp[n][r] = movmatrix_t(split_h2(p * nu));
-                    }
-                }
-                // ---- values
-                uint32_t va[16], vb[16];
-                const uint8_t* vbase = sv + SL::kCodes + (16 * m4) * SL::kRB;
-                VUnpack<BITS>::run(vbase + vr0 * SL::kRB, vbase + vr1 * SL::kRB, g, va);
-                VUnpack<BITS>::run(vbase + (8 + vr0) * SL::kRB, vbase + (8 + vr1) * SL::kRB, g, vb);
+                for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
+                // unit epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f
 #pragma unroll
                 for (int tc = 0; tc < 8; ++tc) {
+                    const float2 sg = __half22float2(sigv[tc]);
+                    const float s0 = sg.x * pinv, s1_ = sg.y * pinv;
 #pragma unroll
-                    for (int n = 0; n < NT; ++n)
-                        mma16816(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1], bp[n][0], bp[n][1]);
-                }
-            }
-            release(uk);
-#pragma unroll
-            for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
-            // unit epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f
-#pragma unroll
-            for (int tc = 0; tc < 8; ++tc) {
-                const float2 sg = __half22float2(sigv[tc]);
-                const float s0 = sg.x * pinv, s1_ = sg.y * pinv;
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    acc[n][2 * tc] += (dv[n][tc][0] + dv[n][tc][1]) * s0;
-                    acc[n][2 * tc + 1] += (dv[n][tc][2] + dv[n][tc][3]) * s1_;
-                }
-            }
-            if constexpr (MODE == kNsn) {
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-#pragma unroll
-                    for (int o = 4; o < 32; o <<= 1) bsum[n] += __shfl_xor_sync(0xffffffffu, bsum[n], o);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float2 ov = __half22float2(offv[k]);
-                        acco[n][2 * k] += bsum[n] * ov.x;
-                        acco[n][2 * k + 1] += bsum[n] * ov.y;
+                    for (int n = 0; n < NT; ++n) {
+                        acc[n][2 * tc] += (dv[n][tc][0] + dv[n][tc][1]) * s0;
+                        acc[n][2 * tc + 1] += (dv[n][tc][2] + dv[n][tc][3]) * s1_;
                     }
                 }
+                if constexpr (MODE == kNsn) {
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+#pragma unroll
+                        for (int o = 4; o < 32; o <<= 1) bsum[n] += __shfl_xor_sync(0xffffffffu, bsum[n], o);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const float2 ov = __half22float2(offv[k]);
+                            acco[n][2 * k] += bsum[n] * ov.x;
+                            acco[n][2 * k + 1] += bsum[n] * ov.y;
+                        }
+                    }
+                }
+                release(uv);
             }
-            release(uv);
+            if (!ok) break;
         }
         if (!ok) break;
-    }
-    float m_run[NT];
+
+        // ---- segment epilogue: the partial of (this warp, pair)
 #pragma unroll
-    for (int n = 0; n < NT; ++n) m_run[n] = m_ref[n];
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) l_run[n] += __shfl_xor_sync(0xffffffffu, l_run[n], o);
+        constexpr int PS = part_stride<D>();
+        float* pp = a.part + ((size_t)part_slot(cta, warp, pair) * G) * PS;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int head = 4 * n + t;
+            if (head < G) {
+                float* pj = pp + (size_t)head * PS;
+                if (g == 0) *reinterpret_cast<float4*>(pj) = make_float4(m_ref[n], l_run[n], 0.0f, 0.0f);
+#pragma unroll
+                for (int k = 0; k < 16; k += 4) {
+                    *reinterpret_cast<float4*>(pj + 4 + 16 * g + k) =
+                        make_float4(acc[n][k], acc[n][k + 1], acc[n][k + 2], acc[n][k + 3]);
+                    *reinterpret_cast<float4*>(pj + 4 + D + 16 * g + k) =
+                        make_float4(acco[n][k], acco[n][k + 1], acco[n][k + 2], acco[n][k + 3]);
+                }
+            }
+        }
+        __syncwarp();
+        pos += seg;
+    }
     if (!ok) {
         // give the copies still in flight a bounded time to land before the
-        // shared memory is reused; the results of this call are void
+        // CTA exits; the results of this call are void
         if (lane == 0) report_error(kErrBarrierTimeout);
         for (int u = waited; u < issued; ++u) mbar_wait(&my_bars[u % kRing], (u / kRing) & 1, 1u << 20);
     }
     __syncwarp();
-    if (lane == 0) {
-        for (int i = 0; i < kRing; ++i) mbar_inval(&my_bars[i]);
-    }
+    if (lane < kRing) mbar_inval(&my_bars[lane]);
+}
 
-    // ---- merge: warps -> shared memory -> one partial per CTA
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) l_run[n] += __shfl_xor_sync(0xffffffffu, l_run[n], o);
-    __syncthreads();  // every warp is done with its ring; reuse it for the merge
-    float* mw = reinterpret_cast<float*>(smem_raw);   // [kNW][kGMax] running max
-    float* lw = mw + kNW * kGMax;                     // [kNW][kGMax] sums
-    float* aw = lw + kNW * kGMax;                     // [kNW][kGMax][D] code-term accumulators
-    float* ow = aw + kNW * kGMax * D;                 // [kNW][kGMax][D] original-domain accumulators
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        const int head = 4 * n + t;
-        if (g == 0) {
-            mw[warp * kGMax + head] = m_run[n];
-            lw[warp * kGMax + head] = l_run[n];
-        }
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            aw[(warp * kGMax + head) * D + 16 * g + k] = acc[n][k];
-            ow[(warp * kGMax + head) * D + 16 * g + k] = (MODE == kNsn) ? acco[n][k] : 0.0f;
-        }
-    }
-    __syncthreads();
+template <int D>
+__host__ __device__ constexpr int combine_smem_bytes() {
+    return kT * D * 2;  // the residual value rows, fp16
+}
 
-    // residual tokens (fp16), handled by the last split on CUDA cores
-    float* pp = a.part + ((size_t)bh * a.nsplit + split) * G * (2 + 2 * D);
-    const bool do_res = (split == a.nsplit - 1) && a.rlen > 0;
-    float* rl = ow + kNW * kGMax * D;  // [kGMax][kT] residual logits / weights
-    float* rm = rl + kGMax * kT;       // [kGMax] residual max, [kGMax] sum
-    if (do_res) {
-        const __half* rk = a.resid[0] + (size_t)bh * kT * D;
-        // warp w scores tokens w, w + kNW, ...; lanes split the channels
-        for (int tr = warp; tr < kT; tr += kNW) {
-            float x[4];
-            if (tr < a.rlen) {
-                const float2 x01 = __half22float2(reinterpret_cast<const __half2*>(rk + (size_t)tr * D)[2 * lane]);
-                const float2 x23 = __half22float2(reinterpret_cast<const __half2*>(rk + (size_t)tr * D)[2 * lane + 1]);
-                x[0] = x01.x; x[1] = x01.y; x[2] = x23.x; x[3] = x23.y;
-            }
-            for (int j = 0; j < G; ++j) {
-                float s = -INFINITY;
-                if (tr < a.rlen) {
-                    s = 0.0f;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) s += s_q[j][4 * lane + k] * x[k];
-#pragma unroll
-                    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                    s *= alpha2;
-                }
-                if (lane == 0) rl[j * kT + tr] = s;
-            }
-        }
-        __syncthreads();
-        for (int j = warp; j < G; j += kNW) {
+// Merge the partials of one (batch, kv head) pair with its fp16 residual
+// tokens; inverse rotation of the code term; division by the softmax sum.
+//
+// The residual part needs nothing from the decode kernel and runs first:
+// the residual value rows are copied to shared memory (cp.async) while the
+// logits are formed one token per thread from global memory; the residual
+// tokens are merged as the first softmax chunk.  Then the kernel waits for
+// the decode kernel and merges the (CTA, warp) partials that meet the pair,
+// 128 candidates per chunk: thread i tests candidate i and publishes its
+// (m, l) per head; per-head weights go through shared memory; each thread
+// (one channel) then reads the accumulators of 4 candidates x GP heads per
+// round with independent predicated loads.
+template <int D, bool HAD, int GP>
+__global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
+    static_assert(D == 128, "one channel per thread");
+    constexpr float kLog2e = 1.4426950408889634f;
+    constexpr int PS = part_stride<D>();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int pair = blockIdx.x;
+    const int G = a.G;  // <= GP
+    const int rlen = a.rlen;
+    const int b = pair / a.H, h = pair % a.H;
+    extern __shared__ __align__(16) uint8_t comb_raw[];
+    __half* s_rv = reinterpret_cast<__half*>(comb_raw);  // [kT][D]
+    __shared__ float s_q[GP][D];
+    __shared__ float s_pm[GP][128], s_pl[GP][128];  // candidate m, then weight; l
+    __shared__ int s_slot[128];
+    __shared__ float s_M[GP], s_L[GP], s_f[GP];
+    __shared__ float s_a[GP][D];
+    const float alpha2 = a.scale * kLog2e;
+    const int c = tid;
+
+    if (rlen > 0) {
+        const uint8_t* rv = reinterpret_cast<const uint8_t*>(a.resid[1] + (size_t)pair * kT * D);
+        const int nchunk = rlen * (D * 2 / 16);
+        for (int i = tid; i < nchunk; i += 128) cp_async16(reinterpret_cast<uint8_t*>(s_rv) + 16 * i, rv + 16 * i);
+    }
+    for (int i = tid; i < G * D; i += 128) {
+        const int j = i / D, cc = i % D;
+        s_q[j][cc] = __half2float(a.q[((size_t)b * a.H * G + (size_t)h * G + j) * D + cc]);
+    }
+    if (tid < GP) { s_M[tid] = -INFINITY; s_L[tid] = 0.0f; s_f[tid] = 0.0f; }
+
+    // merge one chunk of per-head candidate (m, l) published in s_pm / s_pl:
+    // warp w handles heads w, w + 4; weights replace m; s_f gets the rescale
+    auto merge_chunk = [&](int n) {
+        for (int j = warp; j < G; j += 4) {
             float mx = -INFINITY;
-            for (int i = lane; i < kT; i += 32) mx = fmaxf(mx, rl[j * kT + i]);
+            for (int i = lane; i < n; i += 32) mx = fmaxf(mx, s_pm[j][i]);
 #pragma unroll
             for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            float sm = 0.0f;
-            for (int i = lane; i < kT; i += 32) {
-                const float p = (rl[j * kT + i] == -INFINITY) ? 0.0f : fast_exp2(rl[j * kT + i] - mx);
-                rl[j * kT + i] = p;
-                sm += p;
+            const float Mo = s_M[j], Mn = fmaxf(Mo, mx);
+            float ls = 0.0f;
+            for (int i = lane; i < n; i += 32) {
+                const float wt = (s_pm[j][i] == -INFINITY) ? 0.0f : exp2f(s_pm[j][i] - Mn);
+                s_pm[j][i] = wt;
+                ls += wt * s_pl[j][i];
             }
 #pragma unroll
-            for (int o = 16; o; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
-            if (lane == 0) { rm[j] = mx; rm[kGMax + j] = sm; }
+            for (int o = 16; o; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            if (lane == 0) {
+                const float f = (Mo == -INFINITY) ? 0.0f : exp2f(Mo - Mn);
+                s_f[j] = f;
+                s_L[j] = s_L[j] * f + ls;
+                s_M[j] = Mn;
+            }
+        }
+    };
+
+    float A[GP], AO[GP];
+#pragma unroll
+    for (int j = 0; j < GP; ++j) { A[j] = 0.0f; AO[j] = 0.0f; }
+    __syncthreads();
+
+    // ---- residual tokens (independent of the decode kernel)
+    if (rlen > 0) {
+        const __half* rk = a.resid[0] + (size_t)pair * kT * D;
+        float sdot[GP];
+#pragma unroll
+        for (int j = 0; j < GP; ++j) sdot[j] = 0.0f;
+        if (tid < rlen) {
+            const uint4* row = reinterpret_cast<const uint4*>(rk + (size_t)tid * D);
+#pragma unroll 4
+            for (int k8 = 0; k8 < D / 8; ++k8) {
+                const uint4 raw = row[k8];
+                const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = __half22float2(hp[e]);
+#pragma unroll
+                    for (int j = 0; j < GP; ++j)
+                        if (j < G) sdot[j] += s_q[j][8 * k8 + 2 * e] * x.x + s_q[j][8 * k8 + 2 * e + 1] * x.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < GP; ++j) {
+            if (j < G) {
+                s_pm[j][tid] = (tid < rlen) ? sdot[j] * alpha2 : -INFINITY;
+                s_pl[j][tid] = 1.0f;
+            }
+        }
+        __syncthreads();
+        merge_chunk(rlen);
+        cp_async_wait_all();
+        __syncthreads();
+#pragma unroll 4
+        for (int t = 0; t < rlen; ++t) {
+            const float v = __half2float(s_rv[t * D + c]);
+#pragma unroll
+            for (int j = 0; j < GP; ++j)
+                if (j < G) AO[j] += s_pm[j][t] * v;
+        }
+        __syncthreads();  // s_pm is reused below
+    }
+
+    // ---- partials of the decode kernel
+    grid_dep_wait();
+    const int nctas = (int)(a.nwarps / kNW);
+    int c_first = 0, c_last = -1;
+    const int px0 = pair * a.nbq, px1 = px0 + a.nbq;  // the pair's blocks [px0, px1)
+    const CtaSplit split(a.work > 0 ? a.work : 1, nctas > 0 ? nctas : 1);
+    if (a.work > 0 && a.nbq > 0) {
+        c_first = split.cta_of(px0);
+        c_last = split.cta_of(px1 - 1);
+    }
+    // warp w of CTA c holds a partial for this pair iff one of its blocks
+    // (start(c) + w + kNW i) lies in the pair
+    auto has_part = [&](int cta, int w) {
+        const int cs = split.start(cta), ce = split.start(cta + 1);
+        const int lo = max(cs, px0), hi = min(ce, px1);
+        if (hi <= lo) return false;
+        const int first = lo + ((w - (lo - cs)) % kNW + kNW) % kNW;  // first block of warp w at or after lo
+        return first < hi;
+    };
+    const float* pbase = a.part + (size_t)part_slot(0, 0, pair) * G * PS;
+    const int ncand = (c_last - c_first + 1) * kNW;
+    for (int base = 0; base < ncand; base += 128) {
+        {
+            const int i = base + tid;
+            const bool valid = i < ncand && has_part(c_first + i / kNW, i % kNW);
+            const int off = valid ? (int)(part_slot(c_first + i / kNW, i % kNW, pair) - part_slot(0, 0, pair)) : -1;
+            s_slot[tid] = off;
+            for (int j = 0; j < G; ++j) {
+                float m = -INFINITY, l = 0.0f;
+                if (valid) {
+                    const float2 ml = *reinterpret_cast<const float2*>(pbase + ((size_t)off * G + j) * PS);
+                    m = ml.x;
+                    l = ml.y;
+                }
+                s_pm[j][tid] = m;
+                s_pl[j][tid] = l;
+            }
+        }
+        __syncthreads();
+        const int n = min(128, ncand - base);
+        merge_chunk(n);
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < GP; ++j) {
+            if (j < G) { A[j] *= s_f[j]; AO[j] *= s_f[j]; }
+        }
+        for (int i0 = 0; i0 < n; i0 += 4) {
+            float av[4][GP], aov[4][GP], wt[4][GP];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int o = (i0 + k < n) ? s_slot[i0 + k] : -1;
+                const float* pk = pbase + (size_t)(o < 0 ? 0 : o) * G * PS;
+#pragma unroll
+                for (int j = 0; j < GP; ++j) {
+                    const bool use = o >= 0 && j < G;
+                    av[k][j] = use ? pk[(size_t)j * PS + 4 + c] : 0.0f;
+                    aov[k][j] = use ? pk[(size_t)j * PS + 4 + D + c] : 0.0f;
+                    wt[k][j] = use ? s_pm[j][i0 + k] : 0.0f;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                for (int j = 0; j < GP; ++j) {
+                    A[j] += wt[k][j] * av[k][j];
+                    AO[j] += wt[k][j] * aov[k][j];
+                }
+            }
         }
         __syncthreads();
     }
-    // final merge of the kNW warp states (+ residual) for head j, channel c
-    const __half* rv = a.resid[1] + (size_t)bh * kT * D;
-    for (int i = tid; i < G * D; i += kNW * 32) {
-        const int j = i / D, c = i % D;
-        float M = -INFINITY;
-        for (int w = 0; w < kNW; ++w) M = fmaxf(M, mw[w * kGMax + j]);
-        if (do_res) M = fmaxf(M, rm[j]);
-        float L = 0.0f, A = 0.0f, AO = 0.0f;
-        for (int w = 0; w < kNW; ++w) {
-            const float mwj = mw[w * kGMax + j];
-            const float wt = (mwj == -INFINITY) ? 0.0f : fast_exp2(mwj - M);
-            L += wt * lw[w * kGMax + j];
-            A += wt * aw[(w * kGMax + j) * D + c];
-            AO += wt * ow[(w * kGMax + j) * D + c];
+#pragma unroll
+    for (int j = 0; j < GP; ++j)
+        if (j < G) s_a[j][c] = A[j];
+    __syncthreads();
+    if constexpr (HAD) {
+        // inverse rotation of the code term: warp w transforms heads w, w + 4 (lanes own 4 channels)
+        for (int j = warp; j < G; j += 4) {
+            float v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[k] = s_a[j][4 * lane + k];
+            const float x0 = v[0] + v[1], x1 = v[0] - v[1], x2 = v[2] + v[3], x3 = v[2] - v[3];
+            v[0] = x0 + x2; v[2] = x0 - x2; v[1] = x1 + x3; v[3] = x1 - x3;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const bool upper = (lane & m) != 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
+                    v[k] = upper ? (o - v[k]) : (v[k] + o);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int cc = 4 * lane + k;
+                s_a[j][cc] = (a.signs != nullptr && a.signs[cc] < 0) ? -v[k] : v[k];
+            }
         }
-        if (do_res && rm[j] != -INFINITY) {
-            const float wt = fast_exp2(rm[j] - M);
-            L += wt * rm[kGMax + j];
-            float s = 0.0f;
-            for (int tr = 0; tr < a.rlen; ++tr) s += rl[j * kT + tr] * __half2float(rv[(size_t)tr * D + c]);
-            AO += wt * s;
-        }
-        float* pj = pp + (size_t)j * (2 + 2 * D);
-        // partial in natural-log units for the combine kernel
-        if (c == 0) { pj[0] = (M == -INFINITY) ? -INFINITY : M * (1.0f / kLog2e); pj[1] = L; }
-        pj[2 + c] = A;
-        pj[2 + D + c] = AO;
+        __syncthreads();
+    }
+#pragma unroll
+    for (int j = 0; j < GP; ++j) {
+        if (j >= G) continue;
+        const float L = s_L[j];
+        a.out[((size_t)b * a.H * G + (size_t)h * G + j) * D + c] = L > 0.0f ? (s_a[j][c] + AO[j]) / L : 0.0f;
     }
 }
 

@@ -33,6 +33,8 @@ struct DecodeArgs {
     float* part;       // [B*H][nsplit][G][2 + 2D]: m, l, acc[D], acc_o[D]
     const int8_t* signs;
     int H, G, cap, nbq, rlen, nsplit, bps;
+    long long work;    // tensor-core path: quantized blocks of all pairs
+    long long nwarps;  // tensor-core path: warps of the persistent grid
     float scale, rsqd, sqd;
 };
 

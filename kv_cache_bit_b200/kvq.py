@@ -148,7 +148,7 @@ def kvq_decode_attention_noalloc(cfg: "Config", cache: "KVCache", q, q_heads: in
                                             _ptr(out), _stream(stream)), "kvq_decode_attention_noalloc")
 
 
-NOALLOC_SCRATCH_BYTES = 8 << 20
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def kvq_dequantize(cfg: "Config", cache: "KVCache", tensor: int, t0: int, ntok: int, out, stream=None):
