@@ -121,22 +121,22 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle sample
 
-def run_oracle_sample(w, mode, bits, pairs, threads):
+def run_oracle_sample(w, mode, bits, pairs, threads, decode_seconds):
     """The CPU oracle over `pairs` (batch row, kv head) slices of the
-    workload: quantize of the prefill (K and V), then one decode attention of
-    the slices' query heads over the quantized cache (dequantize + fp64
-    attention).  Returns (decode bytes, decode seconds, quantize bytes,
-    quantize seconds)."""
+    workload: quantize of the prefill (K and V), then decode steps over the
+    quantized cache (each one dequantize + fp64 attention of the slices'
+    query heads with a fresh query) until about `decode_seconds` of decode
+    work.  Returns (bytes, seconds, decode steps, quantize seconds): the
+    algorithmic bytes of the quantize and of every decode step, with the
+    same accounting as the GPU path."""
     import oracle
     names, seeded = synth.MODES[mode]
     flags = flags_of(mode)
     cfg = oracle.Cfg(d=w.d, bits=bits, flags=flags,
                      signs=oracle.make_signs(synth.SIGN_SEED, w.d) if seeded else None)
     G = w.Hq // w.Hkv
-    # sample slices: the first `pairs` kv heads of batch row 0 (more rows if needed)
     ws = w.scaled(B=max(1, (pairs + w.Hkv - 1) // w.Hkv))
     K, V = synth.kv(ws)
-    q = synth.queries(ws)
     Kb = K.reshape(-1, 1, w.S, w.d)[:pairs]
     Vb = V.reshape(-1, 1, w.S, w.d)[:pairs]
     k16 = np.ascontiguousarray(Kb).view(np.uint16)
@@ -145,15 +145,32 @@ def run_oracle_sample(w, mode, bits, pairs, threads):
     ck = oracle.quantize(cfg, k16, threads=threads)
     cv = oracle.quantize(cfg, v16, threads=threads)
     tq = time.perf_counter() - t0
-    qh = q.reshape(-1, G, w.d)[:pairs]                      # [pairs, G, d]
-    t0 = time.perf_counter()
-    kh, _ = oracle.dequantize(cfg, ck, 0, w.S, threads)
-    vh, _ = oracle.dequantize(cfg, cv, 0, w.S, threads)
-    oracle.attention(np.ascontiguousarray(qh).view(np.uint16).reshape(pairs, G, w.d), kh, vh, None, threads)
-    td = time.perf_counter() - t0
-    bq = accounting.quantize_bytes(w.d, bits, flags, pairs, 1, w.S)
-    bd = accounting.decode_bytes(w.d, bits, flags, pairs, 1, G, w.S)
-    return bd, td, bq, tq
+    qsteps = synth.queries(ws, steps=256)
+    td, n = 0.0, 0
+    while n < 256 and (n == 0 or td < decode_seconds):
+        qh = qsteps[n].reshape(-1, G, w.d)[:pairs]          # [pairs, G, d]
+        t0 = time.perf_counter()
+        kh, _ = oracle.dequantize(cfg, ck, 0, w.S, threads)
+        vh, _ = oracle.dequantize(cfg, cv, 0, w.S, threads)
+        oracle.attention(np.ascontiguousarray(qh).view(np.uint16).reshape(pairs, G, w.d), kh, vh, None, threads)
+        td += time.perf_counter() - t0
+        n += 1
+    nbytes = (accounting.quantize_bytes(w.d, bits, flags, pairs, 1, w.S)
+              + n * accounting.decode_bytes(w.d, bits, flags, pairs, 1, G, w.S))
+    return nbytes, tq + td, n, tq
+
+
+def oracle_sample_text(w, pairs, n, secs):
+    return (f"{pairs} (batch row, kv head) slices of the {WORKLOAD} workload ({w.S} prefilled tokens, "
+            f"{w.Hq // w.Hkv} query heads each): oracle quantize of the prefill + {n} decode steps "
+            f"(dequantize + fp64 attention), {secs:.1f} s")
+
+
+def bench_config(w, bits, world):
+    return {"workload": WORKLOAD, "mode": MODE, "bits": bits, "batch": w.B, "q_heads": w.Hq,
+            "kv_heads": w.Hkv, "head_dim": w.d, "seq_len": w.S, "streamed": w.stream,
+            "l2": "inputs larger than L2 (packed cache 604 MB, fp16 prefill 2 GiB)",
+            "parallelism": f"weak x{world} (independent batches, no collective)"}
 
 
 def host_cores() -> int:
@@ -169,24 +186,23 @@ def run_reference(args, rank: int, world: int):
     if rank != 0:
         return 0
     w = synth.WORKLOADS[WORKLOAD]
-    threads = host_cores()
-    pairs = 4
+    pairs = max(1, min(host_cores(), 32))
+    threads = pairs
     for _ in range(args.warmup):
-        run_oracle_sample(w, MODE, BITS, pairs, threads)
-    tot_b, tot_s = 0.0, 0.0
+        run_oracle_sample(w, MODE, BITS, pairs, threads, 1.0)
+    tot_b, tot_s, tot_n = 0.0, 0.0, 0
     for _ in range(args.steps):
-        bd, td, bq, tq = run_oracle_sample(w, MODE, BITS, pairs, threads)
-        tot_b += bd
-        tot_s += td
+        nb, secs, n, _ = run_oracle_sample(w, MODE, BITS, pairs, threads, 4.0)
+        tot_b += nb
+        tot_s += secs
+        tot_n += n
     gbs = tot_b / tot_s / 1e9
-    sample = (f"{pairs} (batch row, kv head) slices of the {WORKLOAD} workload per step "
-              f"({w.S} tokens, {w.Hq // w.Hkv} query heads each): oracle dequantize + fp64 attention")
+    sample = oracle_sample_text(w, pairs, tot_n, tot_s) + f" over {args.steps} steps"
     line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "mode": MODE, "bits": BITS, "batch": w.B, "q_heads": w.Hq,
-                       "kv_heads": w.Hkv, "head_dim": w.d, "seq_len": w.S, "streamed": w.stream},
+            "config": bench_config(w, BITS, world),
             "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -307,10 +323,7 @@ def run_ours(args, rank: int, world: int):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "mode": MODE, "bits": BITS, "batch": w.B, "q_heads": w.Hq,
-                   "kv_heads": w.Hkv, "head_dim": w.d, "seq_len": w.S, "streamed": n_stream,
-                   "l2": "inputs larger than L2 (packed cache 604 MB, fp16 prefill 2 GiB)",
-                   "parallelism": f"weak x{world} (independent batches, no collective)"},
+        "config": bench_config(w, BITS, world),
         "decode": {"gbs": dec_gbs, "frac_of_hbm": dec_gbs / peak, "us_per_call": dec_avg_s * 1e6,
                    "tokens_per_s": world * w.B / dec_avg_s, "bytes_per_call": dec_avg_bytes},
         "quantize": {"gbs": q_gbs, "frac_of_hbm": q_gbs / peak, "us_per_call": q_avg_s * 1e6,
@@ -324,11 +337,10 @@ def run_ours(args, rank: int, world: int):
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
-        bd, td, bq, tq = run_oracle_sample(w, MODE, BITS, 4, host_cores())
-        line["cpu_baseline"] = {"value": bd / td / 1e9, "unit": "GB/s", "cores": host_cores(), "kind": "oracle",
-                                "sample": f"4 (batch row, kv head) slices x {w.S} tokens, {G} query heads: "
-                                          f"oracle dequantize + fp64 attention ({td:.1f} s); "
-                                          f"quantize {bq / tq / 1e9:.3f} GB/s ({tq:.1f} s)"}
+        pairs = max(1, min(host_cores(), 32))
+        nb, secs, n, _ = run_oracle_sample(w, MODE, BITS, pairs, pairs, 12.0)
+        line["cpu_baseline"] = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": pairs, "kind": "oracle",
+                                "sample": oracle_sample_text(w, pairs, n, secs)}
     print(json.dumps(line), flush=True)
     return 0
 
