@@ -771,21 +771,22 @@ __host__ __device__ constexpr int combine_smem_bytes() {
 
 // Merge the partials of one (batch, kv head) pair with its fp16 residual
 // tokens; inverse rotation of the code term; division by the softmax sum.
+// Thread c owns output channel c of every query head.
 //
-// The residual part needs nothing from the decode kernel and runs first:
-// the residual value rows are copied to shared memory (cp.async) while the
-// logits are formed one token per thread from global memory; the residual
-// tokens are merged as the first softmax chunk.  Then the kernel waits for
-// the decode kernel and merges the (CTA, warp) partials that meet the pair,
-// 128 candidates per chunk: thread i tests candidate i and publishes its
-// (m, l) per head; per-head weights go through shared memory; each thread
-// (one channel) then reads the accumulators of 4 candidates x GP heads per
-// round with independent predicated loads.
+// The kernel is built to keep its chain of dependent memory round trips
+// short.  Before waiting for the decode kernel (programmatic dependent
+// launch) it loads the queries, the rotation signs and all residual keys at
+// once, copies the residual value rows to shared memory with cp.async, and
+// merges the residual tokens as the first softmax chunk.  After the wait,
+// thread i fetches (m, l) of candidate (CTA, warp) partial i for every head;
+// the accumulators of the first KB candidates are requested before the
+// per-head weights are formed, so their latency overlaps that work.
 template <int D, bool HAD, int GP>
 __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "one channel per thread");
     constexpr float kLog2e = 1.4426950408889634f;
     constexpr int PS = part_stride<D>();
+    constexpr int KB = 32 / GP;  // candidates per batch of accumulator loads
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int pair = blockIdx.x;
     const int G = a.G;  // <= GP
@@ -798,19 +799,32 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     __shared__ int s_slot[128];
     __shared__ float s_M[GP], s_L[GP], s_f[GP];
     __shared__ float s_a[GP][D];
+    __shared__ float s_sg[D];
     const float alpha2 = a.scale * kLog2e;
     const int c = tid;
 
+    // ---- everything that does not depend on the decode kernel
     if (rlen > 0) {
         const uint8_t* rv = reinterpret_cast<const uint8_t*>(a.resid[1] + (size_t)pair * kT * D);
         const int nchunk = rlen * (D * 2 / 16);
         for (int i = tid; i < nchunk; i += 128) cp_async16(reinterpret_cast<uint8_t*>(s_rv) + 16 * i, rv + 16 * i);
     }
-    for (int i = tid; i < G * D; i += 128) {
-        const int j = i / D, cc = i % D;
-        s_q[j][cc] = __half2float(a.q[((size_t)b * a.H * G + (size_t)h * G + j) * D + cc]);
+    {
+        const __half* qp = a.q + ((size_t)b * a.H * G + (size_t)h * G) * D;
+        float qv[GP];
+#pragma unroll
+        for (int j = 0; j < GP; ++j) qv[j] = (j < G) ? __half2float(qp[(size_t)j * D + c]) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < GP; ++j) s_q[j][c] = qv[j];
+        if constexpr (HAD) s_sg[c] = (a.signs != nullptr && a.signs[c] < 0) ? -1.0f : 1.0f;
     }
     if (tid < GP) { s_M[tid] = -INFINITY; s_L[tid] = 0.0f; s_f[tid] = 0.0f; }
+    uint4 krow[D / 8];
+    if (tid < rlen) {
+        const uint4* row = reinterpret_cast<const uint4*>(a.resid[0] + ((size_t)pair * kT + tid) * D);
+#pragma unroll
+        for (int k8 = 0; k8 < D / 8; ++k8) krow[k8] = row[k8];
+    }
 
     // merge one chunk of per-head candidate (m, l) published in s_pm / s_pl:
     // warp w handles heads w, w + 4; weights replace m; s_f gets the rescale
@@ -843,18 +857,14 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     for (int j = 0; j < GP; ++j) { A[j] = 0.0f; AO[j] = 0.0f; }
     __syncthreads();
 
-    // ---- residual tokens (independent of the decode kernel)
     if (rlen > 0) {
-        const __half* rk = a.resid[0] + (size_t)pair * kT * D;
         float sdot[GP];
 #pragma unroll
         for (int j = 0; j < GP; ++j) sdot[j] = 0.0f;
         if (tid < rlen) {
-            const uint4* row = reinterpret_cast<const uint4*>(rk + (size_t)tid * D);
-#pragma unroll 4
+#pragma unroll
             for (int k8 = 0; k8 < D / 8; ++k8) {
-                const uint4 raw = row[k8];
-                const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+                const __half2* hp = reinterpret_cast<const __half2*>(&krow[k8]);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 x = __half22float2(hp[e]);
@@ -882,11 +892,8 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
             for (int j = 0; j < GP; ++j)
                 if (j < G) AO[j] += s_pm[j][t] * v;
         }
-        __syncthreads();  // s_pm is reused below
     }
-
-    // ---- partials of the decode kernel
-    grid_dep_wait();
+    // candidate (CTA, warp) partials of this pair: CTA ranges are contiguous
     const int nctas = (int)(a.nwarps / kNW);
     int c_first = 0, c_last = -1;
     const int px0 = pair * a.nbq, px1 = px0 + a.nbq;  // the pair's blocks [px0, px1)
@@ -906,35 +913,33 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     };
     const float* pbase = a.part + (size_t)part_slot(0, 0, pair) * G * PS;
     const int ncand = (c_last - c_first + 1) * kNW;
+    __syncthreads();  // the residual phase is done with s_pm
+
+    // ---- the decode kernel's partials
+    grid_dep_wait();
     for (int base = 0; base < ncand; base += 128) {
         {
             const int i = base + tid;
             const bool valid = i < ncand && has_part(c_first + i / kNW, i % kNW);
             const int off = valid ? (int)(part_slot(c_first + i / kNW, i % kNW, pair) - part_slot(0, 0, pair)) : -1;
             s_slot[tid] = off;
-            for (int j = 0; j < G; ++j) {
-                float m = -INFINITY, l = 0.0f;
-                if (valid) {
-                    const float2 ml = *reinterpret_cast<const float2*>(pbase + ((size_t)off * G + j) * PS);
-                    m = ml.x;
-                    l = ml.y;
-                }
-                s_pm[j][tid] = m;
-                s_pl[j][tid] = l;
+            float2 ml[GP];
+            const float* pk = pbase + (size_t)(valid ? off : 0) * G * PS;
+#pragma unroll
+            for (int j = 0; j < GP; ++j)
+                ml[j] = (valid && j < G) ? *reinterpret_cast<const float2*>(pk + (size_t)j * PS)
+                                         : make_float2(-INFINITY, 0.0f);
+#pragma unroll
+            for (int j = 0; j < GP; ++j) {
+                if (j < G) { s_pm[j][tid] = ml[j].x; s_pl[j][tid] = ml[j].y; }
             }
         }
         __syncthreads();
         const int n = min(128, ncand - base);
-        merge_chunk(n);
-        __syncthreads();
+        float av[KB][GP], aov[KB][GP];
+        auto load_batch = [&](int i0) {
 #pragma unroll
-        for (int j = 0; j < GP; ++j) {
-            if (j < G) { A[j] *= s_f[j]; AO[j] *= s_f[j]; }
-        }
-        for (int i0 = 0; i0 < n; i0 += 4) {
-            float av[4][GP], aov[4][GP], wt[4][GP];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < KB; ++k) {
                 const int o = (i0 + k < n) ? s_slot[i0 + k] : -1;
                 const float* pk = pbase + (size_t)(o < 0 ? 0 : o) * G * PS;
 #pragma unroll
@@ -942,15 +947,25 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
                     const bool use = o >= 0 && j < G;
                     av[k][j] = use ? pk[(size_t)j * PS + 4 + c] : 0.0f;
                     aov[k][j] = use ? pk[(size_t)j * PS + 4 + D + c] : 0.0f;
-                    wt[k][j] = use ? s_pm[j][i0 + k] : 0.0f;
                 }
             }
+        };
+        load_batch(0);
+        merge_chunk(n);
+        __syncthreads();
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+        for (int j = 0; j < GP; ++j) {
+            if (j < G) { A[j] *= s_f[j]; AO[j] *= s_f[j]; }
+        }
+        for (int i0 = 0; i0 < n; i0 += KB) {
+            if (i0 > 0) load_batch(i0);
+#pragma unroll
+            for (int k = 0; k < KB; ++k) {
 #pragma unroll
                 for (int j = 0; j < GP; ++j) {
-                    A[j] += wt[k][j] * av[k][j];
-                    AO[j] += wt[k][j] * aov[k][j];
+                    const float wt = (i0 + k < n && j < G) ? s_pm[j][i0 + k] : 0.0f;
+                    A[j] += wt * av[k][j];
+                    AO[j] += wt * aov[k][j];
                 }
             }
         }
@@ -978,10 +993,7 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
                 }
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int cc = 4 * lane + k;
-                s_a[j][cc] = (a.signs != nullptr && a.signs[cc] < 0) ? -v[k] : v[k];
-            }
+            for (int k = 0; k < 4; ++k) s_a[j][4 * lane + k] = v[k] * s_sg[4 * lane + k];
         }
         __syncthreads();
     }
