@@ -213,16 +213,140 @@ __device__ __forceinline__ void fwht_reg(float (&v)[D]) {
     fwht_stage<1, D>(v);
 }
 
-// Round-half-even of the exact product u * inv, clamped to [-qmax, qmax],
-// returned as the offset-binary code.  The fused multiply-add rounds the
-// exact product plus 1.5 * 2^23 once to an integer (ties to even); the
-// subtraction is exact while |u * inv| < 2^22, and larger magnitudes clamp.
-template <int QMAX>
-__device__ __forceinline__ uint32_t code_of(float u, float inv) {
-    const float kMagic = 12582912.0f;  // 1.5 * 2^23
-    float r = __fsub_rn(__fmaf_rn(u, inv, kMagic), kMagic);
-    r = fminf(fmaxf(r, -(float)QMAX), (float)QMAX);
-    return static_cast<uint32_t>(static_cast<int>(r) + QMAX + 1);
+// ---------------------------------------------------------------- packed fp32 pairs
+// sm_100 executes add/sub/mul/fma on two fp32 lanes per instruction
+// (.f32x2); every lane is rounded exactly like the scalar instruction, so
+// the packed forms change only the instruction count, never a result.  The
+// quantizer keeps a token row as D/2 pairs P[j] = (channel j, channel
+// j + D/2).
+using f2_t = unsigned long long;
+
+__device__ __forceinline__ f2_t f2_pack(float lo, float hi) {
+    f2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(f2_t x, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+__device__ __forceinline__ f2_t f2_add(f2_t a, f2_t b) {
+    f2_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2_t f2_sub(f2_t a, f2_t b) {
+    f2_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2_t f2_mul(f2_t a, f2_t b) {
+    f2_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
+    f2_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// Pairwise sum of squares over the pairs P[OFF .. OFF+N): lane 0 sums the
+// first half of the row, lane 1 the second, with the same recursive halving.
+// The volatile forms keep the depth-first order of the tree, so that the
+// squares are not all formed (and held) before the first sums.
+__device__ __forceinline__ f2_t f2_mul_ordered(f2_t a, f2_t b) {
+    f2_t r;
+    asm volatile("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2_t f2_add_ordered(f2_t a, f2_t b) {
+    f2_t r;
+    asm volatile("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+template <int OFF, int N, int H2>
+__device__ __forceinline__ f2_t pw_sumsq2(const f2_t (&P)[H2]) {
+    if constexpr (N == 1) return f2_mul_ordered(P[OFF], P[OFF]);
+    else return f2_add_ordered(pw_sumsq2<OFF, N / 2>(P), pw_sumsq2<OFF + N / 2, N / 2>(P));
+}
+
+// Pairwise sum of squares of the whole row: the top split of the halving
+// tree adds the two lanes.
+template <int H2>
+__device__ __forceinline__ float row_sumsq(const f2_t (&P)[H2]) {
+    float lo, hi;
+    f2_unpack(pw_sumsq2<0, H2>(P), lo, hi);
+    return __fadd_rn(lo, hi);
+}
+
+// Butterflies of stride S (channels j, j + S inside each half), ascending.
+template <int S, int H2>
+__device__ __forceinline__ void fwht2_stage(f2_t (&P)[H2]) {
+#pragma unroll
+    for (int i = 0; i < H2; i += 2 * S) {
+#pragma unroll
+        for (int j = 0; j < S; ++j) {
+            const f2_t a = P[i + j], b = P[i + j + S];
+            P[i + j] = f2_add(a, b);
+            P[i + j + S] = f2_sub(a, b);
+        }
+    }
+    if constexpr (2 * S < H2) fwht2_stage<2 * S, H2>(P);
+}
+
+// Unnormalized Walsh-Hadamard transform of the row, strides 1, 2, ..., D/2
+// in that order; the last stride pairs the two lanes of each P[j].
+template <int H2>
+__device__ __forceinline__ void fwht2(f2_t (&P)[H2]) {
+    fwht2_stage<1, H2>(P);
+#pragma unroll
+    for (int j = 0; j < H2; ++j) {
+        float a, b;
+        f2_unpack(P[j], a, b);
+        P[j] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+}
+
+__device__ __forceinline__ uint32_t prmt32(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Codes from the words of r = fma(u, inv, 1.5 * 2^23 + 2^(BITS-1)): for any
+// |rne(u * inv)| <= qmax the float lies in [2^23, 2^24), where its ulp is 1,
+// so the single rounding of the fused product is round-half-even of u * inv
+// (the added constant is even) and the low mantissa bits hold the
+// offset-binary code e.  cw[c] holds that word for channel c; the bits above
+// the code (bit 22 upward) never reach the low 16 bits of the sums below.
+template <int D, int BITS>
+__device__ __forceinline__ void pack_codes(const uint32_t (&cw)[D], uint32_t (&w)[RowLayout<D, BITS>::kWords]) {
+    if constexpr (BITS == 4) {
+#pragma unroll
+        for (int k = 0; k < D / 8; ++k) {
+            const uint32_t* e = cw + 8 * k;
+            const uint32_t h0 = e[0] + 16u * e[1] + 256u * e[2] + 4096u * e[3];
+            const uint32_t h1 = e[4] + 16u * e[5] + 256u * e[6] + 4096u * e[7];
+            w[k] = prmt32(h0, h1, 0x5410u);
+        }
+    } else if constexpr (BITS == 2) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+            const uint32_t* e = cw + 16 * k;
+            uint32_t h0 = 0, h1 = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                h0 += e[i] << (2 * i);
+                h1 += e[8 + i] << (2 * i);
+            }
+            w[k] = prmt32(h0, h1, 0x5410u);
+        }
+    } else {
+        uint32_t e[D];
+#pragma unroll
+        for (int c = 0; c < D; ++c) e[c] = cw[c] & 7u;
+        pack_row<D, BITS>(e, w);
+    }
 }
 
 // ---------------------------------------------------------------- the quantizer
@@ -230,13 +354,16 @@ __device__ __forceinline__ uint32_t code_of(float u, float inv) {
 // Shared-memory scratch of one quantizer CTA.
 template <int D>
 struct QuantSmem {
-    // fp32 [128][D] transpose buffer (NSN column means), swizzled by 16-byte
-    // chunk: chunk k of row t lives at chunk k ^ (t & (D/4 - 1)).
-    static constexpr int kRedFloats = kT * D;
+    // fp16 input tile: 64-channel boxes of 128 rows x 128 bytes, 16-byte
+    // chunk c of row t stored at chunk c ^ (t & 7) (the TMA 128-byte swizzle)
+    const uint8_t* tile;
+    // fp32 [128][D] transpose buffer in pair order (row t holds P[0..D/2)),
+    // 16-byte chunk k of row t stored at chunk k ^ (t & (D/4 - 1))
     float* red;
-    float* vec;        // [D] broadcast vector (means, reciprocal scales)
-    uint32_t* wmax;    // [4][D] per-warp channel maxima (float bits)
-    uint32_t* sgn;     // [D] sign masks (0 or 0x80000000) of the rotation
+    float* vec;      // [D] a per-channel vector in pair order (means, reciprocal scales)
+    float* gpart;    // [4 KB] per-token-group partial sums / maxima
+    float* tokv;     // [128] a per-token scalar (NSN 1/||x|| * sqrt(d))
+    uint32_t* sgn2;  // [D/2] fp16x2 sign masks of channels (2i, 2i+1)
 };
 
 // Output pointers of one (tensor, batch, head, block).
@@ -247,135 +374,281 @@ struct QuantOut {
     __half* off;     // [D] (NSN)
 };
 
-// Quantize the 128 token rows of one block; thread t (0..127) holds row t in
-// v[] (fp32 widened from fp16) and all 128 threads of the CTA must call this.
+template <int D>
+__device__ __forceinline__ void store_pair_row(float* red, const f2_t (&P)[D / 2], int t) {
+    constexpr int NCH = D / 4;  // 16-byte chunks per row
+    char* row = reinterpret_cast<char*>(red) + (size_t)t * D * 4;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+        const int pk = k ^ (t & (NCH - 1));
+        *reinterpret_cast<ulonglong2*>(row + pk * 16) = make_ulonglong2(P[2 * k], P[2 * k + 1]);
+    }
+}
+
+// Sign of channel c of the rotation as an fp16 sign-bit mask.
+__device__ __forceinline__ uint16_t sign16(const uint32_t* sgn2, int c) {
+    return (uint16_t)((sgn2[c >> 1] >> ((c & 1) * 16)) & 0x8000u);
+}
+
+// Offset-binary code words of one pair: lanes of fma(x, inv, kC) (see
+// pack_codes), clamped to [-qmax, qmax] when CLAMP.
+template <bool CLAMP>
+__device__ __forceinline__ void code_pair(f2_t x, f2_t inv, float kQ, float kC, uint32_t& clo, uint32_t& chi) {
+    float lo, hi;
+    f2_unpack(f2_fma(x, inv, f2_pack(kC, kC)), lo, hi);
+    if constexpr (CLAMP) {
+        lo = fminf(fmaxf(lo, kC - kQ), kC + kQ);
+        hi = fminf(fmaxf(hi, kC - kQ), kC + kQ);
+    }
+    clo = __float_as_uint(lo);
+    chi = __float_as_uint(hi);
+}
+
+// Low 16 bits of sum_i e[i] << (NB * i) for N codes of NB bits (the bits of
+// each word above bit 21 stay out of the low half, see pack_codes).
+template <int N, int NB>
+__device__ __forceinline__ uint32_t pack_half(const uint32_t* e) {
+    uint32_t h = e[0];
+#pragma unroll
+    for (int i = 1; i < N; ++i) h += e[i] << (NB * i);
+    return h;
+}
+
+// Codes of the row held in registers (reciprocal scales in pair order in
+// vec), packed group by group so that few code words are live at once.
+template <int D, int BITS, bool CLAMP>
+__device__ __forceinline__ void codes_from_regs(const f2_t (&P)[D / 2], const float* vec,
+                                                uint32_t (&w)[RowLayout<D, BITS>::kWords]) {
+    using L = RowLayout<D, BITS>;
+    constexpr int H2 = D / 2;
+    constexpr float kQ = (float)L::kQmax;
+    constexpr float kC = 12582912.0f + (float)L::kOff;
+    constexpr int GP = (BITS == 4) ? 8 : (BITS == 2 ? 16 : (H2 < 32 ? H2 : 32));
+    const f2_t* iv = reinterpret_cast<const f2_t*>(vec);
+#pragma unroll
+    for (int q = 0; q < H2 / GP; ++q) {
+        uint32_t lo[GP], hi[GP];
+#pragma unroll
+        for (int i = 0; i < GP; i += 2) {
+            const ulonglong2 r = *reinterpret_cast<const ulonglong2*>(iv + q * GP + i);
+            code_pair<CLAMP>(P[q * GP + i], r.x, kQ, kC, lo[i], hi[i]);
+            code_pair<CLAMP>(P[q * GP + i + 1], r.y, kQ, kC, lo[i + 1], hi[i + 1]);
+        }
+        if constexpr (BITS == 4) {
+            w[q] = prmt32(pack_half<4, 4>(lo), pack_half<4, 4>(lo + 4), 0x5410u);
+            w[H2 / 8 + q] = prmt32(pack_half<4, 4>(hi), pack_half<4, 4>(hi + 4), 0x5410u);
+        } else if constexpr (BITS == 2) {
+            w[q] = prmt32(pack_half<8, 2>(lo), pack_half<8, 2>(lo + 8), 0x5410u);
+            w[H2 / 16 + q] = prmt32(pack_half<8, 2>(hi), pack_half<8, 2>(hi + 8), 0x5410u);
+        } else {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const uint32_t* e = half ? hi : lo;
+                const int c0 = half * H2 + q * GP;
+#pragma unroll
+                for (int m = 0; m < GP / 16; ++m) {
+                    uint32_t v = 0;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v |= (e[16 * m + i] & 3u) << (2 * i);
+                    w[c0 / 16 + m] = v;
+                }
+                static_assert(GP == 32, "one bit-plane word per run");
+                uint32_t b = 0;
+#pragma unroll
+                for (int i = 0; i < GP; ++i) b |= ((e[i] >> 2) & 1u) << i;
+                w[D / 16 + c0 / 32] = b;
+            }
+        }
+    }
+}
+
+// Quantize the 128 token rows of one block.  Thread t (0..127) holds row t
+// as pairs P[j] = (x[j], x[j + D/2]) in fp32 (widened from fp16), with the
+// rotation signs already applied under HADAMARD; all 128 threads of the CTA
+// call this.
 //   nsep:  n = ||x||, u = H(s (.) x) * (c0 / n)
 //   NSN:   s1 = ||x|| rsqd, a = x (sqd / ||x||), o = block mean of a (fp16),
 //          b = a - o, s2 = ||b|| rsqd, u = H(s (.) b) * (c0 / ||b||)
 //   naive: u = x
 // with c0 = rsqd under HADAMARD, else 1; then sigma = fp16(max|u| / qmax)
 // per channel over the block (per token for naive) and codes
-// rne(u * (1/sigma)) clamped.
+// rne(u * (1/sigma)) clamped.  Sign flips commute exactly with every step
+// up to the rotation (means, norms, fp16 rounding are all sign-symmetric),
+// which is why they can be applied when the row is loaded; the stored
+// offsets are flipped back.
 template <int D, int BITS, int MODE, bool HAD>
-__device__ __forceinline__ void quantize_rows(float (&v)[D], const int t, const QuantSmem<D>& sm, const QuantOut& out,
-                                              const float rsqd, const float sqd) {
+__device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, const QuantSmem<D>& sm,
+                                              const QuantOut& out, const float rsqd, const float sqd) {
     using L = RowLayout<D, BITS>;
+    constexpr int H2 = D / 2;
+    constexpr int NCH = D / 4;    // 16-byte chunks (two pairs) per row
+    constexpr int TG = NCH;       // tokens per column group
+    constexpr int NG = kT / TG;   // column groups: thread t -> chunk column t % NCH, group t / NCH
+    static_assert(NG * H2 * 8 == 2048, "group partials fill 2 KB");
     const float c0 = HAD ? rsqd : 1.0f;
     float kscale = 1.0f;
+    const int kc = t % NCH, g = t / NCH;
 
     if constexpr (MODE == kNsn) {
-        const float n1 = __fsqrt_rn(pw_sumsq<0, D>(v));
+        const float n1 = __fsqrt_rn(row_sumsq<H2>(P));
         const float s1 = __fmul_rn(n1, rsqd);
         const float r1 = n1 > 0.0f ? __fdiv_rn(sqd, n1) : 0.0f;
+        sm.tokv[t] = r1;
+        const f2_t R1 = f2_pack(r1, r1);
 #pragma unroll
-        for (int c = 0; c < D; ++c) v[c] = __fmul_rn(v[c], r1);
-        // transpose through shared memory for the per-channel block means
-        constexpr int NCH = D / 4;
-#pragma unroll
-        for (int k = 0; k < NCH; ++k) {
-            const int pk = k ^ (t & (NCH - 1));
-            reinterpret_cast<float4*>(sm.red + t * D)[pk] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-        }
+        for (int j = 0; j < H2; ++j) P[j] = f2_mul(P[j], R1);
         __syncthreads();
         {
-            // thread -> (column c, token half). For D = 128 every thread sums
-            // one full column; for D = 64 two threads split the column and
-            // their halves are added last (the top split of the pairwise tree).
-            constexpr int PER = (D == 128) ? 128 : 64;
-            const int c = t % D;
-            const int tbase = (t / D) * PER;
-            float acc[8];
+            // block means of a = x * r1 straight from the fp16 tile (the
+            // unsigned values; the same products as the rows'): thread t
+            // sums the 8 channels of chunk column kc8 over the TGc tokens of
+            // group gc in the pairwise (binary-counter) order
+            constexpr int NKC = D / 8, NGC = kT / NKC, TGC = kT / NGC;
+            const int kc8 = t % NKC, gc = t / NKC;
+            const uint8_t* colp = sm.tile + (kc8 / 8) * (kT * 128);
+            const int ck = kc8 % 8;
+            f2_t acc[4][6];
 #pragma unroll
-            for (int i = 0; i < PER; ++i) {
-                const int tt = tbase + i;
-                const int pk = (c >> 2) ^ (tt & (NCH - 1));
-                float cur = sm.red[tt * D + pk * 4 + (c & 3)];
+            for (int i = 0; i < TGC; ++i) {
+                const int tt = gc * TGC + i;
+                const uint4 raw = *reinterpret_cast<const uint4*>(colp + tt * 128 + ((ck ^ (tt & 7)) << 4));
+                const float rt = sm.tokv[tt];
+                const f2_t RT = f2_pack(rt, rt);
+                const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+                f2_t cur[4];
 #pragma unroll
-                for (int l = 0; l < 7; ++l) {
-                    if ((i >> l) & 1) cur = __fadd_rn(acc[l], cur);
-                    else { acc[l] = cur; break; }
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = __half22float2(hp[e]);
+                    cur[e] = f2_mul(f2_pack(x.x, x.y), RT);
                 }
-                if (i == PER - 1) acc[7] = cur;
-            }
-            if constexpr (D == 128) {
-                const float o = __fmul_rn(acc[7], 1.0f / 128.0f);
-                const __half o16 = __float2half_rn(o);
-                out.off[c] = o16;
-                sm.vec[c] = __half2float(o16);
-            } else {
-                // halves meet in smem: lower half writes, upper half adds
-                __syncthreads();
-                if (t >= D) sm.vec[c] = acc[7];
-                __syncthreads();
-                if (t < D) {
-                    const float o = __fmul_rn(__fadd_rn(acc[7], sm.vec[c]), 1.0f / 128.0f);
-                    const __half o16 = __float2half_rn(o);
-                    out.off[c] = o16;
-                    sm.vec[c] = __half2float(o16);
+#pragma unroll
+                for (int l = 0; l < 6; ++l) {
+                    if ((i >> l) & 1) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) cur[e] = f2_add(acc[e][l], cur[e]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[e][l] = cur[e];
+                        break;
+                    }
+                }
+                if (i == TGC - 1) {
+                    f2_t* gp = reinterpret_cast<f2_t*>(sm.gpart) + (gc * D + 8 * kc8) / 2;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) gp[e] = cur[e];
                 }
             }
         }
         __syncthreads();
+        if (t < D) {
+            // the group sums meet in the top levels of the pairwise tree
+            constexpr int NGC = kT / (D / 8);
+            float g[NGC];
 #pragma unroll
-        for (int c = 0; c < D; ++c) v[c] = __fsub_rn(v[c], sm.vec[c]);
-        const float n2 = __fsqrt_rn(pw_sumsq<0, D>(v));
+            for (int k = 0; k < NGC; ++k) g[k] = sm.gpart[k * D + t];
+#pragma unroll
+            for (int w = 1; w < NGC; w *= 2) {
+#pragma unroll
+                for (int k = 0; k < NGC; k += 2 * w) g[k] = __fadd_rn(g[k], g[k + w]);
+            }
+            const __half o16 = __float2half_rn(__fmul_rn(g[0], 1.0f / 128.0f));
+            out.off[t] = o16;
+            // the rows carry the rotation's signs: subtract s_c * o there
+            float ov = __half2float(o16);
+            if constexpr (HAD) ov = sign16(sm.sgn2, t) ? -ov : ov;
+            sm.vec[2 * (t % H2) + t / H2] = ov;
+        }
+        __syncthreads();
+        const f2_t* mv = reinterpret_cast<const f2_t*>(sm.vec);
+#pragma unroll
+        for (int j = 0; j < H2; ++j) P[j] = f2_sub(P[j], mv[j]);
+        const float n2 = __fsqrt_rn(row_sumsq<H2>(P));
         const float s2 = __fmul_rn(n2, rsqd);
         kscale = n2 > 0.0f ? __fdiv_rn(c0, n2) : 0.0f;
-        __half2 sp = __halves2half2(__float2half_rn(s1), __float2half_rn(s2));
-        reinterpret_cast<__half2*>(out.tok)[t] = sp;
+        reinterpret_cast<__half2*>(out.tok)[t] = __halves2half2(__float2half_rn(s1), __float2half_rn(s2));
     } else if constexpr (MODE == kNsep) {
-        const float n = __fsqrt_rn(pw_sumsq<0, D>(v));
+        const float n = __fsqrt_rn(row_sumsq<H2>(P));
         out.tok[t] = __float2half_rn(n);
         kscale = n > 0.0f ? __fdiv_rn(c0, n) : 0.0f;
     } else {
         kscale = c0;
     }
 
-    if constexpr (HAD) {
-#pragma unroll
-        for (int c = 0; c < D; ++c) v[c] = __uint_as_float(__float_as_uint(v[c]) ^ sm.sgn[c]);
-        fwht_reg<D>(v);
-    }
+    if constexpr (HAD) fwht2<H2>(P);
     if constexpr (MODE != kNaive || HAD) {
+        const f2_t K2 = f2_pack(kscale, kscale);
 #pragma unroll
-        for (int c = 0; c < D; ++c) v[c] = __fmul_rn(v[c], kscale);
+        for (int j = 0; j < H2; ++j) P[j] = f2_mul(P[j], K2);
     }
 
-    uint32_t e[D];
+    constexpr float kQ = (float)L::kQmax;
+    constexpr float kC = 12582912.0f + (float)L::kOff;  // 1.5 * 2^23 + offset
     if constexpr (MODE == kNaive) {
+        uint32_t cw[D];
         float m = 0.0f;
 #pragma unroll
-        for (int c = 0; c < D; ++c) m = fmaxf(m, fabsf(v[c]));
-        const __half s16 = __float2half_rn(__fdiv_rn(m, (float)L::kQmax));
+        for (int j = 0; j < H2; ++j) {
+            float lo, hi;
+            f2_unpack(P[j], lo, hi);
+            m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
+        }
+        const __half s16 = __float2half_rn(__fdiv_rn(m, kQ));
         out.tok[t] = s16;
         const float sf = __half2float(s16);
         const float inv = sf > 0.0f ? __fdiv_rn(1.0f, sf) : 0.0f;
+        const f2_t I2 = f2_pack(inv, inv), C2 = f2_pack(kC, kC);
 #pragma unroll
-        for (int c = 0; c < D; ++c) e[c] = code_of<L::kQmax>(v[c], inv);
+        for (int j = 0; j < H2; ++j) {
+            float lo, hi;
+            f2_unpack(f2_fma(P[j], I2, C2), lo, hi);
+            lo = fminf(fmaxf(lo, kC - kQ), kC + kQ);
+            hi = fminf(fmaxf(hi, kC - kQ), kC + kQ);
+            cw[j] = __float_as_uint(lo);
+            cw[j + H2] = __float_as_uint(hi);
+        }
+        uint32_t w[L::kWords];
+        pack_codes<D, BITS>(cw, w);
+        store_words<L::kWords>(out.codes + (size_t)t * L::kBytes, w);
     } else {
-        // per-channel absmax over the block: warp max, then across warps
-        const int warp = t >> 5, lane = t & 31;
-#pragma unroll
-        for (int c = 0; c < D; ++c) {
-            const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[c])));
-            if (lane == (c & 31)) sm.wmax[warp * D + c] = m;
+        // per-channel absmax over the block through the transpose buffer
+        store_pair_row<D>(sm.red, P, t);
+        __syncthreads();
+        {
+            const char* base = reinterpret_cast<const char*>(sm.red) + (size_t)g * TG * D * 4;
+            float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
+#pragma unroll 4
+            for (int i = 0; i < TG; ++i) {
+                const float4 x = *reinterpret_cast<const float4*>(base + (size_t)i * D * 4 + ((kc ^ i) << 4));
+                m0 = fmaxf(m0, fabsf(x.x));
+                m1 = fmaxf(m1, fabsf(x.y));
+                m2 = fmaxf(m2, fabsf(x.z));
+                m3 = fmaxf(m3, fabsf(x.w));
+            }
+            reinterpret_cast<float4*>(sm.gpart)[g * NCH + kc] = make_float4(m0, m1, m2, m3);
         }
         __syncthreads();
+        int clamp = 0;
         if (t < D) {
-            const float m = fmaxf(fmaxf(__uint_as_float(sm.wmax[t]), __uint_as_float(sm.wmax[D + t])),
-                                  fmaxf(__uint_as_float(sm.wmax[2 * D + t]), __uint_as_float(sm.wmax[3 * D + t])));
-            const __half s16 = __float2half_rn(__fdiv_rn(m, (float)L::kQmax));
-            out.chan[t] = s16;
-            const float sf = __half2float(s16);
-            sm.vec[t] = sf > 0.0f ? __fdiv_rn(1.0f, sf) : 0.0f;
-        }
-        __syncthreads();
+            // t indexes the pair-order vector: pair t >> 1, lane t & 1
+            const int c = (t >> 1) + (t & 1) * H2;
+            float m = 0.0f;
 #pragma unroll
-        for (int c = 0; c < D; ++c) e[c] = code_of<L::kQmax>(v[c], sm.vec[c]);
+            for (int gg = 0; gg < NG; ++gg) m = fmaxf(m, sm.gpart[gg * D + t]);
+            const __half s16 = __float2half_rn(__fdiv_rn(m, kQ));
+            out.chan[c] = s16;
+            const float sf = __half2float(s16);
+            const float inv = sf > 0.0f ? __fdiv_rn(1.0f, sf) : 0.0f;
+            sm.vec[t] = inv;
+            // some |u * inv| of this channel rounds past qmax (an fp16
+            // subnormal scale): the exact sign of m * inv - (qmax + 1/2)
+            clamp = __fmaf_rn(m, inv, -(kQ + 0.5f)) >= 0.0f;
+        }
+        const int any_clamp = __syncthreads_or(clamp);
+        uint32_t w[L::kWords];
+        if (!any_clamp) codes_from_regs<D, BITS, false>(P, sm.vec, w);
+        else codes_from_regs<D, BITS, true>(P, sm.vec, w);
+        store_words<L::kWords>(out.codes + (size_t)t * L::kBytes, w);
     }
-    uint32_t w[L::kWords];
-    pack_row<D, BITS>(e, w);
-    store_words<L::kWords>(out.codes + (size_t)t * L::kBytes, w);
 }
 
 }  // namespace kvq

@@ -20,17 +20,18 @@ struct QuantArgs {
     float rsqd, sqd; // (float)(1/sqrt(d)), (float)sqrt(d)
 };
 
-// The fp16 input tile and (NSN only) the fp32 transpose buffer share the
-// first region.
+// Shared memory of a quantizer CTA: the fp16 input tile, then (per-channel
+// modes) the fp32 transpose buffer for the per-channel maxima, then the
+// small vectors.
 template <int D, int MODE>
-__host__ __device__ constexpr int quant_region_bytes() {
-    return MODE == kNsn ? kT * D * 4 : kT * D * 2;
+__host__ __device__ constexpr int quant_red_bytes() {
+    return MODE == kNaive ? 0 : kT * D * 4;
 }
 
 template <int D, int MODE>
 __host__ __device__ constexpr int quant_smem_bytes() {
-    // 1024 B alignment slack + region + vec + wmax + sgn + mbarrier
-    return 1024 + quant_region_bytes<D, MODE>() + D * 4 + 4 * D * 4 + D * 4 + 64;
+    // 1024 B alignment slack + tile + red + vec + group partials + token vector + sign masks + mbarrier
+    return 1024 + kT * D * 2 + quant_red_bytes<D, MODE>() + D * 4 + 4096 + kT * 4 + D * 4 + 64;
 }
 
 template <int D, int MODE>
@@ -38,13 +39,17 @@ __device__ __forceinline__ QuantSmem<D> carve_quant_smem(uint8_t* base, uint64_t
     uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023));
     QuantSmem<D> sm;
     tile = p;
+    sm.tile = p;
+    p += kT * D * 2;
     sm.red = reinterpret_cast<float*>(p);
-    p += quant_region_bytes<D, MODE>();
+    p += quant_red_bytes<D, MODE>();
     sm.vec = reinterpret_cast<float*>(p);
     p += D * 4;
-    sm.wmax = reinterpret_cast<uint32_t*>(p);
-    p += 4 * D * 4;
-    sm.sgn = reinterpret_cast<uint32_t*>(p);
+    sm.gpart = reinterpret_cast<float*>(p);
+    p += 4096;
+    sm.tokv = reinterpret_cast<float*>(p);
+    p += kT * 4;
+    sm.sgn2 = reinterpret_cast<uint32_t*>(p);
     p += D * 4;
     bar = reinterpret_cast<uint64_t*>(p);
     return sm;
@@ -69,7 +74,31 @@ __device__ __forceinline__ QuantOut quant_out(const QuantArgs& a, int tensor, in
 template <int D, bool HAD>
 __device__ __forceinline__ void load_signs(const QuantArgs& a, const QuantSmem<D>& sm, int t) {
     if constexpr (HAD) {
-        if (t < D) sm.sgn[t] = (a.signs != nullptr && a.signs[t] < 0) ? 0x80000000u : 0u;
+        if (t < D / 2) {
+            const bool n0 = a.signs != nullptr && a.signs[2 * t] < 0;
+            const bool n1 = a.signs != nullptr && a.signs[2 * t + 1] < 0;
+            sm.sgn2[t] = (n0 ? 0x8000u : 0u) | (n1 ? 0x80000000u : 0u);
+        }
+    }
+}
+
+// Widen 8 fp16 channels of the low half (lo) and the matching 8 of the high
+// half (hi) into pairs P[8q .. 8q+8), after the rotation's sign flips.
+template <int D, bool HAD>
+__device__ __forceinline__ void widen_chunk(uint4 lo, uint4 hi, int q, const QuantSmem<D>& sm, f2_t (&P)[D / 2]) {
+    if constexpr (HAD) {
+        const uint4 ml = reinterpret_cast<const uint4*>(sm.sgn2)[q];
+        const uint4 mh = reinterpret_cast<const uint4*>(sm.sgn2)[D / 16 + q];
+        lo.x ^= ml.x; lo.y ^= ml.y; lo.z ^= ml.z; lo.w ^= ml.w;
+        hi.x ^= mh.x; hi.y ^= mh.y; hi.z ^= mh.z; hi.w ^= mh.w;
+    }
+    const __half2* hl = reinterpret_cast<const __half2*>(&lo);
+    const __half2* hh = reinterpret_cast<const __half2*>(&hi);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 a = __half22float2(hl[i]), b = __half22float2(hh[i]);
+        P[8 * q + 2 * i] = f2_pack(a.x, b.x);
+        P[8 * q + 2 * i + 1] = f2_pack(a.y, b.y);
     }
 }
 
@@ -93,6 +122,7 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ C
         mbar_init(bar, 1);
         fence_mbar_init();
     }
+    load_signs<D, HAD>(a, sm, t);
     __syncthreads();
     if (t == 0) {
         mbar_expect_tx(bar, kTileBytes);
@@ -103,7 +133,6 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ C
             else tma_load_2d(tile + h * (kT * 128), &map_v, h * 64, row0, bar);
         }
     }
-    load_signs<D, HAD>(a, sm, t);
     if (!mbar_wait(bar, 0, 1u << 24)) {
         if (t == 0) report_error(kErrTmaTimeout);
         // wait (bounded) for the copy in flight before the CTA's smem is released
@@ -111,26 +140,21 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ C
         return;
     }
 
-    float v[D];
+    // row t as pairs (channel j, channel j + D/2); the tile holds 64-channel
+    // boxes of 128-byte rows, chunk c of row t at chunk c ^ (t & 7)
+    f2_t P[D / 2];
 #pragma unroll
-    for (int h = 0; h < D / 64; ++h) {
-        const uint8_t* rowp = tile + h * (kT * 128) + t * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(rowp + ((c ^ (t & 7)) << 4));
-            const __half2* hp = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = __half22float2(hp[i]);
-                v[h * 64 + c * 8 + 2 * i] = f.x;
-                v[h * 64 + c * 8 + 2 * i + 1] = f.y;
-            }
-        }
+    for (int q = 0; q < D / 16; ++q) {
+        const int cl = 8 * q, ch = D / 2 + 8 * q;
+        const uint8_t* rl = tile + (cl / 64) * (kT * 128) + t * 128;
+        const uint8_t* rh = tile + (ch / 64) * (kT * 128) + t * 128;
+        const uint4 lo = *reinterpret_cast<const uint4*>(rl + ((((cl % 64) / 8) ^ (t & 7)) << 4));
+        const uint4 hi = *reinterpret_cast<const uint4*>(rh + ((((ch % 64) / 8) ^ (t & 7)) << 4));
+        widen_chunk<D, HAD>(lo, hi, q, sm, P);
     }
-    __syncthreads();  // the tile buffer is reused as the transpose buffer
 
     const QuantOut out = quant_out<D, BITS, MODE, HAD>(a, tensor, bh, a.blk0 + blk);
-    quantize_rows<D, BITS, MODE, HAD>(v, t, sm, out, a.rsqd, a.sqd);
+    quantize_rows<D, BITS, MODE, HAD>(P, t, sm, out, a.rsqd, a.sqd);
 }
 
 struct AppendArgs {
@@ -161,22 +185,23 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
     uint8_t* tile;
     QuantSmem<D> sm = carve_quant_smem<D, MODE>(smem_raw, bar, tile);
     load_signs<D, HAD>(a.q, sm, t);
-    const __half* src = (t == kT - 1) ? xn : res + (size_t)t * D;
-    float v[D];
-#pragma unroll
-    for (int k = 0; k < D / 8; ++k) {
-        const uint4 raw = reinterpret_cast<const uint4*>(src)[k];
-        const __half2* hp = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 f = __half22float2(hp[i]);
-            v[8 * k + 2 * i] = f.x;
-            v[8 * k + 2 * i + 1] = f.y;
-        }
-    }
     __syncthreads();
+    const __half* src = (t == kT - 1) ? xn : res + (size_t)t * D;
+    f2_t P[D / 2];
+#pragma unroll
+    for (int q = 0; q < D / 16; ++q) {
+        const uint4 lo = reinterpret_cast<const uint4*>(src)[q];
+        const uint4 hi = reinterpret_cast<const uint4*>(src)[D / 16 + q];
+        if constexpr (MODE == kNsn) {
+            // the fp16 tile in the quantize kernel's layout, for the block means
+            const int cl = 8 * q, ch = D / 2 + 8 * q;
+            *reinterpret_cast<uint4*>(tile + (cl / 64) * (kT * 128) + t * 128 + ((((cl % 64) / 8) ^ (t & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4*>(tile + (ch / 64) * (kT * 128) + t * 128 + ((((ch % 64) / 8) ^ (t & 7)) << 4)) = hi;
+        }
+        widen_chunk<D, HAD>(lo, hi, q, sm, P);
+    }
     const QuantOut out = quant_out<D, BITS, MODE, HAD>(a.q, tensor, bh, a.blk);
-    quantize_rows<D, BITS, MODE, HAD>(v, t, sm, out, a.q.rsqd, a.q.sqd);
+    quantize_rows<D, BITS, MODE, HAD>(P, t, sm, out, a.q.rsqd, a.q.sqd);
 }
 
 struct DequantArgs {
