@@ -78,7 +78,7 @@ def compare_cache(gcache, ck, cv, d, bits, nq, bh_slice=slice(None)):
     res = {"code_mismatch": 0, "tok_ulp": 0, "chan_ulp": 0, "off_ulp": 0, "codes": 0}
     nb = nq // T
     for i, oc in enumerate((ck, cv)):
-        g_codes = gcache.codes[i].cpu().numpy()[bh_slice][:, :, :nq]
+        g_codes = gcache.codes[i][bh_slice][:, :, :nq].cpu().numpy()
         o_codes = oc["codes"][:, :, :nq]
         if not np.array_equal(g_codes, o_codes):
             gq, _ = oracle.unpack_rows(g_codes.reshape(-1, rb), d, bits)
@@ -87,13 +87,13 @@ def compare_cache(gcache, ck, cv, d, bits, nq, bh_slice=slice(None)):
             assert np.abs(diff).max() <= 1, "codes differ by more than one step"
             res["code_mismatch"] += int(np.count_nonzero(diff))
         res["codes"] += o_codes.size * 8 // bits
-        res["tok_ulp"] = max(res["tok_ulp"], fp16_ulp_diff(host16(gcache.tok[i])[bh_slice][:, :, :nq],
+        res["tok_ulp"] = max(res["tok_ulp"], fp16_ulp_diff(host16(gcache.tok[i][bh_slice][:, :, :nq]),
                                                            oc["tok"][:, :, :nq]))
         if oc["chan"] is not None:
-            res["chan_ulp"] = max(res["chan_ulp"], fp16_ulp_diff(host16(gcache.chan[i])[bh_slice][:, :, :nb],
+            res["chan_ulp"] = max(res["chan_ulp"], fp16_ulp_diff(host16(gcache.chan[i][bh_slice][:, :, :nb]),
                                                                  oc["chan"][:, :, :nb]))
         if oc["off"] is not None:
-            res["off_ulp"] = max(res["off_ulp"], fp16_ulp_diff(host16(gcache.off[i])[bh_slice][:, :, :nb],
+            res["off_ulp"] = max(res["off_ulp"], fp16_ulp_diff(host16(gcache.off[i][bh_slice][:, :, :nb]),
                                                                oc["off"][:, :, :nb]))
     return res
 
