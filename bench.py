@@ -166,6 +166,27 @@ def oracle_sample_text(w, pairs, n, secs):
             f"(dequantize + fp64 attention), {secs:.1f} s")
 
 
+def rank_workload(rank: int, batch=None, stream=None):
+    """The benchmark workload of one rank: every rank runs its own batch of
+    the same shape (weak scaling), drawn from a seed of its own."""
+    w = synth.WORKLOADS[WORKLOAD].scaled(seed=rank)
+    if batch:
+        w = w.scaled(B=batch)
+    if stream is not None:
+        w = w.scaled(stream=stream)
+    return w
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: the job's step time under weak scaling."""
+    if world == 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def bench_config(w, bits, world):
     return {"workload": WORKLOAD, "mode": MODE, "bits": bits, "batch": w.B, "q_heads": w.Hq,
             "kv_heads": w.Hkv, "head_dim": w.d, "seq_len": w.S, "streamed": w.stream,
@@ -217,11 +238,7 @@ def run_ours(args, rank: int, world: int):
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    w = synth.WORKLOADS[WORKLOAD].scaled(seed=rank)
-    if args.batch:
-        w = w.scaled(B=args.batch)
-    if args.stream is not None:
-        w = w.scaled(stream=args.stream)
+    w = rank_workload(rank, args.batch, args.stream)
     BITS = args.bits
     flags = flags_of(MODE)
     G = w.Hq // w.Hkv
@@ -296,11 +313,7 @@ def run_ours(args, rank: int, world: int):
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
-    ms = t_start.elapsed_time(t_end) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, dev)
 
     q_ms = [a.elapsed_time(b) for k, a, b in ev if k == "quantize"]
     d_ms = [a.elapsed_time(b) for k, a, b in ev if k == "decode"]
@@ -385,11 +398,7 @@ def run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, de
         step()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
     h2d = (Kh.numel() + Vh.numel()) * 2 + w.stream * (ksh[0].numel() + vsh[0].numel() + qsh[0].numel()) * 2
     d2h = w.stream * out.numel() * 4
     return {"value": world * step_bytes / (ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
