@@ -167,11 +167,22 @@ struct QuantLaunch {
         CUtensorMap mk, mv;
         const uint64_t rows = (uint64_t)bh * (uint64_t)a.ntok;
         if (!make_row_map(&mk, k, rows, D) || !make_row_map(&mv, v, rows, D)) return KVQ_ERR_CUDA;
-        constexpr int smem = quant_smem_bytes<D, MODE>();
+        constexpr int smem = quant_smem_bytes<D>();
+        auto kern = quantize_kernel<D, BITS, MODE, HAD>;
         static bool attr = false;
-        if (!attr) attr = set_smem(quantize_kernel<D, BITS, MODE, HAD>, smem);
+        if (!attr) attr = set_smem(kern, smem);
         if (!attr) return KVQ_ERR_CUDA;
-        quantize_kernel<D, BITS, MODE, HAD><<<dim3(nblk, bh, 2), kT, smem, st>>>(mk, mv, a);
+        int dev = 0, sms = 0, occ = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kT, smem) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        const long long items = (long long)nblk * bh * 2;
+        if (items >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
+        long long grid = (long long)sms * (occ > 0 ? occ : 1);
+        if (grid > items) grid = items;
+        a.bh = bh;
+        kern<<<(unsigned)grid, kT, smem, st>>>(mk, mv, a);
         return launch_status();
     }
 };
@@ -182,7 +193,7 @@ struct AppendLaunch {
     cudaStream_t st;
     template <int D, int BITS, int MODE, bool HAD>
     kvq_status run() {
-        constexpr int smem = quant_smem_bytes<D, MODE>();
+        constexpr int smem = quant_smem_bytes<D>();
         static bool attr = false;
         if (!attr) attr = set_smem(append_kernel<D, BITS, MODE, HAD>, smem);
         if (!attr) return KVQ_ERR_CUDA;

@@ -351,15 +351,21 @@ __device__ __forceinline__ void pack_codes(const uint32_t (&cw)[D], uint32_t (&w
 
 // ---------------------------------------------------------------- the quantizer
 
+// Bytes of the per-token-group partials: the NSN column sums are
+// (128 / (D / 8)) groups x D floats, the per-channel maxima half of that.
+constexpr int kGpartBytes = 4096;
+
 // Shared-memory scratch of one quantizer CTA.
 template <int D>
 struct QuantSmem {
     // fp16 input tile: 64-channel boxes of 128 rows x 128 bytes, 16-byte
     // chunk c of row t stored at chunk c ^ (t & 7) (the TMA 128-byte swizzle)
     const uint8_t* tile;
-    // fp32 [128][D] transpose buffer in pair order (row t holds P[0..D/2)),
-    // 16-byte chunk k of row t stored at chunk k ^ (t & (D/4 - 1))
-    float* red;
+    // fp32 [128][D] transpose buffer in pair order, in two halves: pairs
+    // [0, D/4) of every row in red_lo, pairs [D/4, D/2) in red_hi; 16-byte
+    // chunk k of a half row t stored at chunk k ^ (t & (D/8 - 1))
+    float* red_lo;
+    float* red_hi;
     float* vec;      // [D] a per-channel vector in pair order (means, reciprocal scales)
     float* gpart;    // [4 KB] per-token-group partial sums / maxima
     float* tokv;     // [128] a per-token scalar (NSN 1/||x|| * sqrt(d))
@@ -475,19 +481,16 @@ __device__ __forceinline__ void codes_from_regs(const f2_t (&P)[D / 2], const fl
 // rne(u * (1/sigma)) clamped.  Sign flips commute exactly with every step
 // up to the rotation (means, norms, fp16 rounding are all sign-symmetric),
 // which is why they can be applied when the row is loaded; the stored
-// offsets are flipped back.
-template <int D, int BITS, int MODE, bool HAD>
+// offsets are flipped back.  done() is called by every thread right after
+// the barrier that follows the last read of the fp16 tile and of the
+// transpose buffer.
+template <int D, int BITS, int MODE, bool HAD, typename Done>
 __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, const QuantSmem<D>& sm,
-                                              const QuantOut& out, const float rsqd, const float sqd) {
+                                              const QuantOut& out, const float rsqd, const float sqd, Done done) {
     using L = RowLayout<D, BITS>;
     constexpr int H2 = D / 2;
-    constexpr int NCH = D / 4;    // 16-byte chunks (two pairs) per row
-    constexpr int TG = NCH;       // tokens per column group
-    constexpr int NG = kT / TG;   // column groups: thread t -> chunk column t % NCH, group t / NCH
-    static_assert(NG * H2 * 8 == 2048, "group partials fill 2 KB");
     const float c0 = HAD ? rsqd : 1.0f;
     float kscale = 1.0f;
-    const int kc = t % NCH, g = t / NCH;
 
     if constexpr (MODE == kNsn) {
         const float n1 = __fsqrt_rn(row_sumsq<H2>(P));
@@ -504,6 +507,7 @@ __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, con
             // sums the 8 channels of chunk column kc8 over the TGc tokens of
             // group gc in the pairwise (binary-counter) order
             constexpr int NKC = D / 8, NGC = kT / NKC, TGC = kT / NGC;
+            static_assert(NGC * D * 4 <= kGpartBytes, "group sums fit the partials buffer");
             const int kc8 = t % NKC, gc = t / NKC;
             const uint8_t* colp = sm.tile + (kc8 / 8) * (kT * 128);
             const int ck = kc8 % 8;
@@ -584,6 +588,8 @@ __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, con
     constexpr float kQ = (float)L::kQmax;
     constexpr float kC = 12582912.0f + (float)L::kOff;  // 1.5 * 2^23 + offset
     if constexpr (MODE == kNaive) {
+        __syncthreads();
+        done();
         uint32_t cw[D];
         float m = 0.0f;
 #pragma unroll
@@ -610,20 +616,37 @@ __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, con
         pack_codes<D, BITS>(cw, w);
         store_words<L::kWords>(out.codes + (size_t)t * L::kBytes, w);
     } else {
-        // per-channel absmax over the block through the transpose buffer
-        store_pair_row<D>(sm.red, P, t);
+        // per-channel absmax over the block through the transpose buffer:
+        // thread t takes chunk column kc (two pairs) of the TG tokens of group g
+        constexpr int NCH = D / 4, NCH2 = D / 8, TG = NCH, NG = kT / TG;
+        static_assert(NG * D * 4 <= kGpartBytes, "group maxima fit the partials buffer");
+        const int kc = t % NCH, g = t / NCH;
+        {
+            char* lo = reinterpret_cast<char*>(sm.red_lo) + (size_t)t * (D / 2) * 4;
+            char* hi = reinterpret_cast<char*>(sm.red_hi) + (size_t)t * (D / 2) * 4;
+#pragma unroll
+            for (int k = 0; k < NCH; ++k) {
+                const int pk = (k % NCH2) ^ (t & (NCH2 - 1));
+                *reinterpret_cast<ulonglong2*>((k < NCH2 ? lo : hi) + pk * 16) = make_ulonglong2(P[2 * k], P[2 * k + 1]);
+            }
+        }
         __syncthreads();
         {
-            const char* base = reinterpret_cast<const char*>(sm.red) + (size_t)g * TG * D * 4;
+            const char* base = reinterpret_cast<const char*>(kc < NCH2 ? sm.red_lo : sm.red_hi) +
+                               (size_t)g * TG * (D / 2) * 4;
+            const int kh = kc % NCH2;
             float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
 #pragma unroll 4
             for (int i = 0; i < TG; ++i) {
-                const float4 x = *reinterpret_cast<const float4*>(base + (size_t)i * D * 4 + ((kc ^ i) << 4));
+                const int tt = g * TG + i;
+                const float4 x =
+                    *reinterpret_cast<const float4*>(base + (size_t)i * (D / 2) * 4 + ((kh ^ (tt & (NCH2 - 1))) << 4));
                 m0 = fmaxf(m0, fabsf(x.x));
                 m1 = fmaxf(m1, fabsf(x.y));
                 m2 = fmaxf(m2, fabsf(x.z));
                 m3 = fmaxf(m3, fabsf(x.w));
             }
+            // group maxima in pair order: [group][pair-order index of the row]
             reinterpret_cast<float4*>(sm.gpart)[g * NCH + kc] = make_float4(m0, m1, m2, m3);
         }
         __syncthreads();
@@ -644,6 +667,7 @@ __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, con
             clamp = __fmaf_rn(m, inv, -(kQ + 0.5f)) >= 0.0f;
         }
         const int any_clamp = __syncthreads_or(clamp);
+        done();
         uint32_t w[L::kWords];
         if (!any_clamp) codes_from_regs<D, BITS, false>(P, sm.vec, w);
         else codes_from_regs<D, BITS, true>(P, sm.vec, w);

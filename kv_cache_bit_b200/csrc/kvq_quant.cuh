@@ -14,39 +14,40 @@ struct QuantArgs {
     __half* off[2];
     const int8_t* signs;
     int H;           // kv heads
+    int bh;          // batch * kv heads
     int cap;         // cache capacity (tokens)
     int ntok;        // tokens in this call (multiple of 128)
     int blk0;        // first destination block
     float rsqd, sqd; // (float)(1/sqrt(d)), (float)sqrt(d)
 };
 
-// Shared memory of a quantizer CTA: the fp16 input tile, then (per-channel
-// modes) the fp32 transpose buffer for the per-channel maxima, then the
-// small vectors.
-template <int D, int MODE>
-__host__ __device__ constexpr int quant_red_bytes() {
-    return MODE == kNaive ? 0 : kT * D * 4;
+// Shared memory of a quantizer CTA: three regions of one fp16 tile each
+// (128 x D x 2 bytes, which is also half of the fp32 transpose buffer), the
+// small vectors and three mbarriers.
+template <int D>
+__host__ __device__ constexpr int quant_region_bytes() {
+    return kT * D * 2;
 }
 
-template <int D, int MODE>
+template <int D>
 __host__ __device__ constexpr int quant_smem_bytes() {
-    // 1024 B alignment slack + tile + red + vec + group partials + token vector + sign masks + mbarrier
-    return 1024 + kT * D * 2 + quant_red_bytes<D, MODE>() + D * 4 + 4096 + kT * 4 + D * 4 + 64;
+    // 1024 B alignment slack + 3 regions + vec + group partials + token vector + sign masks + mbarriers
+    return 1024 + 3 * quant_region_bytes<D>() + D * 4 + kGpartBytes + kT * 4 + D * 4 + 3 * 8;
 }
 
-template <int D, int MODE>
-__device__ __forceinline__ QuantSmem<D> carve_quant_smem(uint8_t* base, uint64_t*& bar, uint8_t*& tile) {
+template <int D>
+__device__ __forceinline__ QuantSmem<D> carve_quant_smem(uint8_t* base, uint64_t*& bar, uint8_t*& regions) {
     uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023));
     QuantSmem<D> sm;
-    tile = p;
+    regions = p;
     sm.tile = p;
-    p += kT * D * 2;
-    sm.red = reinterpret_cast<float*>(p);
-    p += quant_red_bytes<D, MODE>();
+    sm.red_lo = reinterpret_cast<float*>(p + quant_region_bytes<D>());
+    sm.red_hi = reinterpret_cast<float*>(p + 2 * quant_region_bytes<D>());
+    p += 3 * quant_region_bytes<D>();
     sm.vec = reinterpret_cast<float*>(p);
     p += D * 4;
     sm.gpart = reinterpret_cast<float*>(p);
-    p += 4096;
+    p += kGpartBytes;
     sm.tokv = reinterpret_cast<float*>(p);
     p += kT * 4;
     sm.sgn2 = reinterpret_cast<uint32_t*>(p);
@@ -102,59 +103,99 @@ __device__ __forceinline__ void widen_chunk(uint4 lo, uint4 hi, int q, const Qua
     }
 }
 
-// One CTA = one 128-token block of one (tensor, batch, head).  grid:
-// x = block within the call, y = batch * H + head, z = tensor.  The tile is
-// brought in by TMA as 64-channel boxes with 128-byte swizzle, so that each
-// thread can then read its own token row from shared memory without bank
-// conflicts (chunk c of row t sits at chunk c ^ (t & 7)).
+// Persistent quantizer: CTA c takes the work items c, c + gridDim.x, ... of
+// the list (batch * head, block, tensor).  Three tile-sized regions rotate:
+// item i's fp16 tile arrives by TMA in region i % 3 (64-channel boxes with
+// 128-byte swizzle, chunk c of row t at chunk c ^ (t & 7)) while item i - 1
+// is quantized; once item i has read its tile, that region and the free one
+// form its fp32 transpose buffer, and when the transpose buffer has been read
+// the free region takes item i + 2.
 template <int D, int BITS, int MODE, bool HAD>
 __global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ CUtensorMap map_k,
                                                        const __grid_constant__ CUtensorMap map_v, QuantArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const int t = threadIdx.x;
-    const int blk = blockIdx.x, bh = blockIdx.y, tensor = blockIdx.z;
-    uint64_t* bar;
-    uint8_t* tile;
-    QuantSmem<D> sm = carve_quant_smem<D, MODE>(smem_raw, bar, tile);
-    constexpr uint32_t kTileBytes = kT * D * 2;
+    uint64_t* bar;  // [3]
+    uint8_t* regions;
+    QuantSmem<D> sm = carve_quant_smem<D>(smem_raw, bar, regions);
+    constexpr uint32_t kTileBytes = quant_region_bytes<D>();
+    const int nblk = a.ntok / kT;
+    const int nitems = nblk * a.bh * 2;  // < 2^31, checked on the host
 
     if (t == 0) {
-        mbar_init(bar, 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
         fence_mbar_init();
     }
     load_signs<D, HAD>(a, sm, t);
     __syncthreads();
-    if (t == 0) {
-        mbar_expect_tx(bar, kTileBytes);
+    // item w: tensor w & 1, block (w >> 1) % nblk, batch * head (w >> 1) / nblk
+    auto issue = [&](int w, int reg) {
+        const int tensor = w & 1;
+        const int r = w >> 1;
+        const int bh = r / nblk, blk = r - bh * nblk;
+        uint8_t* tile = regions + reg * kTileBytes;
+        mbar_expect_tx(&bar[reg], kTileBytes);
         const int row0 = bh * a.ntok + blk * kT;
 #pragma unroll
         for (int h = 0; h < D / 64; ++h) {
-            if (tensor == 0) tma_load_2d(tile + h * (kT * 128), &map_k, h * 64, row0, bar);
-            else tma_load_2d(tile + h * (kT * 128), &map_v, h * 64, row0, bar);
+            if (tensor == 0) tma_load_2d(tile + h * (kT * 128), &map_k, h * 64, row0, &bar[reg]);
+            else tma_load_2d(tile + h * (kT * 128), &map_v, h * 64, row0, &bar[reg]);
+        }
+    };
+    const int stride = gridDim.x;
+    int w = blockIdx.x;
+    if (t == 0) {
+        if (w < nitems) issue(w, 0);
+        if (w + stride < nitems) issue(w + stride, 1);
+    }
+    int it = 0;
+    uint32_t phases = 0;  // bit k: parity of the next completion of region k
+    for (; w < nitems; w += stride, ++it) {
+        const int reg = it % 3;
+        const bool landed = mbar_wait(&bar[reg], (phases >> reg) & 1, 1u << 24);
+        if (__syncthreads_or(!landed)) {
+            if (t == 0) report_error(kErrTmaTimeout);
+            break;
+        }
+        phases ^= 1u << reg;
+        const uint8_t* tile = regions + reg * kTileBytes;
+        const int spare = (it + 2) % 3;
+        sm.tile = tile;
+        sm.red_lo = reinterpret_cast<float*>(regions + reg * kTileBytes);
+        sm.red_hi = reinterpret_cast<float*>(regions + spare * kTileBytes);
+        const int tensor = w & 1;
+        const int r = w >> 1;
+        const int bh = r / nblk, blk = r - bh * nblk;
+        // row t as pairs (channel j, channel j + D/2)
+        f2_t P[D / 2];
+#pragma unroll
+        for (int q = 0; q < D / 16; ++q) {
+            const int cl = 8 * q, ch = D / 2 + 8 * q;
+            const uint8_t* rl = tile + (cl / 64) * (kT * 128) + t * 128;
+            const uint8_t* rh = tile + (ch / 64) * (kT * 128) + t * 128;
+            const uint4 lo = *reinterpret_cast<const uint4*>(rl + ((((cl % 64) / 8) ^ (t & 7)) << 4));
+            const uint4 hi = *reinterpret_cast<const uint4*>(rh + ((((ch % 64) / 8) ^ (t & 7)) << 4));
+            widen_chunk<D, HAD>(lo, hi, q, sm, P);
+        }
+        if constexpr (MODE != kNsn) __syncthreads();  // the tile region becomes transpose buffer
+        const int wn = w + 2 * stride;
+        const QuantOut out = quant_out<D, BITS, MODE, HAD>(a, tensor, bh, a.blk0 + blk);
+        quantize_rows<D, BITS, MODE, HAD>(P, t, sm, out, a.rsqd, a.sqd, [&] {
+            if (t == 0 && wn < nitems) {
+                fence_proxy_async_smem();
+                issue(wn, spare);
+            }
+        });
+        __syncthreads();  // the next item's row loads reuse the shared vectors
+    }
+    // after an early exit, the copies still in flight (items w and w + stride)
+    // land before the CTA ends
+    if (t == 0 && w < nitems) {
+        for (int k = 0; k < 2; ++k) {
+            const int reg = (it + k) % 3;
+            if (w + k * stride < nitems) mbar_wait(&bar[reg], (phases >> reg) & 1, 1u << 24);
         }
     }
-    if (!mbar_wait(bar, 0, 1u << 24)) {
-        if (t == 0) report_error(kErrTmaTimeout);
-        // wait (bounded) for the copy in flight before the CTA's smem is released
-        mbar_wait(bar, 0, 1u << 24);
-        return;
-    }
-
-    // row t as pairs (channel j, channel j + D/2); the tile holds 64-channel
-    // boxes of 128-byte rows, chunk c of row t at chunk c ^ (t & 7)
-    f2_t P[D / 2];
-#pragma unroll
-    for (int q = 0; q < D / 16; ++q) {
-        const int cl = 8 * q, ch = D / 2 + 8 * q;
-        const uint8_t* rl = tile + (cl / 64) * (kT * 128) + t * 128;
-        const uint8_t* rh = tile + (ch / 64) * (kT * 128) + t * 128;
-        const uint4 lo = *reinterpret_cast<const uint4*>(rl + ((((cl % 64) / 8) ^ (t & 7)) << 4));
-        const uint4 hi = *reinterpret_cast<const uint4*>(rh + ((((ch % 64) / 8) ^ (t & 7)) << 4));
-        widen_chunk<D, HAD>(lo, hi, q, sm, P);
-    }
-
-    const QuantOut out = quant_out<D, BITS, MODE, HAD>(a, tensor, bh, a.blk0 + blk);
-    quantize_rows<D, BITS, MODE, HAD>(P, t, sm, out, a.rsqd, a.sqd);
 }
 
 struct AppendArgs {
@@ -183,7 +224,7 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint64_t* bar;
     uint8_t* tile;
-    QuantSmem<D> sm = carve_quant_smem<D, MODE>(smem_raw, bar, tile);
+    QuantSmem<D> sm = carve_quant_smem<D>(smem_raw, bar, tile);
     load_signs<D, HAD>(a.q, sm, t);
     __syncthreads();
     const __half* src = (t == kT - 1) ? xn : res + (size_t)t * D;
@@ -201,7 +242,7 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
         widen_chunk<D, HAD>(lo, hi, q, sm, P);
     }
     const QuantOut out = quant_out<D, BITS, MODE, HAD>(a.q, tensor, bh, a.blk);
-    quantize_rows<D, BITS, MODE, HAD>(P, t, sm, out, a.q.rsqd, a.q.sqd);
+    quantize_rows<D, BITS, MODE, HAD>(P, t, sm, out, a.q.rsqd, a.q.sqd, [] {});
 }
 
 struct DequantArgs {
