@@ -126,6 +126,21 @@ bool make_row_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D view [rows][row_bytes] of packed code rows (row_bytes 64 or 32), as
+// the destination of TMA stores of 128-row tiles with the matching swizzle
+// (64-byte rows: 64-byte swizzle; 32-byte rows: 32-byte swizzle).
+bool make_code_map(CUtensorMap* m, void* base, uint64_t rows, int row_bytes) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)kT};
+    cuuint32_t es[2] = {1, 1};
+    const CUtensorMapSwizzle sw = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Dynamic shared memory size, and the largest shared-memory carveout so that
 // the residency the occupancy calculator reports is the one the launch gets.
 template <typename K>
@@ -164,9 +179,18 @@ struct QuantLaunch {
     cudaStream_t st;
     template <int D, int BITS, int MODE, bool HAD>
     kvq_status run() {
-        CUtensorMap mk, mv;
+        CUtensorMap mk, mv, mck, mcv;
         const uint64_t rows = (uint64_t)bh * (uint64_t)a.ntok;
         if (!make_row_map(&mk, k, rows, D) || !make_row_map(&mv, v, rows, D)) return KVQ_ERR_CUDA;
+        memset(&mck, 0, sizeof(mck));
+        memset(&mcv, 0, sizeof(mcv));
+        constexpr int rb = D * BITS / 8;
+        if constexpr ((BITS == 4 && rb == 64) || (BITS == 2 && rb == 32)) {
+            const uint64_t crow = (uint64_t)bh * (uint64_t)a.cap;
+            if (crow >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+            if (!make_code_map(&mck, a.codes[0], crow, rb) || !make_code_map(&mcv, a.codes[1], crow, rb))
+                return KVQ_ERR_CUDA;
+        }
         constexpr int smem = quant_smem_bytes<D>();
         auto kern = quantize_kernel<D, BITS, MODE, HAD>;
         static bool attr = false;
@@ -182,7 +206,7 @@ struct QuantLaunch {
         long long grid = (long long)sms * (occ > 0 ? occ : 1);
         if (grid > items) grid = items;
         a.bh = bh;
-        kern<<<(unsigned)grid, kT, smem, st>>>(mk, mv, a);
+        kern<<<(unsigned)grid, kT, smem, st>>>(mk, mv, mck, mcv, a);
         return launch_status();
     }
 };

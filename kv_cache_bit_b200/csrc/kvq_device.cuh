@@ -74,6 +74,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// 2-D tiled TMA store shared -> global (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the committed bulk stores have read their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 // 1-D bulk copy global -> shared (no multicast); size and both addresses
 // must be multiples of 16 bytes.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -375,10 +386,35 @@ struct QuantSmem {
 // Output pointers of one (tensor, batch, head, block).
 struct QuantOut {
     uint8_t* codes;  // [128][row_bytes] rows of this block
+    uint8_t* stage;  // if set, codes go here instead, for a TMA store: row t at t * row_bytes,
+                     // 16-byte chunk c at chunk c ^ ((t >> 1) & 3) (INT4, 64-byte swizzle) or
+                     // c ^ ((t >> 2) & 1) (INT2, 32-byte swizzle)
     __half* tok;     // [128][ntok]
     __half* chan;    // [D] (PER_CHANNEL)
     __half* off;     // [D] (NSN)
 };
+
+// Row t of packed codes: straight to global memory, or into the swizzled
+// staging tile of a TMA store (then visible to the async proxy).
+template <int D, int BITS>
+__device__ __forceinline__ void store_codes(const QuantOut& out, int t, const uint32_t (&w)[RowLayout<D, BITS>::kWords]) {
+    using L = RowLayout<D, BITS>;
+    if constexpr (BITS == 4 || BITS == 2) {
+        if (out.stage != nullptr) {
+            constexpr int NC = L::kBytes / 16;  // 16-byte chunks per row
+            const int sw = (L::kBytes == 64) ? ((t >> 1) & 3) : ((t >> 2) & 1);
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                const int pc = (c ^ sw) & (NC - 1);
+                *reinterpret_cast<uint4*>(out.stage + (size_t)t * L::kBytes + pc * 16) =
+                    make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+            }
+            fence_proxy_async_smem();
+            return;
+        }
+    }
+    store_words<L::kWords>(out.codes + (size_t)t * L::kBytes, w);
+}
 
 template <int D>
 __device__ __forceinline__ void store_pair_row(float* red, const f2_t (&P)[D / 2], int t) {
@@ -614,7 +650,7 @@ __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, con
         }
         uint32_t w[L::kWords];
         pack_codes<D, BITS>(cw, w);
-        store_words<L::kWords>(out.codes + (size_t)t * L::kBytes, w);
+        store_codes<D, BITS>(out, t, w);
     } else {
         // per-channel absmax over the block through the transpose buffer:
         // thread t takes chunk column kc (two pairs) of the TG tokens of group g
@@ -671,7 +707,7 @@ __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, con
         uint32_t w[L::kWords];
         if (!any_clamp) codes_from_regs<D, BITS, false>(P, sm.vec, w);
         else codes_from_regs<D, BITS, true>(P, sm.vec, w);
-        store_words<L::kWords>(out.codes + (size_t)t * L::kBytes, w);
+        store_codes<D, BITS>(out, t, w);
     }
 }
 

@@ -69,6 +69,7 @@ __device__ __forceinline__ QuantOut quant_out(const QuantArgs& a, int tensor, in
     o.tok = (v ? a.tok[1] : a.tok[0]) + ((size_t)bh * a.cap + (size_t)blk * kT) * ntk;
     o.chan = (MODE != kNaive) ? (v ? a.chan[1] : a.chan[0]) + ((size_t)bh * nb + blk) * D : nullptr;
     o.off = (MODE == kNsn) ? (v ? a.off[1] : a.off[0]) + ((size_t)bh * nb + blk) * D : nullptr;
+    o.stage = nullptr;
     return o;
 }
 
@@ -112,7 +113,12 @@ __device__ __forceinline__ void widen_chunk(uint4 lo, uint4 hi, int q, const Qua
 // the free region takes item i + 2.
 template <int D, int BITS, int MODE, bool HAD>
 __global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ CUtensorMap map_k,
-                                                       const __grid_constant__ CUtensorMap map_v, QuantArgs a) {
+                                                       const __grid_constant__ CUtensorMap map_v,
+                                                       const __grid_constant__ CUtensorMap map_ck,
+                                                       const __grid_constant__ CUtensorMap map_cv, QuantArgs a) {
+    // INT4 / INT2 code rows leave through a TMA store of a swizzled staging
+    // tile (the region just read), so that each warp writes whole lines
+    constexpr bool kTmaStore = (BITS == 4 && D * BITS / 8 == 64) || (BITS == 2 && D * BITS / 8 == 32);
     extern __shared__ uint8_t smem_raw[];
     const int t = threadIdx.x;
     uint64_t* bar;  // [3]
@@ -153,6 +159,7 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ C
     for (; w < nitems; w += stride, ++it) {
         const int reg = it % 3;
         const bool landed = mbar_wait(&bar[reg], (phases >> reg) & 1, 1u << 24);
+        if (kTmaStore && t == 0) bulk_wait_read();  // the last code store has read its staging tile
         if (__syncthreads_or(!landed)) {
             if (t == 0) report_error(kErrTmaTimeout);
             break;
@@ -179,15 +186,21 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ C
         }
         if constexpr (MODE != kNsn) __syncthreads();  // the tile region becomes transpose buffer
         const int wn = w + 2 * stride;
-        const QuantOut out = quant_out<D, BITS, MODE, HAD>(a, tensor, bh, a.blk0 + blk);
+        QuantOut out = quant_out<D, BITS, MODE, HAD>(a, tensor, bh, a.blk0 + blk);
+        if constexpr (kTmaStore) out.stage = regions + reg * kTileBytes;
         quantize_rows<D, BITS, MODE, HAD>(P, t, sm, out, a.rsqd, a.sqd, [&] {
             if (t == 0 && wn < nitems) {
                 fence_proxy_async_smem();
                 issue(wn, spare);
             }
         });
-        __syncthreads();  // the next item's row loads reuse the shared vectors
+        __syncthreads();  // the next item's row loads reuse the shared vectors; codes staged
+        if (kTmaStore && t == 0) {
+            tma_store_2d(tensor ? &map_cv : &map_ck, 0, bh * a.cap + (a.blk0 + blk) * kT, out.stage);
+            bulk_commit();
+        }
     }
+    if (kTmaStore && t == 0) bulk_wait_read();
     // after an early exit, the copies still in flight (items w and w + stride)
     // land before the CTA ends
     if (t == 0 && w < nitems) {
