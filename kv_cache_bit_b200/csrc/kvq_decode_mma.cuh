@@ -84,6 +84,15 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D = A * B (the accumulation starts from zero), m16n8k16, fp16 inputs.
+__device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
     float r;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
@@ -593,13 +602,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                 for (int o = 16; o; o >>= 1) numax = fmaxf(numax, __shfl_xor_sync(0xffffffffu, numax, o));
                 const int fexp = numax > 0.0f ? 13 - (int)kTau - ceil_log2(numax) : 0;
                 const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
-                float dv[NT][8][4];
-#pragma unroll
-                for (int n = 0; n < NT; ++n)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) dv[n][i][k] = 0.0f;
+                float dv[NT][8][4];  // set by the first tile's MMAs
                 float lsum[NT], bsum[NT];
 #pragma unroll
                 for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
@@ -613,9 +616,11 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                     bool over = false;
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
-                        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+                        float d0[4], d1[4];
+                        mma16816_z(d0, pa[0], pb[0], pa[1], pb[1], bq[n][0], bq[n][1]);
+                        mma16816_z(d1, pa[2], pb[2], pa[3], pb[3], bq[n][2], bq[n][3]);
 #pragma unroll
-                        for (int s = 0; s < 8; s += 2) {
+                        for (int s = 2; s < 8; s += 2) {
                             mma16816(d0, pa[2 * s], pb[2 * s], pa[2 * s + 1], pb[2 * s + 1], bq[n][2 * s],
                                      bq[n][2 * s + 1]);
                             mma16816(d1, pa[2 * s + 2], pb[2 * s + 2], pa[2 * s + 3], pb[2 * s + 3],
@@ -655,10 +660,12 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                                 acc[n][k] *= corr;
                                 if (MODE == kNsn) acco[n][k] *= corr;
                             }
+                            if (m4 > 0) {
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
+                                for (int i = 0; i < 8; ++i)
 #pragma unroll
-                                for (int k = 0; k < 4; ++k) dv[n][i][k] *= corr;
+                                    for (int k = 0; k < 4; ++k) dv[n][i][k] *= corr;
+                            }
                         }
                     }
                     // ---- P' = p * nu (scaled), as (hi, lo) rows, moved into the B layout
@@ -691,9 +698,14 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 #pragma unroll
                     for (int tc = 0; tc < 8; ++tc) {
 #pragma unroll
-                        for (int n = 0; n < NT; ++n)
-                            mma16816(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1], bp[n][0],
-                                     bp[n][1]);
+                        for (int n = 0; n < NT; ++n) {
+                            if (m4 == 0)
+                                mma16816_z(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1],
+                                           bp[n][0], bp[n][1]);
+                            else
+                                mma16816(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1],
+                                         bp[n][0], bp[n][1]);
+                        }
                     }
                 }
                 release(uk);
