@@ -44,6 +44,29 @@ BITS = 4
 METRIC = "INT4-KV decode attention GB/s (% of HBM peak) & tokens/s; quantize GB/s"
 
 
+KERNEL_SOURCES = ["kvq_api.cu", "kvq_decode_mma.cuh", "kvq_decode_simple.cuh", "kvq_device.cuh", "kvq_quant.cuh"]
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "decode_traffic_throughput.md")
+
+
+def decode_traffic():
+    """DRAM bytes of one decode call from the committed ncu summary, or None
+    when the kernels have changed since it was captured."""
+    import hashlib
+    try:
+        text = open(TRAFFIC_PROFILE).read()
+        fields = dict(ln.split(":", 1) for ln in text.splitlines() if ln.startswith(("traffic_bytes_per_call:",
+                                                                                      "source_sha256:")))
+        h = hashlib.sha256()
+        for f in KERNEL_SOURCES:
+            with open(os.path.join(ROOT, "kv_cache_bit_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
+        if h.hexdigest() != fields["source_sha256"].strip():
+            return None
+        return float(fields["traffic_bytes_per_call:".rstrip(":")].strip())
+    except Exception:
+        return None
+
+
 def measured_peak_gbs():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -268,14 +291,18 @@ def run_ours(args, rank: int, world: int):
         if record:
             e1 = torch.cuda.Event(enable_timing=True); e1.record(stream)
             ev.append(("quantize", e0, e1))
+            prev = e1
         for i in range(n_stream):
             kvq.kvq_append_token(cfg, cache, ksd[i], vsd[i], stream)
             if record:
                 d0 = torch.cuda.Event(enable_timing=True); d0.record(stream)
+                flush = (w.S + i + 1) % 128 == 0
+                ev.append(("flush" if flush else "append", prev, d0))
             kvq.kvq_decode_attention(cfg, cache, qsd[i], w.Hq, 0.0, out, ws, ws_bytes, stream)
             if record:
                 d1 = torch.cuda.Event(enable_timing=True); d1.record(stream)
                 ev.append(("decode", d0, d1))
+                prev = d1
 
     # algorithmic bytes of one step
     step_bytes = accounting.quantize_bytes(w.d, BITS, flags, w.B, w.Hkv, w.S)
@@ -317,6 +344,8 @@ def run_ours(args, rank: int, world: int):
 
     q_ms = [a.elapsed_time(b) for k, a, b in ev if k == "quantize"]
     d_ms = [a.elapsed_time(b) for k, a, b in ev if k == "decode"]
+    a_ms = [a.elapsed_time(b) for k, a, b in ev if k == "append"]
+    f_ms = [a.elapsed_time(b) for k, a, b in ev if k == "flush"]
     dec_avg_bytes = sum(dec_bytes) / len(dec_bytes)
     dec_avg_s = (sum(d_ms) / len(d_ms)) / 1e3
     q_avg_s = (sum(q_ms) / len(q_ms)) / 1e3
@@ -325,6 +354,9 @@ def run_ours(args, rank: int, world: int):
     dec_gbs = dec_avg_bytes / dec_avg_s / 1e9
     q_gbs = q_bytes / q_avg_s / 1e9
     value = world * step_bytes / (ms / 1e3) / 1e9
+
+    int2 = None if (args.no_int2 or world > 1 or BITS != 4) else run_int2(w, flags, Kd, Vd, ksd, vsd, qsd, stream,
+                                                                          dev, peak)
 
     # end to end through the public calls, host buffers, copies inside the region
     e2e = None if args.no_e2e else run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, dev,
@@ -338,14 +370,21 @@ def run_ours(args, rank: int, world: int):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": bench_config(w, BITS, world),
         "decode": {"gbs": dec_gbs, "frac_of_hbm": dec_gbs / peak, "us_per_call": dec_avg_s * 1e6,
-                   "tokens_per_s": world * w.B / dec_avg_s, "bytes_per_call": dec_avg_bytes},
+                   "tokens_per_s": world * w.B / dec_avg_s, "bytes_per_call": dec_avg_bytes,
+                   "cache_tokens_per_s": world * w.B * w.Hkv * (w.S + (n_stream + 1) / 2) / dec_avg_s},
+        "append": {"us_per_call": 1e3 * sum(a_ms) / max(1, len(a_ms)),
+                   "flush_us_per_call": 1e3 * sum(f_ms) / max(1, len(f_ms)) if f_ms else None,
+                   "flushes_per_step": len(f_ms) // max(1, args.steps)},
         "quantize": {"gbs": q_gbs, "frac_of_hbm": q_gbs / peak, "us_per_call": q_avg_s * 1e6,
                      "bytes_per_call": q_bytes},
         "tokens_per_s": world * w.B * n_stream / (ms / 1e3),
         "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
-                     "traffic": None, "kernel": "kvq_decode_attention (split + combine launches)",
-                     "peak_kind": f"{peak_kind} copy bandwidth"},
+                     "traffic": decode_traffic(),
+                     "kernel": "kvq_decode_attention (decode + combine launches), per call",
+                     "peak_kind": f"{peak_kind} copy bandwidth (burst)",
+                     "traffic_source": "profiles/decode_traffic_throughput.md (ncu dram bytes, one call)"},
         "e2e": e2e,
+        "int2": int2,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -356,6 +395,52 @@ def run_ours(args, rank: int, world: int):
                                 "sample": oracle_sample_text(w, pairs, n, secs)}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def run_int2(w, flags, Kd, Vd, ksd, vsd, qsd, stream, dev, peak):
+    """The same workload quantized to INT2 codes: quantize of the prefill,
+    the streamed appends, then decode calls at the final length (CUDA events
+    on the launching stream)."""
+    import torch
+    from kv_cache_bit_b200 import kvq
+    bits = 2
+    cap = ((w.S + w.stream + 127) // 128) * 128
+    cfg = kvq.Config(w.d, bits, flags, None, device=dev)
+    cache = kvq.KVCache.allocate(cfg, w.B, w.Hkv, cap, device=dev)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    ws_bytes = kvq.kvq_decode_workspace_bytes(cfg, cache, w.Hq)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        cache.c.len = 0
+        kvq.kvq_quantize_block(cfg, cache, Kd, Vd, 0, w.S, stream)
+    q0, q1 = ev(), ev()
+    reps = 3
+    q0.record(stream)
+    for _ in range(reps):
+        cache.c.len = 0
+        kvq.kvq_quantize_block(cfg, cache, Kd, Vd, 0, w.S, stream)
+    q1.record(stream)
+    for i in range(w.stream):
+        kvq.kvq_append_token(cfg, cache, ksd[i], vsd[i], stream)
+    qlast = qsd[w.stream - 1] if w.stream else qsd[0]
+    for _ in range(3):
+        kvq.kvq_decode_attention(cfg, cache, qlast, w.Hq, 0.0, out, ws, ws_bytes, stream)
+    d0, d1 = ev(), ev()
+    n = 32
+    d0.record(stream)
+    for _ in range(n):
+        kvq.kvq_decode_attention(cfg, cache, qlast, w.Hq, 0.0, out, ws, ws_bytes, stream)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    q_s = q0.elapsed_time(q1) / reps / 1e3
+    d_s = d0.elapsed_time(d1) / n / 1e3
+    qb = accounting.quantize_bytes(w.d, bits, flags, w.B, w.Hkv, w.S)
+    db = accounting.decode_bytes(w.d, bits, flags, w.B, w.Hkv, w.Hq, w.S + w.stream)
+    return {"quantize": {"gbs": qb / q_s / 1e9, "frac_of_hbm": qb / q_s / 1e9 / peak, "us_per_call": q_s * 1e6,
+                         "bytes_per_call": qb},
+            "decode": {"gbs": db / d_s / 1e9, "frac_of_hbm": db / d_s / 1e9 / peak, "us_per_call": d_s * 1e6,
+                       "bytes_per_call": db, "length": w.S + w.stream}}
 
 
 def run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, dev, step_bytes, world):
@@ -413,6 +498,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--no-int2", action="store_true", help="skip the INT2 measurement of the same workload")
     ap.add_argument("--batch", type=int, default=None, help="override the batch size (smaller profiling cases)")
     ap.add_argument("--stream", type=int, default=None, help="override the number of streamed decode steps")
     ap.add_argument("--bits", type=int, default=BITS, choices=[2, 3, 4])
