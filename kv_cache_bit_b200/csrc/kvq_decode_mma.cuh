@@ -806,7 +806,6 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     const int b = pair / a.H, h = pair % a.H;
     extern __shared__ __align__(16) uint8_t comb_raw[];
     __half* s_rv = reinterpret_cast<__half*>(comb_raw);  // [kT][D]
-    __shared__ float s_q[GP][D];
     __shared__ float s_pm[GP][128], s_pl[GP][128];  // candidate m, then weight; l
     __shared__ int s_slot[128];
     __shared__ float s_M[GP], s_L[GP], s_f[GP];
@@ -821,21 +820,19 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
         const int nchunk = rlen * (D * 2 / 16);
         for (int i = tid; i < nchunk; i += 128) cp_async16(reinterpret_cast<uint8_t*>(s_rv) + 16 * i, rv + 16 * i);
     }
-    {
-        const __half* qp = a.q + ((size_t)b * a.H * G + (size_t)h * G) * D;
-        float qv[GP];
-#pragma unroll
-        for (int j = 0; j < GP; ++j) qv[j] = (j < G) ? __half2float(qp[(size_t)j * D + c]) : 0.0f;
-#pragma unroll
-        for (int j = 0; j < GP; ++j) s_q[j][c] = qv[j];
-        if constexpr (HAD) s_sg[c] = (a.signs != nullptr && a.signs[c] < 0) ? -1.0f : 1.0f;
-    }
+    if constexpr (HAD) s_sg[c] = (a.signs != nullptr && a.signs[c] < 0) ? -1.0f : 1.0f;
     if (tid < GP) { s_M[tid] = -INFINITY; s_L[tid] = 0.0f; s_f[tid] = 0.0f; }
-    uint4 krow[D / 8];
-    if (tid < rlen) {
-        const uint4* row = reinterpret_cast<const uint4*>(a.resid[0] + ((size_t)pair * kT + tid) * D);
+    // residual logits on the tensor cores: K rows (fp16) times the queries
+    // (fp16, exact); lane (g, t) loads channels 32t .. 32t + 31 of tokens
+    // g and g + 8 of each 16-token tile and of query head g; k-step s covers
+    // channels 32t + 4s + {0, 1} (k = 2t, 2t + 1) and + {2, 3} (k = 2t + 8, 2t + 9)
+    const int g = lane >> 2, t4 = lane & 3;
+    uint4 qf[4];
+    {
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        const __half* qp = a.q + ((size_t)b * a.H * G + (size_t)h * G + g) * D + 32 * t4;
 #pragma unroll
-        for (int k8 = 0; k8 < D / 8; ++k8) krow[k8] = row[k8];
+        for (int i = 0; i < 4; ++i) qf[i] = (g < G && rlen > 0) ? reinterpret_cast<const uint4*>(qp)[i] : z4;
     }
 
     // merge one chunk of per-head candidate (m, l) published in s_pm / s_pl:
@@ -870,27 +867,33 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     __syncthreads();
 
     if (rlen > 0) {
-        float sdot[GP];
+        static_assert(GP <= 8, "one n-tile of query heads");
+        const __half* rk = a.resid[0] + (size_t)pair * kT * D;
+        const uint32_t* qw = reinterpret_cast<const uint32_t*>(qf);
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        for (int r0 = 16 * warp; r0 < rlen; r0 += 64) {
+            const int ta = r0 + g, tb = r0 + g + 8;
+            uint4 ka[4], kb[4];
 #pragma unroll
-        for (int j = 0; j < GP; ++j) sdot[j] = 0.0f;
-        if (tid < rlen) {
-#pragma unroll
-            for (int k8 = 0; k8 < D / 8; ++k8) {
-                const __half2* hp = reinterpret_cast<const __half2*>(&krow[k8]);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 x = __half22float2(hp[e]);
-#pragma unroll
-                    for (int j = 0; j < GP; ++j)
-                        if (j < G) sdot[j] += s_q[j][8 * k8 + 2 * e] * x.x + s_q[j][8 * k8 + 2 * e + 1] * x.y;
-                }
+            for (int i = 0; i < 4; ++i) {
+                ka[i] = ta < rlen ? reinterpret_cast<const uint4*>(rk + (size_t)ta * D + 32 * t4)[i] : z4;
+                kb[i] = tb < rlen ? reinterpret_cast<const uint4*>(rk + (size_t)tb * D + 32 * t4)[i] : z4;
             }
-        }
+            const uint32_t* wa = reinterpret_cast<const uint32_t*>(ka);
+            const uint32_t* wb = reinterpret_cast<const uint32_t*>(kb);
+            float d[4];
+            mma16816_z(d, wa[0], wb[0], wa[1], wb[1], qw[0], qw[1]);
 #pragma unroll
-        for (int j = 0; j < GP; ++j) {
-            if (j < G) {
-                s_pm[j][tid] = (tid < rlen) ? sdot[j] * alpha2 : -INFINITY;
-                s_pl[j][tid] = 1.0f;
+            for (int s2 = 1; s2 < 8; ++s2)
+                mma16816(d, wa[2 * s2], wb[2 * s2], wa[2 * s2 + 1], wb[2 * s2 + 1], qw[2 * s2], qw[2 * s2 + 1]);
+            // d: (token ta, head 2 t4), (ta, 2 t4 + 1), (tb, 2 t4), (tb, 2 t4 + 1)
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int j = 2 * t4 + cc;
+                if (j < G) {
+                    if (ta < rlen) { s_pm[j][ta] = d[cc] * alpha2; s_pl[j][ta] = 1.0f; }
+                    if (tb < rlen) { s_pm[j][tb] = d[2 + cc] * alpha2; s_pl[j][tb] = 1.0f; }
+                }
             }
         }
         __syncthreads();
