@@ -211,6 +211,19 @@ class KVCache:
                       (ctypes.c_void_p * 2)(*[_ptr(x) for x in resid]))
         return cls(c, codes, tok, chan, off, resid)
 
+    def rows(self, b0: int, b1: int) -> "KVCache":
+        """A view of batch rows [b0, b1) sharing this cache's memory (its own
+        kvq_cache struct, len copied)."""
+        sl = lambda ts: [t[b0:b1] if t is not None else None for t in ts]
+        codes, tok, chan, off, resid = sl(self.codes), sl(self.tok), sl(self.chan), sl(self.off), sl(self.resid)
+        c = kvq_cache(b1 - b0, self.c.kv_heads, self.c.head_dim, self.c.capacity, self.c.len,
+                      (ctypes.c_void_p * 2)(*[_ptr(x) for x in codes]),
+                      (ctypes.c_void_p * 2)(*[_ptr(x) for x in tok]),
+                      (ctypes.c_void_p * 2)(*[_ptr(x) for x in chan]),
+                      (ctypes.c_void_p * 2)(*[_ptr(x) for x in off]),
+                      (ctypes.c_void_p * 2)(*[_ptr(x) for x in resid]))
+        return KVCache(c, codes, tok, chan, off, resid)
+
     @property
     def len(self) -> int:
         return self.c.len
