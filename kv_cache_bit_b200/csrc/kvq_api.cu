@@ -300,14 +300,17 @@ struct DecodeLaunch {
     }
 };
 
-// Splits of the sequence for decode: about six waves of CTAs on 148 SMs
-// (two resident per SM) with at least 8 blocks per split, fixed per cache
-// shape so that the workspace size does not depend on len.
+// Splits of the sequence for the CUDA-core decode (head dim 64): about six
+// waves of CTAs on 148 SMs (two resident per SM), at least 8 blocks per
+// split when the sequence is long enough to fill the waves that way, else
+// as few as one block per split (short caches are latency-bound).  Fixed
+// per cache shape so that the workspace size does not depend on len.
 int decode_splits(const kvq_cache* c) {
     const int bh = c->batch * c->kv_heads;
     const int nb = c->capacity / kT;
     int ns = (6 * 296 + bh - 1) / bh;
-    if (ns > nb / 8) ns = nb / 8;
+    const int cap8 = nb / 8;
+    if (ns > cap8) ns = cap8 >= 2 ? cap8 : nb;
     if (ns < 1) ns = 1;
     return ns;
 }
