@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -150,6 +151,21 @@ bool set_smem(K kernel, int bytes) {
                                 cudaSharedmemCarveoutMaxShared) == cudaSuccess;
 }
 
+// set_smem once per (kernel, device): function attributes belong to a
+// device's context.  One bit per device id; racing callers both set the same
+// attributes, which is harmless.
+template <auto Kernel>
+bool ensure_smem(int bytes) {
+    static std::atomic<uint64_t> done{0};  // one mask per kernel instantiation
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    const uint64_t bit = uint64_t(1) << dev;
+    if (done.load(std::memory_order_acquire) & bit) return true;
+    if (!set_smem(Kernel, bytes)) return false;
+    done.fetch_or(bit, std::memory_order_release);
+    return true;
+}
+
 QuantArgs quant_args(const kvq_config* cfg, const kvq_cache* c) {
     QuantArgs a;
     for (int i = 0; i < 2; ++i) {
@@ -193,9 +209,7 @@ struct QuantLaunch {
         }
         constexpr int smem = quant_smem_bytes<D>();
         auto kern = quantize_kernel<D, BITS, MODE, HAD>;
-        static bool attr = false;
-        if (!attr) attr = set_smem(kern, smem);
-        if (!attr) return KVQ_ERR_CUDA;
+        if (!ensure_smem<quantize_kernel<D, BITS, MODE, HAD>>(smem)) return KVQ_ERR_CUDA;
         int dev = 0, sms = 0, occ = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
@@ -218,9 +232,7 @@ struct AppendLaunch {
     template <int D, int BITS, int MODE, bool HAD>
     kvq_status run() {
         constexpr int smem = quant_smem_bytes<D>();
-        static bool attr = false;
-        if (!attr) attr = set_smem(append_kernel<D, BITS, MODE, HAD>, smem);
-        if (!attr) return KVQ_ERR_CUDA;
+        if (!ensure_smem<append_kernel<D, BITS, MODE, HAD>>(smem)) return KVQ_ERR_CUDA;
         append_kernel<D, BITS, MODE, HAD><<<dim3(bh, 2), kT, a.slot == kT - 1 ? smem : 0, st>>>(a);
         return launch_status();
     }
@@ -241,9 +253,7 @@ template <int D, int BITS, int MODE, bool HAD, int GP>
 kvq_status launch_decode_mma(DecodeArgs a, int bh, cudaStream_t st) {
     constexpr int smem = mma_smem_bytes<D, BITS, MODE, GP>();
     auto kern = decode_mma_kernel<D, BITS, MODE, HAD, GP>;
-    static bool attr = false;
-    if (!attr) attr = set_smem(kern, smem);
-    if (!attr) return KVQ_ERR_CUDA;
+    if (!ensure_smem<decode_mma_kernel<D, BITS, MODE, HAD, GP>>(smem)) return KVQ_ERR_CUDA;
     int dev = 0, sms = 0, occ = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
@@ -263,9 +273,7 @@ kvq_status launch_decode_mma(DecodeArgs a, int bh, cudaStream_t st) {
     // its residual phase overlaps the decode kernel's tail
     auto comb = decode_combine_mma_kernel<D, HAD, GP>;
     constexpr int csmem = combine_smem_bytes<D>();
-    static bool cattr = false;
-    if (!cattr) cattr = set_smem(comb, csmem);
-    if (!cattr) return KVQ_ERR_CUDA;
+    if (!ensure_smem<decode_combine_mma_kernel<D, HAD, GP>>(csmem)) return KVQ_ERR_CUDA;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(bh);
     lc.blockDim = dim3(128);
