@@ -167,3 +167,31 @@ def test_streaming_flush_equals_bulk_quantize():
         assert bool((cache.tok[i][:, :, :384] == bulk.tok[i][:, :, :384]).all())
         assert bool((cache.chan[i][:, :, :3] == bulk.chan[i][:, :, :3]).all())
         assert bool((cache.off[i][:, :, :3] == bulk.off[i][:, :, :3]).all())
+
+
+def test_batch_row_views_quantize_and_decode_like_the_whole_cache():
+    """kvq_quantize_block on batch-row views (KVCache.rows) stores the same
+    bytes as one call over the whole batch, and decode over the whole cache
+    then gives the same outputs; the views share the cache's memory."""
+    import torch
+    from kv_cache_bit_b200 import kvq
+    mode, d, bits = "nsn+hadamard", 128, 4
+    w = small_workload(mode, d, B=4, H=2, Hq=8, S=384)
+    K, V = synth.kv(w)
+    q = synth.queries(w)
+    cfg, whole = gpu_prefill(mode, d, bits, K, V, cap=512)
+    _, parts = gpu_prefill(mode, d, bits, K, V, cap=512, ntok=0)
+    kd = to_dev(f16bits(K).view(np.int16))
+    vd = to_dev(f16bits(V).view(np.int16))
+    for b0 in (0, 1, 3):
+        b1 = {0: 1, 1: 3, 3: 4}[b0]
+        view = parts.rows(b0, b1)
+        kvq.kvq_quantize_block(cfg, view, kd[b0:b1], vd[b0:b1], 0, w.S)
+    torch.cuda.synchronize()
+    for i in range(2):
+        assert bool((parts.codes[i] == whole.codes[i]).all())
+        assert bool((parts.tok[i] == whole.tok[i]).all())
+        assert bool((parts.chan[i] == whole.chan[i]).all())
+        assert bool((parts.off[i] == whole.off[i]).all())
+    parts.c.len = w.S
+    assert np.array_equal(gpu_decode(cfg, parts, q), gpu_decode(cfg, whole, q))
