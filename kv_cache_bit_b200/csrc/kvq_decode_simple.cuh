@@ -53,6 +53,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(DecodeArgs a) {
     __shared__ float s_lg[kGMax][kT];  // logits, then p * nu
     __shared__ float s_sigv[D], s_offv[D], s_offk[D];
     __shared__ float s_nu[kT], s_s1[kT];
+    __shared__ uint32_t s_vw[kT][RowLayout<D, BITS>::kWords];  // V code rows of the current block
     __shared__ float s_m[kGMax], s_l[kGMax], s_corr[kGMax], s_beta[kGMax], s_qok[kGMax];
 
     const int b = bh / a.H, h = bh % a.H;
@@ -170,16 +171,23 @@ __global__ void __launch_bounds__(128) decode_split_kernel(DecodeArgs a) {
             }
         }
         __syncthreads();
-        // 4. V accumulation, one channel per thread
+        // 4. V accumulation, one channel per thread, from the block's V code
+        //    rows staged in shared memory (thread i copies row i)
+        {
+            const uint8_t* vrow = a.codes[1] + ((size_t)bh * a.cap + (size_t)blk * kT + t) * L::kBytes;
+            uint32_t w[L::kWords];
+            load_words<L::kWords>(vrow, w);
+#pragma unroll
+            for (int k = 0; k < L::kWords; ++k) s_vw[t][k] = w[k];
+        }
+        __syncthreads();
         if (t < D) {
             float aj[kGMax];
 #pragma unroll
             for (int j = 0; j < kGMax; ++j) aj[j] = 0.0f;
-            const uint8_t* vrow = a.codes[1] + ((size_t)bh * a.cap + (size_t)blk * kT) * L::kBytes;
+#pragma unroll 4
             for (int i = 0; i < kT; ++i) {
-                uint32_t w[L::kWords];
-                load_words<L::kWords>(vrow + (size_t)i * L::kBytes, w);
-                const float q = (float)((int)code_at<D, BITS>(w, t) - L::kOff);
+                const float q = (float)((int)code_at<D, BITS>(s_vw[i], t) - L::kOff);
 #pragma unroll
                 for (int j = 0; j < kGMax; ++j)
                     if (j < G) aj[j] += s_lg[j][i] * q;
