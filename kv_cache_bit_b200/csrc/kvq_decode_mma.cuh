@@ -302,6 +302,12 @@ struct SlotLayout {
 };
 
 constexpr int kQS = 128 + 4;  // row stride of the skewed rotated-query table
+// Raw-query table: channel c of head j at j * kQW + c + c / 16.  The NSN
+// offset dot product reads channels 16g + 2k of head t across a warp; the
+// one-word skew per 16 channels and the row stride (8 mod 32 words) put the
+// 32 lanes on 32 different banks.
+constexpr int kQW = 128 + 8;
+__host__ __device__ constexpr int qw_index(int j, int c) { return j * kQW + c + (c >> 4); }
 
 // Partial record of one (segment, head): [m, l, 0, 0, acc[D], acc_o[D]]; the
 // two pad floats keep acc and acc_o 16-byte aligned for vector stores.
@@ -313,7 +319,7 @@ struct MmaSmem {
     static constexpr int kRing0 = 0;
     static constexpr int kBars = kNW * kRing * SlotLayout<D, BITS, MODE>::kStride;
     static constexpr int kQ = kBars + kNW * kRing * 8;        // per warp: q [GP][D] fp32
-    static constexpr int kQs = kQ + kNW * GP * D * 4;         // per warp: skewed scaled rotated q [GP][kQS]
+    static constexpr int kQs = kQ + kNW * GP * kQW * 4;       // per warp: skewed scaled rotated q [GP][kQS]
     static constexpr int kQsc = kQs + kNW * GP * kQS * 4;     // per warp: [GP] scales
     static constexpr int kBytes = kQsc + kNW * GP * 4 + 128;
 };
@@ -400,7 +406,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 
     uint8_t* my_ring = smem_raw + SM::kRing0 + warp * kRing * SL::kStride;
     uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem_raw + SM::kBars) + warp * kRing;
-    float* wq = reinterpret_cast<float*>(smem_raw + SM::kQ) + warp * GP * D;       // [GP][D]
+    float* wq = reinterpret_cast<float*>(smem_raw + SM::kQ) + warp * GP * kQW;     // [GP][kQW], qw_index
     float* wqs = reinterpret_cast<float*>(smem_raw + SM::kQs) + warp * GP * kQS;    // [GP][kQS]
     float* wqsc = reinterpret_cast<float*>(smem_raw + SM::kQsc) + warp * GP;        // [GP]
 
@@ -481,7 +487,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                 const int c = 4 * lane + k;
                 const float qv =
                     (j < G) ? __half2float(a.q[((size_t)b * a.H * G + (size_t)h * G + j) * D + c]) : 0.0f;
-                wq[j * D + c] = qv;
+                wq[qw_index(j, c)] = qv;
                 v[k] = (HAD && a.signs != nullptr && a.signs[c] < 0) ? -qv : qv;
             }
             if constexpr (HAD) {
@@ -558,7 +564,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                         const __half2* okp = reinterpret_cast<const __half2*>(sk + SL::kOff) + 8 * g;
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
-                            const float* qh = &wq[(4 * n + t) * D + 16 * g];
+                            const float* qh = &wq[qw_index(4 * n + t, 16 * g)];  // 16 channels, skew g
                             float s = 0.0f;
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
