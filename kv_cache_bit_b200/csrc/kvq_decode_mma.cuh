@@ -185,6 +185,29 @@ struct KUnpack<2> {
     }
 };
 
+// INT3: the 2-bit field of field index jj (bits 2jj, 2jj + 1 of each half)
+// and the high bit moved to bit 2jj + 2 form e * 4^jj in the mantissa of
+// 1024 + e * 4^jj (two LOP3s); one FMA gives e - 4.
+__device__ __forceinline__ uint32_t lop_or_and(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xF8;" : "=r"(r) : "r"(a), "r"(b), "r"(c));  // a | (b & c)
+    return r;
+}
+
+// x: 2-bit fields at bits 2jj (+16); hs: high bits already at bit 2jj + 2 (+16)
+__device__ __forceinline__ uint32_t dec3(uint32_t x, uint32_t hs, int jj) {
+    const float m = float(1 << (2 * jj));
+    const uint32_t u = lop_and_or(x, 0x00030003u << (2 * jj), kMagic);
+    const uint32_t v = lop_or_and(u, hs, 0x00040004u << (2 * jj));
+    return h2_fma(v, h2c(1.0f / m), h2c(-(1024.0f / m + 4.0f)));
+}
+
+// shift moving bit j to bit 2 (j & 3) + 2
+__device__ __forceinline__ uint32_t hi_to(uint32_t h, int j) {
+    const int sh = 2 * (j & 3) + 2 - j;
+    return sh >= 0 ? (h << sh) : (h >> (-sh));
+}
+
 template <>
 struct KUnpack<3> {
     static constexpr int kSliceBytes = 8;  // low 2-bit plane; plus 4 bytes of the high plane
@@ -194,18 +217,13 @@ struct KUnpack<3> {
         const uint2 v = *reinterpret_cast<const uint2*>(row + 8 * t);
         const uint32_t H = *reinterpret_cast<const uint32_t*>(row + 32 + 4 * t);
         const uint32_t w[2] = {v.x, v.y};
-        const uint32_t one = 0x3C003C00u, four = h2c(4.0f);
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
+            // high bits of channels 16i + j and 16i + 8 + j at bits j and 16 + j
+            const uint32_t Hi = prmt(H, 0u, i ? 0x4342u : 0x4140u);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t lo = dec2<4>(j < 4 ? w[i] : (w[i] >> 8), j & 3);  // e_lo - 4
-                // high bits of channels 16i + j and 16i + j + 8 -> fp16x2 0/1
-                const uint32_t hb = prmt((H >> (16 * i + j)) & 0x101u, 0u, 0x4140u);
-                const uint32_t hf = h2_sub(hb | kMagic, h2c(1024.0f));
-                (void)one;
-                pr[8 * i + j] = h2_fma(hf, four, lo);
-            }
+            for (int j = 0; j < 8; ++j)
+                pr[8 * i + j] = dec3(j < 4 ? w[i] : (w[i] >> 8), hi_to(Hi, j), j & 3);
         }
     }
 };
@@ -265,17 +283,13 @@ struct VUnpack<3> {
         const uint32_t ha = *reinterpret_cast<const uint16_t*>(r0 + 32 + 2 * g);
         const uint32_t hb = *reinterpret_cast<const uint16_t*>(r1 + 32 + 2 * g);
         const uint32_t hh2 = ha | (hb << 16);  // bit k: row 0 channel k; bit 16 + k: row 1 channel k
-        const uint32_t four = h2c(4.0f);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             const uint32_t x = prmt(a, b, hh ? 0x7632u : 0x5410u);
+            const uint32_t hsrc = hh ? (hh2 >> 8) : hh2;  // channel 8hh + j at bits j, 16 + j
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int k = 8 * hh + j;
-                const uint32_t lo = dec2<4>(j < 4 ? x : (x >> 8), j & 3);
-                const uint32_t hf = h2_sub(((hh2 >> k) & 0x00010001u) | kMagic, h2c(1024.0f));
-                pr[k] = h2_fma(hf, four, lo);
-            }
+            for (int j = 0; j < 8; ++j)
+                pr[8 * hh + j] = dec3(j < 4 ? x : (x >> 8), hi_to(hsrc, j), j & 3);
         }
     }
 };
