@@ -622,18 +622,14 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                 for (int o = 16; o; o >>= 1) numax = fmaxf(numax, __shfl_xor_sync(0xffffffffu, numax, o));
                 const int fexp = numax > 0.0f ? 13 - (int)kTau - ceil_log2(numax) : 0;
                 const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
-                float dv[NT][8][4];  // set by the first tile's MMAs
-                float lsum[NT], bsum[NT];
-#pragma unroll
-                for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
+                // ---- scores of the unit's 64 tokens (four independent 16-token tiles)
+                float l2[4][NT][2];
+                bool over = false;
 #pragma unroll
                 for (int m4 = 0; m4 < 4; ++m4) {
-                    // ---- scores of the tile's 16 tokens
                     uint32_t pa[16], pb[16];
                     KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr0) * SL::kRB, t, pa);
                     KUnpack<BITS>::run(sk + SL::kCodes + (16 * m4 + tr1) * SL::kRB, t, pb);
-                    float l2[NT][2];
-                    bool over = false;
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
                         float d0[4], d1[4];
@@ -658,37 +654,39 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                             } else {
                                 kap = __half2float(tk[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
                             }
-                            l2[n][r] = (sv_ * (kap * kcol[n]) + add) * alpha2;
-                            over |= l2[n][r] > m_ref[n] + kTau;
+                            l2[m4][n][r] = (sv_ * (kap * kcol[n]) + add) * alpha2;
+                            over |= l2[m4][n][r] > m_ref[n] + kTau;
                         }
                     }
-                    // ---- rare: move the reference max up and rescale what was accumulated
-                    if (__any_sync(0xffffffffu, over)) {
+                }
+                release(uk);
+                // ---- rare: move the reference max up to the unit's max and rescale
+                if (__any_sync(0xffffffffu, over)) {
 #pragma unroll
-                        for (int n = 0; n < NT; ++n) {
-                            float mx = fmaxf(l2[n][0], l2[n][1]);
+                    for (int n = 0; n < NT; ++n) {
+                        float mx = l2[0][n][0];
 #pragma unroll
-                            for (int o = 4; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                            const float mn = fmaxf(m_ref[n], mx);
-                            const float corr = fast_exp2(m_ref[n] - mn);
-                            m_ref[n] = mn;
-                            l_run[n] *= corr;
-                            lsum[n] *= corr;
-                            bsum[n] *= corr;
+                        for (int m4 = 0; m4 < 4; ++m4) mx = fmaxf(mx, fmaxf(l2[m4][n][0], l2[m4][n][1]));
 #pragma unroll
-                            for (int k = 0; k < 16; ++k) {
-                                acc[n][k] *= corr;
-                                if (MODE == kNsn) acco[n][k] *= corr;
-                            }
-                            if (m4 > 0) {
+                        for (int o = 4; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                        const float mn = fmaxf(m_ref[n], mx);
+                        const float corr = fast_exp2(m_ref[n] - mn);
+                        m_ref[n] = mn;
+                        l_run[n] *= corr;
 #pragma unroll
-                                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                                    for (int k = 0; k < 4; ++k) dv[n][i][k] *= corr;
-                            }
+                        for (int k = 0; k < 16; ++k) {
+                            acc[n][k] *= corr;
+                            if (MODE == kNsn) acco[n][k] *= corr;
                         }
                     }
-                    // ---- P' = p * nu (scaled), as (hi, lo) rows, moved into the B layout
+                }
+                // ---- P' = p * nu (scaled) and the values, tile by tile
+                float dv[NT][8][4];  // set by the first tile's MMAs
+                float lsum[NT], bsum[NT];
+#pragma unroll
+                for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
                     uint32_t bp[NT][2];
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
@@ -704,13 +702,12 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                         nu *= pscale;
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
-                            const float p = fast_exp2(l2[n][r] - m_ref[n]);
+                            const float p = fast_exp2(l2[m4][n][r] - m_ref[n]);
                             lsum[n] += p;
                             if constexpr (MODE == kNsn) bsum[n] += p * s1o;
                             bp[n][r] = movmatrix_t(split_h2(p * nu));
                         }
                     }
-                    // ---- values
                     uint32_t va[16], vb[16];
                     const uint8_t* vbase = sv + SL::kCodes + (16 * m4) * SL::kRB;
                     VUnpack<BITS>::run(vbase + vr0 * SL::kRB, vbase + vr1 * SL::kRB, g, va);
@@ -728,7 +725,6 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                         }
                     }
                 }
-                release(uk);
 #pragma unroll
                 for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
                 // unit epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f
