@@ -93,6 +93,15 @@ __device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
+// D = A * B + C with the same C pair (c0, c1) on rows g and g + 8.
+__device__ __forceinline__ void mma16816_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1, float c0, float c1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%10,%11};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
     float r;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
@@ -138,23 +147,33 @@ __device__ __forceinline__ uint32_t h2c(float v) { return pack_h2(v, v); }
 template <int BITS>
 struct KUnpack;
 
+// INT4: a low nibble OR-ed into fp16 1024 reads 1024 + e, and one
+// subtraction gives q = e - 8.  A high nibble (bits 4..7 of its byte) OR-ed
+// into 1024 reads 1024 + 16 e = 16 (q + 72) and is used in that biased form,
+// one LOP3 per pair with no fp16 arithmetic (kBiased): the kernel scales the
+// other operand of those channels by 1/16 and removes the bias with one MMA
+// against a constant A of -1152 = -16 * 72.
+constexpr float kBiasA = -1152.0f;
+
 template <>
 struct KUnpack<4> {
     static constexpr int kSliceBytes = 16;
+    static constexpr bool kBiased = true;
     __device__ static int ca(int p) { return 8 * (p >> 2) + (p & 3); }
     __device__ static int cb(int p) { return ca(p) + 4; }
-    // row points at the row's first byte; returns pairs of codes (q = e - 8)
+    // row points at the row's first byte; even pairs p hold q = e - 8, odd
+    // pairs (high nibbles) 16 (q + 72)
     __device__ static void run(const uint8_t* row, int t, uint32_t (&pr)[16]) {
         const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * t);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        const uint32_t sub = h2c(1032.0f), s16 = h2c(1.0f / 16.0f), o16 = h2c(-72.0f);
+        const uint32_t sub = h2c(1032.0f);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t W = w[i], W8 = w[i] >> 8;
             pr[4 * i + 0] = h2_sub(lop_and_or(W, 0x000F000Fu, kMagic), sub);
-            pr[4 * i + 1] = h2_fma(lop_and_or(W, 0x00F000F0u, kMagic), s16, o16);
+            pr[4 * i + 1] = lop_and_or(W, 0x00F000F0u, kMagic);
             pr[4 * i + 2] = h2_sub(lop_and_or(W8, 0x000F000Fu, kMagic), sub);
-            pr[4 * i + 3] = h2_fma(lop_and_or(W8, 0x00F000F0u, kMagic), s16, o16);
+            pr[4 * i + 3] = lop_and_or(W8, 0x00F000F0u, kMagic);
         }
     }
 };
@@ -168,6 +187,7 @@ __device__ __forceinline__ uint32_t dec2(uint32_t x, int j) {
 
 template <>
 struct KUnpack<2> {
+    static constexpr bool kBiased = false;
     static constexpr int kSliceBytes = 8;
     __device__ static int ca(int p) { return 16 * (p >> 3) + (p & 7); }
     __device__ static int cb(int p) { return ca(p) + 8; }
@@ -210,6 +230,7 @@ __device__ __forceinline__ uint32_t hi_to(uint32_t h, int j) {
 
 template <>
 struct KUnpack<3> {
+    static constexpr bool kBiased = false;
     static constexpr int kSliceBytes = 8;  // low 2-bit plane; plus 4 bytes of the high plane
     __device__ static int ca(int p) { return 16 * (p >> 3) + (p & 7); }
     __device__ static int cb(int p) { return ca(p) + 8; }
@@ -236,10 +257,11 @@ struct VUnpack;
 
 template <>
 struct VUnpack<4> {
+    static constexpr bool kBiased = true;  // odd channels (high nibbles) as 16 (q + 72)
     __device__ static void run(const uint8_t* r0, const uint8_t* r1, int g, uint32_t (&pr)[16]) {
         const uint2 u0 = *reinterpret_cast<const uint2*>(r0 + 8 * g);
         const uint2 u1 = *reinterpret_cast<const uint2*>(r1 + 8 * g);
-        const uint32_t sub = h2c(1032.0f), s16 = h2c(1.0f / 16.0f), o16 = h2c(-72.0f);
+        const uint32_t sub = h2c(1032.0f);
         const uint32_t a[2] = {u0.x, u0.y}, b[2] = {u1.x, u1.y};
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -250,9 +272,9 @@ struct VUnpack<4> {
                 const uint32_t x8 = x >> 8;
                 const int k = 8 * i + 4 * hh;
                 pr[k + 0] = h2_sub(lop_and_or(x, 0x000F000Fu, kMagic), sub);
-                pr[k + 1] = h2_fma(lop_and_or(x, 0x00F000F0u, kMagic), s16, o16);
+                pr[k + 1] = lop_and_or(x, 0x00F000F0u, kMagic);
                 pr[k + 2] = h2_sub(lop_and_or(x8, 0x000F000Fu, kMagic), sub);
-                pr[k + 3] = h2_fma(lop_and_or(x8, 0x00F000F0u, kMagic), s16, o16);
+                pr[k + 3] = lop_and_or(x8, 0x00F000F0u, kMagic);
             }
         }
     }
@@ -260,6 +282,7 @@ struct VUnpack<4> {
 
 template <>
 struct VUnpack<2> {
+    static constexpr bool kBiased = false;
     __device__ static void run(const uint8_t* r0, const uint8_t* r1, int g, uint32_t (&pr)[16]) {
         const uint32_t a = *reinterpret_cast<const uint32_t*>(r0 + 4 * g);
         const uint32_t b = *reinterpret_cast<const uint32_t*>(r1 + 4 * g);
@@ -277,6 +300,7 @@ struct VUnpack<2> {
 
 template <>
 struct VUnpack<3> {
+    static constexpr bool kBiased = false;
     __device__ static void run(const uint8_t* r0, const uint8_t* r1, int g, uint32_t (&pr)[16]) {
         const uint32_t a = *reinterpret_cast<const uint32_t*>(r0 + 4 * g);
         const uint32_t b = *reinterpret_cast<const uint32_t*>(r1 + 4 * g);
@@ -403,6 +427,8 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     constexpr float kLog2e = 1.4426950408889634f;
     constexpr int QMAX = (1 << (BITS - 1)) - 1;
     constexpr float kTau = 8.0f;  // reference-max slack (log2 units): p <= 2^kTau
+    constexpr bool KB = KUnpack<BITS>::kBiased, VB = VUnpack<BITS>::kBiased;
+    const uint32_t kBiasH2 = h2c(kBiasA);
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     grid_dep_launch();
@@ -544,6 +570,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
             for (int k = 0; k < 16; ++k) { acc[n][k] = 0.0f; acco[n][k] = 0.0f; }
         }
         uint32_t bq[NT][16];
+        float kb[NT][2];  // -1152 * sum of B over the biased pairs (hi, lo columns)
         float qoK[NT];
         __half2 sigv[8], offv[8];
 
@@ -562,8 +589,10 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 #pragma unroll
                         for (int p = 0; p < 16; ++p) {
                             const int ca = KUnpack<BITS>::ca(p), cb = KUnpack<BITS>::cb(p);
-                            const float fa = qrow[ca] * (PCH ? __half2float(sig[ca]) : 1.0f);
-                            const float fb = qrow[cb] * (PCH ? __half2float(sig[cb]) : 1.0f);
+                            // odd pairs meet biased codes 16 (q + 72): 1/16
+                            const float bs = (KB && (p & 1)) ? 0.0625f : 1.0f;
+                            const float fa = qrow[ca] * (PCH ? __half2float(sig[ca]) * bs : bs);
+                            const float fb = qrow[cb] * (PCH ? __half2float(sig[cb]) * bs : bs);
                             const __half2 hh = __floats2half2_rn(fa, fb);
                             if (blo) {
                                 const float2 hf = __half22float2(hh);
@@ -571,6 +600,23 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                             } else {
                                 bq[n][p] = *reinterpret_cast<const uint32_t*>(&hh);
                             }
+                        }
+                    }
+                    if constexpr (KB) {
+                        // bias of the score chains: A = 0 on the even pairs of
+                        // a k-step (a0, a1), -1152 on the odd ones (a2, a3)
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) {
+                            float c0[4], c1[4];
+                            mma16816_z(c0, 0u, 0u, kBiasH2, kBiasH2, bq[n][0], bq[n][1]);
+                            mma16816_z(c1, 0u, 0u, kBiasH2, kBiasH2, bq[n][2], bq[n][3]);
+#pragma unroll
+                            for (int s = 2; s < 8; s += 2) {
+                                mma16816(c0, 0u, 0u, kBiasH2, kBiasH2, bq[n][2 * s], bq[n][2 * s + 1]);
+                                mma16816(c1, 0u, 0u, kBiasH2, kBiasH2, bq[n][2 * s + 2], bq[n][2 * s + 3]);
+                            }
+                            kb[n][0] = c0[0] + c1[0];
+                            kb[n][1] = c0[1] + c1[1];
                         }
                     }
                     if constexpr (MODE == kNsn) {
@@ -633,7 +679,10 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
                         float d0[4], d1[4];
-                        mma16816_z(d0, pa[0], pb[0], pa[1], pb[1], bq[n][0], bq[n][1]);
+                        if constexpr (KB)
+                            mma16816_c(d0, pa[0], pb[0], pa[1], pb[1], bq[n][0], bq[n][1], kb[n][0], kb[n][1]);
+                        else
+                            mma16816_z(d0, pa[0], pb[0], pa[1], pb[1], bq[n][0], bq[n][1]);
                         mma16816_z(d1, pa[2], pb[2], pa[3], pb[3], bq[n][2], bq[n][3]);
 #pragma unroll
                         for (int s = 2; s < 8; s += 2) {
@@ -682,12 +731,13 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                 }
                 // ---- P' = p * nu (scaled) and the values, tile by tile
                 float dv[NT][8][4];  // set by the first tile's MMAs
+                float vbias[NT][2];  // -1152 * sum of the unit's P' (hi, lo columns)
                 float lsum[NT], bsum[NT];
 #pragma unroll
                 for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
+                uint32_t bpa[4][NT][2];
 #pragma unroll
                 for (int m4 = 0; m4 < 4; ++m4) {
-                    uint32_t bp[NT][2];
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
                         const int tok = 16 * m4 + (r ? tr1 : tr0);
@@ -705,13 +755,31 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                             const float p = fast_exp2(l2[m4][n][r] - m_ref[n]);
                             lsum[n] += p;
                             if constexpr (MODE == kNsn) bsum[n] += p * s1o;
-                            bp[n][r] = movmatrix_t(split_h2(p * nu));
+                            bpa[m4][n][r] = movmatrix_t(split_h2(p * nu));
                         }
                     }
+                }
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+                    const uint32_t (&bp)[NT][2] = bpa[m4];
                     uint32_t va[16], vb[16];
                     const uint8_t* vbase = sv + SL::kCodes + (16 * m4) * SL::kRB;
                     VUnpack<BITS>::run(vbase + vr0 * SL::kRB, vbase + vr1 * SL::kRB, g, va);
                     VUnpack<BITS>::run(vbase + (8 + vr0) * SL::kRB, vbase + (8 + vr1) * SL::kRB, g, vb);
+                    if constexpr (VB) {
+                        // every row of this product is the same: carry one
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) {
+                            float r4[4];
+                            if (m4 == 0)
+                                mma16816_z(r4, kBiasH2, kBiasH2, kBiasH2, kBiasH2, bp[n][0], bp[n][1]);
+                            else
+                                mma16816_c(r4, kBiasH2, kBiasH2, kBiasH2, kBiasH2, bp[n][0], bp[n][1], vbias[n][0],
+                                           vbias[n][1]);
+                            vbias[n][0] = r4[0];
+                            vbias[n][1] = r4[1];
+                        }
+                    }
 #pragma unroll
                     for (int tc = 0; tc < 8; ++tc) {
 #pragma unroll
@@ -728,14 +796,23 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 #pragma unroll
                 for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
                 // unit epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f
+                // odd channels (rows g + 8) hold biased codes: the bias is
+                // removed and 1/16 goes into their scale
+                float vbs[NT];
+#pragma unroll
+                for (int n = 0; n < NT; ++n) vbs[n] = VB ? vbias[n][0] + vbias[n][1] : 0.0f;
+                const float pinv_v = VB ? pinv * 0.0625f : pinv;
 #pragma unroll
                 for (int tc = 0; tc < 8; ++tc) {
                     const float2 sg = __half22float2(sigv[tc]);
-                    const float s0 = sg.x * pinv, s1_ = sg.y * pinv;
+                    const float s0 = sg.x * pinv, s1_ = sg.y * pinv_v;
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
                         acc[n][2 * tc] += (dv[n][tc][0] + dv[n][tc][1]) * s0;
-                        acc[n][2 * tc + 1] += (dv[n][tc][2] + dv[n][tc][3]) * s1_;
+                        if constexpr (VB)
+                            acc[n][2 * tc + 1] += ((dv[n][tc][2] + dv[n][tc][3]) + vbs[n]) * s1_;
+                        else
+                            acc[n][2 * tc + 1] += (dv[n][tc][2] + dv[n][tc][3]) * s1_;
                     }
                 }
                 if constexpr (MODE == kNsn) {
