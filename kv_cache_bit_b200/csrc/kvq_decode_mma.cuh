@@ -158,6 +158,7 @@ constexpr float kBiasA = -1152.0f;
 template <>
 struct KUnpack<4> {
     static constexpr int kSliceBytes = 16;
+    static constexpr int kPairGroup = 4;  // pairs 4i + j: channels 8i + j and 8i + 4 + j
     static constexpr bool kBiased = true;
     __device__ static int ca(int p) { return 8 * (p >> 2) + (p & 3); }
     __device__ static int cb(int p) { return ca(p) + 4; }
@@ -188,6 +189,7 @@ __device__ __forceinline__ uint32_t dec2(uint32_t x, int j) {
 template <>
 struct KUnpack<2> {
     static constexpr bool kBiased = false;
+    static constexpr int kPairGroup = 8;  // pairs 8i + j: channels 16i + j and 16i + 8 + j
     static constexpr int kSliceBytes = 8;
     __device__ static int ca(int p) { return 16 * (p >> 3) + (p & 7); }
     __device__ static int cb(int p) { return ca(p) + 8; }
@@ -231,6 +233,7 @@ __device__ __forceinline__ uint32_t hi_to(uint32_t h, int j) {
 template <>
 struct KUnpack<3> {
     static constexpr bool kBiased = false;
+    static constexpr int kPairGroup = 8;  // pairs 8i + j: channels 16i + j and 16i + 8 + j
     static constexpr int kSliceBytes = 8;  // low 2-bit plane; plus 4 bytes of the high plane
     __device__ static int ca(int p) { return 16 * (p >> 3) + (p & 7); }
     __device__ static int cb(int p) { return ca(p) + 8; }
@@ -339,13 +342,19 @@ struct SlotLayout {
     static constexpr int kStride = (kBytesLo + 127) / 128 * 128;
 };
 
-constexpr int kQS = 128 + 4;  // row stride of the skewed rotated-query table
-// Raw-query table: channel c of head j at j * kQW + c + c / 16.  The NSN
-// offset dot product reads channels 16g + 2k of head t across a warp; the
-// one-word skew per 16 channels and the row stride (8 mod 32 words) put the
-// 32 lanes on 32 different banks.
-constexpr int kQW = 128 + 8;
-__host__ __device__ constexpr int qw_index(int j, int c) { return j * kQW + c + (c >> 4); }
+// Rotated-query table (fp32): channel c of head j at j * kQS + c + 4 (c / 32).
+// The B-fragment build reads 16-byte chunks of the 32-channel slice t of one
+// head per thread quad; the 4-word skew per slice puts the four slices of a
+// quarter warp on different banks.
+constexpr int kQS = 128 + 16;
+__host__ __device__ constexpr int qs_index(int j, int c) { return j * kQS + c + 4 * (c >> 5); }
+// Raw-query table (fp16, exact copies of the query): channels (c, c + 1),
+// c even, of head j in 32-bit word j * kQWW + c / 2 + c / 64.  The NSN offset
+// dot product reads the words of channels 16g + 2k of head t across a warp;
+// the row stride (2 mod 32 words) and the one-word skew per 64 channels put
+// the 32 lanes on 32 different banks.
+constexpr int kQWW = 64 + 2;
+__host__ __device__ constexpr int qw_word(int j, int c) { return j * kQWW + (c >> 1) + (c >> 6); }
 
 // Partial record of one (segment, head): [m, l, 0, 0, acc[D], acc_o[D]]; the
 // two pad floats keep acc and acc_o 16-byte aligned for vector stores.
@@ -356,8 +365,8 @@ template <int D, int BITS, int MODE, int GP>
 struct MmaSmem {
     static constexpr int kRing0 = 0;
     static constexpr int kBars = kNW * kRing * SlotLayout<D, BITS, MODE>::kStride;
-    static constexpr int kQ = kBars + kNW * kRing * 8;        // per warp: q [GP][D] fp32
-    static constexpr int kQs = kQ + kNW * GP * kQW * 4;       // per warp: skewed scaled rotated q [GP][kQS]
+    static constexpr int kQ = kBars + kNW * kRing * 8;        // per warp: raw q [GP][kQWW] fp16 pairs
+    static constexpr int kQs = kQ + kNW * GP * kQWW * 4;      // per warp: skewed scaled rotated q [GP][kQS]
     static constexpr int kQsc = kQs + kNW * GP * kQS * 4;     // per warp: [GP] scales
     static constexpr int kBytes = kQsc + kNW * GP * 4 + 128;
 };
@@ -446,7 +455,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 
     uint8_t* my_ring = smem_raw + SM::kRing0 + warp * kRing * SL::kStride;
     uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem_raw + SM::kBars) + warp * kRing;
-    float* wq = reinterpret_cast<float*>(smem_raw + SM::kQ) + warp * GP * kQW;     // [GP][kQW], qw_index
+    uint32_t* wqw = reinterpret_cast<uint32_t*>(smem_raw + SM::kQ) + warp * GP * kQWW;  // [GP][kQWW], qw_word
     float* wqs = reinterpret_cast<float*>(smem_raw + SM::kQs) + warp * GP * kQS;    // [GP][kQS]
     float* wqsc = reinterpret_cast<float*>(smem_raw + SM::kQsc) + warp * GP;        // [GP]
 
@@ -521,14 +530,18 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
         // ---- segment prologue: this pair's queries, rotated and scaled (lane owns 4 channels)
 #pragma unroll
         for (int j = 0; j < GP; ++j) {
-            float v[4];
+            const uint2 raw = (j < G) ? *reinterpret_cast<const uint2*>(
+                                            a.q + ((size_t)b * a.H * G + (size_t)h * G + j) * D + 4 * lane)
+                                      : make_uint2(0u, 0u);
+            wqw[qw_word(j, 4 * lane)] = raw.x;
+            wqw[qw_word(j, 4 * lane + 2)] = raw.y;
+            const float2 q01 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+            const float2 q23 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+            float v[4] = {q01.x, q01.y, q23.x, q23.y};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int c = 4 * lane + k;
-                const float qv =
-                    (j < G) ? __half2float(a.q[((size_t)b * a.H * G + (size_t)h * G + j) * D + c]) : 0.0f;
-                wq[qw_index(j, c)] = qv;
-                v[k] = (HAD && a.signs != nullptr && a.signs[c] < 0) ? -qv : qv;
+                if (HAD && a.signs != nullptr && a.signs[c] < 0) v[k] = -v[k];
             }
             if constexpr (HAD) {
                 const float x0_ = v[0] + v[1], x1_ = v[0] - v[1], x2_ = v[2] + v[3], x3_ = v[2] - v[3];
@@ -551,8 +564,9 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
             const float qsc = bound > 0.0f ? pow2i(13 - ceil_log2(bound)) : 1.0f;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const int c = 4 * lane + k;
-                wqs[j * kQS + c + (c >> 5)] = v[k] * qsc;
+                // odd channels meet biased INT4 codes 16 (q + 72): 1/16
+                const float bs = (KB && (k & 1)) ? 0.0625f : 1.0f;
+                wqs[qs_index(j, 4 * lane + k)] = v[k] * qsc * bs;
             }
             if (lane == 0) wqsc[j] = qsc;
         }
@@ -581,24 +595,44 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                 if (!wait_unit(uk)) { ok = false; break; }
                 uint8_t* sk = my_ring + (uk % kRing) * SL::kStride;
                 if (half == 0) {
-                    // B fragments: q' = qs * sigma^K as (hi, lo) fp16 parts
-                    const __half* sig = reinterpret_cast<const __half*>(sk + SL::kChan) + 32 * t;
+                    // B fragments: q' = qs * sigma^K as (hi, lo) fp16 parts; a
+                    // group of PG pairs takes 2 PG channels of the slice
+                    constexpr int PG = KUnpack<BITS>::kPairGroup;
+                    const uint4* sg4 = reinterpret_cast<const uint4*>(sk + SL::kChan) + 4 * t;  // slice t
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
-                        const float* qrow = &wqs[(4 * n + (g >> 1)) * kQS + 33 * t];
+                        const float4* q4 = reinterpret_cast<const float4*>(&wqs[qs_index(4 * n + (g >> 1), 32 * t)]);
 #pragma unroll
-                        for (int p = 0; p < 16; ++p) {
-                            const int ca = KUnpack<BITS>::ca(p), cb = KUnpack<BITS>::cb(p);
-                            // odd pairs meet biased codes 16 (q + 72): 1/16
-                            const float bs = (KB && (p & 1)) ? 0.0625f : 1.0f;
-                            const float fa = qrow[ca] * (PCH ? __half2float(sig[ca]) * bs : bs);
-                            const float fb = qrow[cb] * (PCH ? __half2float(sig[cb]) * bs : bs);
-                            const __half2 hh = __floats2half2_rn(fa, fb);
-                            if (blo) {
-                                const float2 hf = __half22float2(hh);
-                                bq[n][p] = cvt_h2(fa - hf.x, fb - hf.y);
-                            } else {
-                                bq[n][p] = *reinterpret_cast<const uint32_t*>(&hh);
+                        for (int grp = 0; grp < 16 / PG; ++grp) {
+                            float qv[2 * PG], sv[2 * PG];
+#pragma unroll
+                            for (int v = 0; v < PG / 2; ++v) {
+                                const float4 f = q4[grp * (PG / 2) + v];
+                                qv[4 * v] = f.x; qv[4 * v + 1] = f.y; qv[4 * v + 2] = f.z; qv[4 * v + 3] = f.w;
+                            }
+#pragma unroll
+                            for (int v = 0; v < PG / 4; ++v) {
+                                const uint4 hv = PCH ? sg4[grp * (PG / 4) + v] : make_uint4(0u, 0u, 0u, 0u);
+                                const uint32_t w4[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+                                for (int w = 0; w < 4; ++w) {
+                                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[w]));
+                                    sv[8 * v + 2 * w] = PCH ? f.x : 1.0f;
+                                    sv[8 * v + 2 * w + 1] = PCH ? f.y : 1.0f;
+                                }
+                            }
+#pragma unroll
+                            for (int j = 0; j < PG; ++j) {
+                                const int p = PG * grp + j;
+                                const float fa = qv[j] * sv[j];            // channel ca(p)
+                                const float fb = qv[PG + j] * sv[PG + j];  // channel cb(p)
+                                const __half2 hh = __floats2half2_rn(fa, fb);
+                                if (blo) {
+                                    const float2 hf = __half22float2(hh);
+                                    bq[n][p] = cvt_h2(fa - hf.x, fb - hf.y);
+                                } else {
+                                    bq[n][p] = *reinterpret_cast<const uint32_t*>(&hh);
+                                }
                             }
                         }
                     }
@@ -624,12 +658,13 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                         const __half2* okp = reinterpret_cast<const __half2*>(sk + SL::kOff) + 8 * g;
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
-                            const float* qh = &wq[qw_index(4 * n + t, 16 * g)];  // 16 channels, skew g
+                            const uint32_t* qh = &wqw[qw_word(4 * n + t, 16 * g)];  // channels 16g .. 16g + 15
                             float s = 0.0f;
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
                                 const float2 o2 = __half22float2(okp[k]);
-                                s += qh[2 * k] * o2.x + qh[2 * k + 1] * o2.y;
+                                const float2 q2 = __half22float2(*reinterpret_cast<const __half2*>(&qh[k]));
+                                s += q2.x * o2.x + q2.y * o2.y;
                             }
 #pragma unroll
                             for (int o = 4; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
