@@ -579,7 +579,10 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
         for (int n = 0; n < NT; ++n) {
             m_ref[n] = -INFINITY;
             l_run[n] = 0.0f;
-            kcol[n] = 1.0f / wqsc[4 * n + t];
+            // 2^-qsc with the softmax scale (log2 units) and the fixed token
+            // factor of the mode folded in
+            kcol[n] = alpha2 * ((MODE == kNsn && !HAD) ? a.sqd : (MODE == kNsep && HAD) ? a.rsqd : 1.0f) /
+                      wqsc[4 * n + t];
 #pragma unroll
             for (int k = 0; k < 16; ++k) { acc[n][k] = 0.0f; acco[n][k] = 0.0f; }
         }
@@ -668,7 +671,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                             }
 #pragma unroll
                             for (int o = 4; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                            qoK[n] = s;
+                            qoK[n] = s * alpha2;
                         }
                     }
                 }
@@ -703,6 +706,9 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                 for (int o = 16; o; o >>= 1) numax = fmaxf(numax, __shfl_xor_sync(0xffffffffu, numax, o));
                 const int fexp = numax > 0.0f ? 13 - (int)kTau - ceil_log2(numax) : 0;
                 const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
+                // 2^f with the fixed token factor of the mode
+                const float pscale_m =
+                    pscale * ((MODE == kNsn && !HAD) ? a.sqd : (MODE == kNsep && HAD) ? a.rsqd : 1.0f);
                 // ---- scores of the unit's 64 tokens (four independent 16-token tiles)
                 float l2[4][NT][2];
                 bool over = false;
@@ -730,15 +736,13 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                         for (int r = 0; r < 2; ++r) {
                             const int tok = 16 * m4 + (r ? tr1 : tr0);
                             const float sv_ = (d0[2 * r] + d0[2 * r + 1]) + (d1[2 * r] + d1[2 * r + 1]);
-                            float kap, add = 0.0f;
+                            // logit in log2 units: kap (sv q'.k + q.o) alpha2 for NSN
                             if constexpr (MODE == kNsn) {
                                 const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tk)[tok]);
-                                kap = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
-                                add = s12.x * qoK[n];
+                                l2[m4][n][r] = s12.x * fmaf(sv_, s12.y * kcol[n], qoK[n]);
                             } else {
-                                kap = __half2float(tk[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                                l2[m4][n][r] = sv_ * (__half2float(tk[tok]) * kcol[n]);
                             }
-                            l2[m4][n][r] = (sv_ * (kap * kcol[n]) + add) * alpha2;
                             over |= l2[m4][n][r] > m_ref[n] + kTau;
                         }
                     }
@@ -776,15 +780,14 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
                         const int tok = 16 * m4 + (r ? tr1 : tr0);
-                        float nu, s1o = 0.0f;
+                        float nu, s1o = 0.0f;  // nu: the token's value scale times 2^f
                         if constexpr (MODE == kNsn) {
                             const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
                             s1o = s12.x;
-                            nu = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
+                            nu = s12.x * (s12.y * pscale_m);
                         } else {
-                            nu = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                            nu = __half2float(tv[tok]) * pscale_m;
                         }
-                        nu *= pscale;
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
                             const float p = fast_exp2(l2[m4][n][r] - m_ref[n]);
