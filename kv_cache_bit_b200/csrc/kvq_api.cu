@@ -271,9 +271,9 @@ kvq_status launch_decode_mma(DecodeArgs a, int bh, cudaStream_t st) {
     }
     // the combine kernel is a programmatic dependent of the decode kernel:
     // its residual phase overlaps the decode kernel's tail
-    auto comb = decode_combine_mma_kernel<D, HAD, GP>;
+    auto comb = decode_combine_mma_kernel<D, GP>;
     constexpr int csmem = combine_smem_bytes<D>();
-    if (!ensure_smem<decode_combine_mma_kernel<D, HAD, GP>>(csmem)) return KVQ_ERR_CUDA;
+    if (!ensure_smem<decode_combine_mma_kernel<D, GP>>(csmem)) return KVQ_ERR_CUDA;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(bh);
     lc.blockDim = dim3(128);

@@ -6,8 +6,8 @@
 // CTA; warp w of a CTA takes blocks w, w + kNW, ... of the range (so the
 // warps of a CTA stream neighbouring blocks) through its own ring of kRing
 // shared-memory slots, and writes one partial softmax state per pair segment
-// it covers.  A
-// slot holds one tensor's half block (packed codes, per-token parameters,
+// it covers, with the code term already rotated back to the original
+// domain.  A slot holds one tensor's half block (packed codes, per-token parameters,
 // and on the first half the channel scales and NSN means), brought in by 1-D
 // bulk copies (no multicast) that complete on the slot's mbarrier.  Per block
 // the unit order is K lo, V lo, K hi, V hi.  decode_combine_mma_kernel then
@@ -356,10 +356,11 @@ __host__ __device__ constexpr int qs_index(int j, int c) { return j * kQS + c + 
 constexpr int kQWW = 64 + 2;
 __host__ __device__ constexpr int qw_word(int j, int c) { return j * kQWW + (c >> 1) + (c >> 6); }
 
-// Partial record of one (segment, head): [m, l, 0, 0, acc[D], acc_o[D]]; the
-// two pad floats keep acc and acc_o 16-byte aligned for vector stores.
+// Partial record of one (segment, head): [m, l, 0, 0, acc[D]] with acc in the
+// original domain (the code term already rotated back, plus the NSN offset
+// term); the two pad floats keep acc 16-byte aligned for vector stores.
 template <int D>
-__host__ __device__ constexpr int part_stride() { return 4 + 2 * D; }
+__host__ __device__ constexpr int part_stride() { return 4 + D; }
 
 template <int D, int BITS, int MODE, int GP>
 struct MmaSmem {
@@ -424,8 +425,8 @@ __device__ __forceinline__ uint32_t split_h2(float x) {
 // (0 = hi, 1 = lo) of head 4n + j.  Thread (g, t) of a warp therefore owns
 // head 4n + t of every n-tile in the C fragments and sums its two columns.
 // Partial state of a (warp, pair) segment goes to slot part_slot() of a.part:
-// [m (log2 units), l, pad, pad, acc[D] (rotated domain), acc_o[D] (original
-// domain)] per head (part_stride floats).
+// [m (log2 units), l, pad, pad, acc[D] (original domain)] per head
+// (part_stride floats).
 template <int D, int BITS, int MODE, bool HAD, int GP>
 __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "tensor-core decode is built for head dim 128");
@@ -877,6 +878,39 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
         for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) l_run[n] += __shfl_xor_sync(0xffffffffu, l_run[n], o);
+        // code term back to the original domain: acc <- s (.) H acc (the
+        // thread's 16 channels 16g + k are the low four index bits, the
+        // lanes 4g + t with the same t the high three), plus the offset term
+        if constexpr (HAD) {
+            const bool sg_ok = a.signs != nullptr;
+            const uint4 sraw = sg_ok ? *reinterpret_cast<const uint4*>(a.signs + 16 * g) : make_uint4(0u, 0u, 0u, 0u);
+            const int8_t* sgn = reinterpret_cast<const int8_t*>(&sraw);
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+#pragma unroll
+                for (int m = 1; m < 16; m <<= 1) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        if (k & m) continue;
+                        const float x0_ = acc[n][k], x1_ = acc[n][k + m];
+                        acc[n][k] = x0_ + x1_;
+                        acc[n][k + m] = x0_ - x1_;
+                    }
+                }
+#pragma unroll
+                for (int m = 4; m < 32; m <<= 1) {
+                    const bool upper = (lane & m) != 0;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float o = __shfl_xor_sync(0xffffffffu, acc[n][k], m);
+                        acc[n][k] = upper ? (o - acc[n][k]) : (acc[n][k] + o);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    if (sgn[k] < 0) acc[n][k] = -acc[n][k];
+            }
+        }
         constexpr int PS = part_stride<D>();
         float* pp = a.part + ((size_t)part_slot(cta, warp, pair) * G) * PS;
 #pragma unroll
@@ -887,10 +921,11 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                 if (g == 0) *reinterpret_cast<float4*>(pj) = make_float4(m_ref[n], l_run[n], 0.0f, 0.0f);
 #pragma unroll
                 for (int k = 0; k < 16; k += 4) {
-                    *reinterpret_cast<float4*>(pj + 4 + 16 * g + k) =
-                        make_float4(acc[n][k], acc[n][k + 1], acc[n][k + 2], acc[n][k + 3]);
-                    *reinterpret_cast<float4*>(pj + 4 + D + 16 * g + k) =
-                        make_float4(acco[n][k], acco[n][k + 1], acco[n][k + 2], acco[n][k + 3]);
+                    float4 v4 = make_float4(acc[n][k], acc[n][k + 1], acc[n][k + 2], acc[n][k + 3]);
+                    if constexpr (MODE == kNsn) {
+                        v4.x += acco[n][k]; v4.y += acco[n][k + 1]; v4.z += acco[n][k + 2]; v4.w += acco[n][k + 3];
+                    }
+                    *reinterpret_cast<float4*>(pj + 4 + 16 * g + k) = v4;
                 }
             }
         }
@@ -912,19 +947,18 @@ __host__ __device__ constexpr int combine_smem_bytes() {
     return kT * D * 2;  // the residual value rows, fp16
 }
 
-// Merge the partials of one (batch, kv head) pair with its fp16 residual
-// tokens; inverse rotation of the code term; division by the softmax sum.
+// Merge the partials of one (batch, kv head) pair (already in the original
+// domain) with its fp16 residual tokens; division by the softmax sum.
 // Thread c owns output channel c of every query head.
 //
 // The kernel is built to keep its chain of dependent memory round trips
 // short.  Before waiting for the decode kernel (programmatic dependent
-// launch) it loads the queries, the rotation signs and all residual keys at
-// once, copies the residual value rows to shared memory with cp.async, and
+// launch) it loads the queries and all residual keys at once, copies the residual value rows to shared memory with cp.async, and
 // merges the residual tokens as the first softmax chunk.  After the wait,
 // thread i fetches (m, l) of candidate (CTA, warp) partial i for every head;
 // the accumulators of the first KB candidates are requested before the
 // per-head weights are formed, so their latency overlaps that work.
-template <int D, bool HAD, int GP>
+template <int D, int GP>
 __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "one channel per thread");
     constexpr float kLog2e = 1.4426950408889634f;
@@ -940,8 +974,6 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     __shared__ float s_pm[GP][128], s_pl[GP][128];  // candidate m, then weight; l
     __shared__ int s_slot[128];
     __shared__ float s_M[GP], s_L[GP], s_f[GP];
-    __shared__ float s_a[GP][D];
-    __shared__ float s_sg[D];
     const float alpha2 = a.scale * kLog2e;
     const int c = tid;
 
@@ -951,7 +983,6 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
         const int nchunk = rlen * (D * 2 / 16);
         for (int i = tid; i < nchunk; i += 128) cp_async16(reinterpret_cast<uint8_t*>(s_rv) + 16 * i, rv + 16 * i);
     }
-    if constexpr (HAD) s_sg[c] = (a.signs != nullptr && a.signs[c] < 0) ? -1.0f : 1.0f;
     if (tid < GP) { s_M[tid] = -INFINITY; s_L[tid] = 0.0f; s_f[tid] = 0.0f; }
     // residual logits on the tensor cores: K rows (fp16) times the queries
     // (fp16, exact); lane (g, t) loads channels 32t .. 32t + 31 of tokens
@@ -1082,7 +1113,7 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
         }
         __syncthreads();
         const int n = min(128, ncand - base);
-        float av[KB][GP], aov[KB][GP];
+        float av[KB][GP];
         auto load_batch = [&](int i0) {
 #pragma unroll
             for (int k = 0; k < KB; ++k) {
@@ -1092,7 +1123,6 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
                 for (int j = 0; j < GP; ++j) {
                     const bool use = o >= 0 && j < G;
                     av[k][j] = use ? pk[(size_t)j * PS + 4 + c] : 0.0f;
-                    aov[k][j] = use ? pk[(size_t)j * PS + 4 + D + c] : 0.0f;
                 }
             }
         };
@@ -1111,35 +1141,8 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
                 for (int j = 0; j < GP; ++j) {
                     const float wt = (i0 + k < n && j < G) ? s_pm[j][i0 + k] : 0.0f;
                     A[j] += wt * av[k][j];
-                    AO[j] += wt * aov[k][j];
                 }
             }
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int j = 0; j < GP; ++j)
-        if (j < G) s_a[j][c] = A[j];
-    __syncthreads();
-    if constexpr (HAD) {
-        // inverse rotation of the code term: warp w transforms heads w, w + 4 (lanes own 4 channels)
-        for (int j = warp; j < G; j += 4) {
-            float v[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) v[k] = s_a[j][4 * lane + k];
-            const float x0 = v[0] + v[1], x1 = v[0] - v[1], x2 = v[2] + v[3], x3 = v[2] - v[3];
-            v[0] = x0 + x2; v[2] = x0 - x2; v[1] = x1 + x3; v[3] = x1 - x3;
-#pragma unroll
-            for (int m = 1; m < 32; m <<= 1) {
-                const bool upper = (lane & m) != 0;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float o = __shfl_xor_sync(0xffffffffu, v[k], m);
-                    v[k] = upper ? (o - v[k]) : (v[k] + o);
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) s_a[j][4 * lane + k] = v[k] * s_sg[4 * lane + k];
         }
         __syncthreads();
     }
@@ -1147,7 +1150,7 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     for (int j = 0; j < GP; ++j) {
         if (j >= G) continue;
         const float L = s_L[j];
-        a.out[((size_t)b * a.H * G + (size_t)h * G + j) * D + c] = L > 0.0f ? (s_a[j][c] + AO[j]) / L : 0.0f;
+        a.out[((size_t)b * a.H * G + (size_t)h * G + j) * D + c] = L > 0.0f ? (A[j] + AO[j]) / L : 0.0f;
     }
 }
 
