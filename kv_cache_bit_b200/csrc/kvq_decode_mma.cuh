@@ -953,11 +953,12 @@ __host__ __device__ constexpr int combine_smem_bytes() {
 //
 // The kernel is built to keep its chain of dependent memory round trips
 // short.  Before waiting for the decode kernel (programmatic dependent
-// launch) it loads the queries and all residual keys at once, copies the residual value rows to shared memory with cp.async, and
-// merges the residual tokens as the first softmax chunk.  After the wait,
-// thread i fetches (m, l) of candidate (CTA, warp) partial i for every head;
-// the accumulators of the first KB candidates are requested before the
-// per-head weights are formed, so their latency overlaps that work.
+// launch) it loads the queries and all residual keys at once, copies the
+// residual value rows to shared memory with cp.async, merges the residual
+// tokens as the first softmax chunk and lists the candidate (CTA, warp)
+// partial slots.  After the wait, thread i fetches (m, l) of candidate i for
+// every head while the accumulators of the first KB candidates are fetched
+// in the same round trip.
 template <int D, int GP>
 __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "one channel per thread");
@@ -1090,28 +1091,23 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     };
     const float* pbase = a.part + (size_t)part_slot(0, 0, pair) * G * PS;
     const int ncand = (c_last - c_first + 1) * kNW;
-    __syncthreads();  // the residual phase is done with s_pm
+    // slot offsets of candidates base .. base + 127 (-1: no partial); they
+    // depend on the split only, so the first chunk is listed before the wait
+    auto fill_slots = [&](int base) {
+        const int i = base + tid;
+        const bool valid = i < ncand && has_part(c_first + i / kNW, i % kNW);
+        s_slot[tid] = valid ? (int)(part_slot(c_first + i / kNW, i % kNW, pair) - part_slot(0, 0, pair)) : -1;
+    };
+    fill_slots(0);
+    __syncthreads();  // slots listed; the residual phase is done with s_pm
 
     // ---- the decode kernel's partials
     grid_dep_wait();
     for (int base = 0; base < ncand; base += 128) {
-        {
-            const int i = base + tid;
-            const bool valid = i < ncand && has_part(c_first + i / kNW, i % kNW);
-            const int off = valid ? (int)(part_slot(c_first + i / kNW, i % kNW, pair) - part_slot(0, 0, pair)) : -1;
-            s_slot[tid] = off;
-            float2 ml[GP];
-            const float* pk = pbase + (size_t)(valid ? off : 0) * G * PS;
-#pragma unroll
-            for (int j = 0; j < GP; ++j)
-                ml[j] = (valid && j < G) ? *reinterpret_cast<const float2*>(pk + (size_t)j * PS)
-                                         : make_float2(-INFINITY, 0.0f);
-#pragma unroll
-            for (int j = 0; j < GP; ++j) {
-                if (j < G) { s_pm[j][tid] = ml[j].x; s_pl[j][tid] = ml[j].y; }
-            }
+        if (base > 0) {
+            fill_slots(base);
+            __syncthreads();
         }
-        __syncthreads();
         const int n = min(128, ncand - base);
         float av[KB][GP];
         auto load_batch = [&](int i0) {
@@ -1126,7 +1122,22 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
                 }
             }
         };
+        // the first accumulators and every candidate's (m, l) in one round trip
         load_batch(0);
+        {
+            const int off = s_slot[tid];
+            float2 ml[GP];
+            const float* pk = pbase + (size_t)(off >= 0 ? off : 0) * G * PS;
+#pragma unroll
+            for (int j = 0; j < GP; ++j)
+                ml[j] = (off >= 0 && j < G) ? *reinterpret_cast<const float2*>(pk + (size_t)j * PS)
+                                            : make_float2(-INFINITY, 0.0f);
+#pragma unroll
+            for (int j = 0; j < GP; ++j) {
+                if (j < G) { s_pm[j][tid] = ml[j].x; s_pl[j][tid] = ml[j].y; }
+            }
+        }
+        __syncthreads();
         merge_chunk(n);
         __syncthreads();
 #pragma unroll
