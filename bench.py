@@ -466,8 +466,11 @@ def run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, de
     timed region, and every decode output is copied back.  The copies run on
     their own streams and overlap the kernels: the prefill moves in batch
     chunks, each quantized as soon as it has landed (kvq_quantize_block on a
-    batch-row view of the cache); the next decode step's inputs and the last
-    step's output move while the current step computes (double buffers,
+    batch-row view of the cache), and the next step's prefill moves while
+    this step decodes (its device buffer is free once this step's quantize
+    calls have read it); the streamed tokens' inputs of a step move in one
+    copy per tensor at its start (double-buffered across steps) and each
+    decode output moves back while the next token computes (double buffers,
     ordered by events)."""
     import torch
     from kv_cache_bit_b200 import kvq
@@ -475,64 +478,63 @@ def run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, de
     Kh, Vh, ksh, vsh, qsh = pin(K), pin(V), pin(ks), pin(vs), pin(qs)
     Kd = torch.empty_like(Kh, device=dev)
     Vd = torch.empty_like(Vh, device=dev)
-    ktok = [torch.empty_like(ksh[0], device=dev) for _ in range(2)]
-    vtok = [torch.empty_like(vsh[0], device=dev) for _ in range(2)]
-    qd = [torch.empty_like(qsh[0], device=dev) for _ in range(2)]
+    # the streamed tokens' inputs of a whole step, double-buffered across steps
+    tokd = [[torch.empty_like(x, device=dev) for x in (ksh, vsh, qsh)] for _ in range(2)]
     outd = [out, torch.empty_like(out)]
     outh = torch.empty((w.stream,) + tuple(out.shape), dtype=torch.float32).pin_memory()
-    h2d_s = torch.cuda.Stream(dev)
+    h2d_s = torch.cuda.Stream(dev)  # streamed-token inputs
+    pre_s = torch.cuda.Stream(dev)  # prefill chunks
     d2h_s = torch.cuda.Stream(dev)
     nchunk = 8 if w.B % 8 == 0 else 1
     bc = w.B // nchunk
     views = [cache.rows(c * bc, (c + 1) * bc) for c in range(nchunk)]
     ev = lambda: torch.cuda.Event()
-    # events carried across steps: the input buffers' last reader, the output
-    # buffers' last copy
-    in_ready = [None, None]
-    in_free = [None, None]
+    # events carried across steps: each buffer's last reader or last copy
+    tok_free = [None, None]
     out_free = [None, None]
+    pre_free = [None]  # the prefill buffer's last reader (the previous step's quantize)
+    parity = [0]
 
     def step():
+        tb = parity[0]
+        parity[0] ^= 1
+        with torch.cuda.stream(h2d_s):
+            if tok_free[tb] is not None:
+                h2d_s.wait_event(tok_free[tb])
+            for dst, src in zip(tokd[tb], (ksh, vsh, qsh)):
+                dst.copy_(src, non_blocking=True)
+            tok_ready = ev()
+            tok_ready.record(h2d_s)
         cache.c.len = 0
-        # prefill: chunk c copied on h2d_s, quantized on the compute stream
+        # prefill: chunk c copied on pre_s, quantized on the compute stream
         for c in range(nchunk):
             rows = slice(c * bc, (c + 1) * bc)
-            with torch.cuda.stream(h2d_s):
+            with torch.cuda.stream(pre_s):
+                if c == 0 and pre_free[0] is not None:
+                    pre_s.wait_event(pre_free[0])
                 Kd[rows].copy_(Kh[rows], non_blocking=True)
                 Vd[rows].copy_(Vh[rows], non_blocking=True)
-                e = ev(); e.record(h2d_s)
+                e = ev(); e.record(pre_s)
             stream.wait_event(e)
             views[c].c.len = 0
             kvq.kvq_quantize_block(cfg, views[c], Kd[rows], Vd[rows], 0, w.S, stream)
+        pre_free[0] = ev(); pre_free[0].record(stream)
         cache.c.len = w.S
 
-        def fetch(i):
-            j = i % 2
-            with torch.cuda.stream(h2d_s):
-                if in_free[j] is not None:
-                    h2d_s.wait_event(in_free[j])
-                ktok[j].copy_(ksh[i], non_blocking=True)
-                vtok[j].copy_(vsh[i], non_blocking=True)
-                qd[j].copy_(qsh[i], non_blocking=True)
-                in_ready[j] = ev(); in_ready[j].record(h2d_s)
-
-        if w.stream:
-            fetch(0)
+        kd, vd, qd = tokd[tb]
+        stream.wait_event(tok_ready)
         for i in range(w.stream):
             j = i % 2
-            if i + 1 < w.stream:
-                fetch(i + 1)
-            stream.wait_event(in_ready[j])
             if out_free[j] is not None:
                 stream.wait_event(out_free[j])
-            kvq.kvq_append_token(cfg, cache, ktok[j], vtok[j], stream)
-            kvq.kvq_decode_attention(cfg, cache, qd[j], w.Hq, 0.0, outd[j], ws, ws_bytes, stream)
+            kvq.kvq_append_token(cfg, cache, kd[i], vd[i], stream)
+            kvq.kvq_decode_attention(cfg, cache, qd[i], w.Hq, 0.0, outd[j], ws, ws_bytes, stream)
             done = ev(); done.record(stream)
-            in_free[j] = done
             with torch.cuda.stream(d2h_s):
                 d2h_s.wait_event(done)
                 outh[i].copy_(outd[j], non_blocking=True)
                 out_free[j] = ev(); out_free[j].record(d2h_s)
+        tok_free[tb] = ev(); tok_free[tb].record(stream)
         # the step ends when its last output is on the host
         for e in out_free:
             if e is not None:
@@ -540,13 +542,14 @@ def run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, de
 
     step()
     torch.cuda.synchronize()
-    steps = max(1, min(args.steps, 3))
+    steps = max(1, min(args.steps, 5))
     if world > 1:
         torch.distributed.barrier()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
     h2d_s.wait_event(a)
+    pre_s.wait_event(a)
     d2h_s.wait_event(a)
     for _ in range(steps):
         step()
@@ -558,7 +561,8 @@ def run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, de
     same = bool(torch.equal(outh[w.stream - 1].to(dev), ref_last)) if w.stream else None
     return {"value": world * step_bytes / (ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
-            "overlap": f"copies on two streams; prefill in {nchunk} batch chunks",
+            "overlap": f"copies on three streams; prefill in {nchunk} batch chunks, the next step's prefill "
+                       "and streamed-token inputs copied during this step's decode loop",
             "last_output_equals_device_run": same}
 
 
