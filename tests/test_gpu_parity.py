@@ -91,6 +91,9 @@ DECODE_CASES = [
     ("nsn", 128, 4, 1, 2, 4, 256, 0),
     ("nsep+pchan", 128, 2, 1, 2, 16, 256, 0),     # g = 8
     ("nsep+pchan", 64, 3, 1, 2, 2, 128, 1),
+    # rotation with two n-tiles of query heads (G = 6 and 8)
+    ("rht+nsep+pchan", 128, 4, 1, 2, 12, 384, 9),
+    ("nsn+hadamard", 128, 4, 1, 1, 8, 256, 3),
     # one long pair spread over every CTA of the persistent grid: more than
     # 128 candidate partials per pair in the combine
     ("nsn+hadamard", 128, 4, 1, 1, 4, 200 * 128, 17),
