@@ -468,6 +468,7 @@ kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t
     if (t0 + ntok > (cache->len / kT) * kT) return KVQ_ERR_INVALID_ARG;
     DequantLaunch L;
     L.a.codes = cache->codes[tensor];
+    L.a.pairv = tensor;  // V rows of head dim 128 are pair-interleaved
     L.a.tok = reinterpret_cast<const __half*>(cache->tok[tensor]);
     L.a.chan = reinterpret_cast<const __half*>(cache->chan[tensor]);
     L.a.off = reinterpret_cast<const __half*>(cache->off[tensor]);

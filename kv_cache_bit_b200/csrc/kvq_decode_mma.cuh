@@ -21,8 +21,9 @@
 //           keeps ~22 bits; codes are exact in fp16).
 //   softmax logits in the log2 domain, online max/sum per head.
 //   values  Acc[c][col] += sum_tok code^V[tok][c] * P'[tok][col] with
-//           mma.m16n8k16 (A = V codes transposed, two token rows interleaved
-//           by byte permutes; B = P' = p * nu split into hi + lo, moved from
+//           mma.m16n8k16 (A = V codes transposed: the pair-interleaved V
+//           rows give two tokens' codes of a channel per 32-bit word; B =
+//           P' = p * nu split into hi + lo, moved from
 //           the score accumulator layout into the B layout with movmatrix),
 //           then scaled by sigma^V of the block into fp32 accumulators.
 // The channel and token orders inside a fragment are permutations chosen so
@@ -253,32 +254,29 @@ struct KUnpack<3> {
 };
 
 // V side.  Thread g of a warp owns channels [16g, 16g + 16) of a token row.
-// For two token rows r0, r1 it produces the 16 fp16x2 values
-// (code[r0][c], code[r1][c]) for c = 16g + k, k = 0..15, in pr[k].
+// V rows are stored pair-interleaved (word u of the pair block of tokens 2k,
+// 2k + 1 holds unit u of both rows, see pairv_layout), so the registers the
+// value MMA wants, (code[2k][c], code[2k + 1][c]) for c = 16g + j, come
+// straight from the pair block pb: pr[j] for j = 0..15.
 template <int BITS>
 struct VUnpack;
 
 template <>
 struct VUnpack<4> {
     static constexpr bool kBiased = true;  // odd channels (high nibbles) as 16 (q + 72)
-    __device__ static void run(const uint8_t* r0, const uint8_t* r1, int g, uint32_t (&pr)[16]) {
-        const uint2 u0 = *reinterpret_cast<const uint2*>(r0 + 8 * g);
-        const uint2 u1 = *reinterpret_cast<const uint2*>(r1 + 8 * g);
+    // units 4g .. 4g + 3: the 16-byte chunk g, at g ^ (2 (k & 1))
+    __device__ static void run(const uint8_t* pb, int k, int g, uint32_t (&pr)[16]) {
+        const uint4 v = *reinterpret_cast<const uint4*>(pb + 16 * (g ^ pairv_chunk_xor<4>(k)));
+        const uint32_t x4[4] = {v.x, v.y, v.z, v.w};
         const uint32_t sub = h2c(1032.0f);
-        const uint32_t a[2] = {u0.x, u0.y}, b[2] = {u1.x, u1.y};
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                // bytes 2hh, 2hh+1 of both rows: channels 8i + 4hh .. + 3
-                const uint32_t x = prmt(a[i], b[i], hh ? 0x7632u : 0x5410u);
-                const uint32_t x8 = x >> 8;
-                const int k = 8 * i + 4 * hh;
-                pr[k + 0] = h2_sub(lop_and_or(x, 0x000F000Fu, kMagic), sub);
-                pr[k + 1] = lop_and_or(x, 0x00F000F0u, kMagic);
-                pr[k + 2] = h2_sub(lop_and_or(x8, 0x000F000Fu, kMagic), sub);
-                pr[k + 3] = lop_and_or(x8, 0x00F000F0u, kMagic);
-            }
+        for (int i = 0; i < 4; ++i) {
+            // unit 4g + i of both rows: channels 16g + 4i .. + 3
+            const uint32_t x = x4[i], x8 = x >> 8;
+            pr[4 * i + 0] = h2_sub(lop_and_or(x, 0x000F000Fu, kMagic), sub);
+            pr[4 * i + 1] = lop_and_or(x, 0x00F000F0u, kMagic);
+            pr[4 * i + 2] = h2_sub(lop_and_or(x8, 0x000F000Fu, kMagic), sub);
+            pr[4 * i + 3] = lop_and_or(x8, 0x00F000F0u, kMagic);
         }
     }
 };
@@ -286,12 +284,12 @@ struct VUnpack<4> {
 template <>
 struct VUnpack<2> {
     static constexpr bool kBiased = false;
-    __device__ static void run(const uint8_t* r0, const uint8_t* r1, int g, uint32_t (&pr)[16]) {
-        const uint32_t a = *reinterpret_cast<const uint32_t*>(r0 + 4 * g);
-        const uint32_t b = *reinterpret_cast<const uint32_t*>(r1 + 4 * g);
+    // units 2g, 2g + 1: words 2g, 2g + 1 of the pair block
+    __device__ static void run(const uint8_t* pb, int, int g, uint32_t (&pr)[16]) {
+        const uint2 v = *reinterpret_cast<const uint2*>(pb + 8 * g);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t x = prmt(a, b, hh ? 0x7632u : 0x5410u);  // channels 8hh .. 8hh + 7
+            const uint32_t x = hh ? v.y : v.x;  // channels 16g + 8hh .. + 7
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 pr[8 * hh + j] = dec2<2>(x, j);
@@ -304,15 +302,14 @@ struct VUnpack<2> {
 template <>
 struct VUnpack<3> {
     static constexpr bool kBiased = false;
-    __device__ static void run(const uint8_t* r0, const uint8_t* r1, int g, uint32_t (&pr)[16]) {
-        const uint32_t a = *reinterpret_cast<const uint32_t*>(r0 + 4 * g);
-        const uint32_t b = *reinterpret_cast<const uint32_t*>(r1 + 4 * g);
-        const uint32_t ha = *reinterpret_cast<const uint16_t*>(r0 + 32 + 2 * g);
-        const uint32_t hb = *reinterpret_cast<const uint16_t*>(r1 + 32 + 2 * g);
-        const uint32_t hh2 = ha | (hb << 16);  // bit k: row 0 channel k; bit 16 + k: row 1 channel k
+    // 2-bit plane: units 2g, 2g + 1 (words 2g, 2g + 1); bit plane: unit 16 + g
+    __device__ static void run(const uint8_t* pb, int, int g, uint32_t (&pr)[16]) {
+        const uint2 v = *reinterpret_cast<const uint2*>(pb + 8 * g);
+        // bit j: channel 16g + j of row 2k; bit 16 + j: of row 2k + 1
+        const uint32_t hh2 = *reinterpret_cast<const uint32_t*>(pb + 64 + 4 * g);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t x = prmt(a, b, hh ? 0x7632u : 0x5410u);
+            const uint32_t x = hh ? v.y : v.x;
             const uint32_t hsrc = hh ? (hh2 >> 8) : hh2;  // channel 8hh + j at bits j, 16 + j
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -380,11 +377,6 @@ __host__ __device__ constexpr int mma_smem_bytes() {
 __device__ __forceinline__ void mbar_inval(uint64_t* bar) {
     asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-
-// Token held by fragment row r (0..15) of a 16-token tile: rows 2k and 2k + 1
-// swap when k is odd.  Thread quads then read token rows of alternating
-// parity, which spreads the V-side loads over both halves of the banks.
-__device__ __forceinline__ int tile_tok(int r) { return r ^ ((r >> 1) & 1); }
 
 // Split of `work` blocks over nctas CTAs: the first r CTAs take q + 1 blocks,
 // the others q (q = work / nctas, r = work % nctas; work < 2^31).
@@ -518,8 +510,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
 
     const float alpha2 = a.scale * kLog2e;
     const bool blo = (g & 1) != 0;  // B column of this thread: head 4n + g/2, part g%2
-    const int tr0 = tile_tok(g), tr1 = 8 + tile_tok(g);
-    const int vr0 = tile_tok(2 * t), vr1 = tile_tok(2 * t + 1);
+    const int tr0 = g, tr1 = 8 + g;  // tokens of the score fragment rows (and of P' rows)
 
     int pos = 0;
     while (pos < nmine && ok) {
@@ -803,8 +794,10 @@ __global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
                     const uint32_t (&bp)[NT][2] = bpa[m4];
                     uint32_t va[16], vb[16];
                     const uint8_t* vbase = sv + SL::kCodes + (16 * m4) * SL::kRB;
-                    VUnpack<BITS>::run(vbase + vr0 * SL::kRB, vbase + vr1 * SL::kRB, g, va);
-                    VUnpack<BITS>::run(vbase + (8 + vr0) * SL::kRB, vbase + (8 + vr1) * SL::kRB, g, vb);
+                    // k-steps 2t, 2t + 1 of the value MMA: tokens 2t, 2t + 1 (pair t of
+                    // the tile) for va and 8 + 2t, 9 + 2t (pair 4 + t) for vb
+                    VUnpack<BITS>::run(vbase + t * 2 * SL::kRB, t, g, va);
+                    VUnpack<BITS>::run(vbase + (4 + t) * 2 * SL::kRB, t, g, vb);
                     if constexpr (VB) {
                         // every row of this product is the same: carry one
 #pragma unroll

@@ -383,6 +383,19 @@ struct QuantSmem {
     uint32_t* sgn2;  // [D/2] fp16x2 sign masks of channels (2i, 2i+1)
 };
 
+// V code rows of head dim 128 are stored pair-interleaved, the layout the
+// decode kernel's value operand wants (two tokens' codes of one channel in
+// one 32-bit register): the rows of tokens 2k and 2k + 1 of a block form a
+// pair block of 2 * row_bytes bytes whose 32-bit word u holds the 2-byte unit
+// u (bytes 2u, 2u + 1) of row 2k in its low half and of row 2k + 1 in its
+// high half.  For INT4 the 16-byte chunk c of pair block k sits at chunk
+// c ^ (2 (k & 1)), which spreads a quarter warp's 16-byte loads over the
+// banks; token 2k + s fills the s-th row_bytes half of its pair block.
+template <int D>
+__host__ __device__ constexpr bool pairv_layout() { return D == 128; }
+template <int BITS>
+__host__ __device__ constexpr int pairv_chunk_xor(int k) { return BITS == 4 ? 2 * (k & 1) : 0; }
+
 // Output pointers of one (tensor, batch, head, block).
 struct QuantOut {
     uint8_t* codes;  // [128][row_bytes] rows of this block
@@ -392,13 +405,50 @@ struct QuantOut {
     __half* tok;     // [128][ntok]
     __half* chan;    // [D] (PER_CHANNEL)
     __half* off;     // [D] (NSN)
+    bool pairv;      // V codes of head dim 128: pair-interleaved rows
 };
 
 // Row t of packed codes: straight to global memory, or into the swizzled
 // staging tile of a TMA store (then visible to the async proxy).
+// Words of token t's row_bytes half of its pair block (pair-interleaved V
+// rows), exchanged with the partner token t ^ 1 (same warp; every lane
+// calls this): token 2k + s takes units s W .. s W + W - 1 of both rows.
+template <int BITS, int W>
+__device__ __forceinline__ void pairv_words(int t, const uint32_t (&w)[W], uint32_t (&v)[W]) {
+    static_assert(W % 2 == 0, "even number of words per row");
+    const bool odd = (t & 1) != 0;
+#pragma unroll
+    for (int j = 0; j < W / 2; ++j) {
+        const uint32_t p = __shfl_xor_sync(0xffffffffu, odd ? w[j] : w[W / 2 + j], 1);
+        const uint32_t r0 = odd ? p : w[j];               // row 2k: units 2j, 2j + 1 of this half
+        const uint32_t r1 = odd ? w[W / 2 + j] : p;       // row 2k + 1
+        v[2 * j] = prmt32(r0, r1, 0x5410u);
+        v[2 * j + 1] = prmt32(r0, r1, 0x7632u);
+    }
+    if constexpr (BITS == 4) {
+        static_assert(W == 16, "INT4 rows of head dim 128: four 16-byte chunks per half");
+        // chunk c of the pair block at c ^ (2 (k & 1)): on odd pairs the
+        // chunks 0, 1 of this half trade places with 2, 3
+        if ((t >> 1) & 1) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t x = v[i];
+                v[i] = v[i + 8];
+                v[i + 8] = x;
+            }
+        }
+    }
+}
+
 template <int D, int BITS>
-__device__ __forceinline__ void store_codes(const QuantOut& out, int t, const uint32_t (&w)[RowLayout<D, BITS>::kWords]) {
+__device__ __forceinline__ void store_codes(const QuantOut& out, int t, const uint32_t (&w0)[RowLayout<D, BITS>::kWords]) {
     using L = RowLayout<D, BITS>;
+    uint32_t w[L::kWords];
+#pragma unroll
+    for (int i = 0; i < L::kWords; ++i) w[i] = w0[i];
+    if constexpr (pairv_layout<D>()) {
+        if (out.pairv) pairv_words<BITS, L::kWords>(t, w0, w);
+    }
     if constexpr (BITS == 4 || BITS == 2) {
         if (out.stage != nullptr) {
             constexpr int NC = L::kBytes / 16;  // 16-byte chunks per row

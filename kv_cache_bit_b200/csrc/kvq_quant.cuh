@@ -70,6 +70,7 @@ __device__ __forceinline__ QuantOut quant_out(const QuantArgs& a, int tensor, in
     o.chan = (MODE != kNaive) ? (v ? a.chan[1] : a.chan[0]) + ((size_t)bh * nb + blk) * D : nullptr;
     o.off = (MODE == kNsn) ? (v ? a.off[1] : a.off[0]) + ((size_t)bh * nb + blk) * D : nullptr;
     o.stage = nullptr;
+    o.pairv = pairv_layout<D>() && v;
     return o;
 }
 
@@ -260,6 +261,7 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
 
 struct DequantArgs {
     const uint8_t* codes;
+    int pairv;  // V codes of head dim 128: pair-interleaved rows
     const __half* tok;
     const __half* chan;
     const __half* off;
@@ -290,7 +292,24 @@ __global__ void __launch_bounds__(128) dequantize_kernel(DequantArgs a) {
     __syncthreads();
     const size_t tok_idx = (size_t)bh * a.cap + (size_t)blk * kT + t;
     uint32_t w32[L::kWords];
-    load_words<L::kWords>(a.codes + tok_idx * L::kBytes, w32);
+    if (pairv_layout<D>() && a.pairv) {
+        // unit u of row t: word u of pair block t / 2, half t & 1
+        const uint8_t* pb = a.codes + ((size_t)bh * a.cap + (size_t)blk * kT + (t & ~1)) * L::kBytes;
+        const int k = t >> 1;
+#pragma unroll
+        for (int j = 0; j < L::kWords; ++j) {
+            uint32_t h[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int u = 2 * j + e;
+                const int c = (u >> 2) ^ pairv_chunk_xor<BITS>(k);
+                h[e] = *reinterpret_cast<const uint16_t*>(pb + 16 * c + 4 * (u & 3) + 2 * (t & 1));
+            }
+            w32[j] = h[0] | (h[1] << 16);
+        }
+    } else {
+        load_words<L::kWords>(a.codes + tok_idx * L::kBytes, w32);
+    }
     const __half* tp = a.tok + tok_idx * ntk;
     float w[D];
     const float tsig = (MODE == kNaive) ? __half2float(tp[0]) : 0.0f;

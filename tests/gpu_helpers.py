@@ -8,6 +8,7 @@ import numpy as np
 import oracle
 from kv_cache_bit_b200 import synth
 from tests.modes import f16bits, oracle_cfg
+from tests.layout import pairv_applies, pairv_to_rows
 
 T = 128
 
@@ -79,6 +80,8 @@ def compare_cache(gcache, ck, cv, d, bits, nq, bh_slice=slice(None)):
     nb = nq // T
     for i, oc in enumerate((ck, cv)):
         g_codes = gcache.codes[i][bh_slice][:, :, :nq].cpu().numpy()
+        if i == 1 and pairv_applies(d):
+            g_codes = pairv_to_rows(g_codes, bits)  # the library's V layout -> token-major rows
         o_codes = oc["codes"][:, :, :nq]
         if not np.array_equal(g_codes, o_codes):
             gq, _ = oracle.unpack_rows(g_codes.reshape(-1, rb), d, bits)
