@@ -95,6 +95,13 @@ typedef struct {
  *   e[4j+2] << 4 | e[4j+3] << 6; INT3 = head_dim/4 bytes of (e & 3) in the
  *   INT2 layout followed by head_dim/8 bytes whose bit i of byte j is bit 2
  *   of e[8j+i].
+ * V codes of head_dim 128 are stored pair-interleaved (the layout the decode
+ *   kernel's value operand takes): the rows of tokens 2k and 2k+1 form a
+ *   pair block of 2*row_bytes bytes at the place of those two rows, whose
+ *   little-endian 32-bit word u holds bytes 2u, 2u+1 of row 2k in its low
+ *   half and of row 2k+1 in its high half; at INT4 the 16-byte chunk c of
+ *   pair block k is stored at chunk c ^ (2*(k & 1)).  K codes, and V codes
+ *   of head_dim 64, are plain token rows.
  * `len` is the number of tokens stored: tokens [0, 128*floor(len/128)) are in
  * the quantized blocks, the remaining len % 128 are residual slots
  * 0 .. len%128-1.  The library updates `len` on the host struct after a
