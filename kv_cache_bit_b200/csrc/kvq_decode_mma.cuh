@@ -158,7 +158,6 @@ constexpr float kBiasA = -1152.0f;
 
 template <>
 struct KUnpack<4> {
-    static constexpr int kSliceBytes = 16;
     static constexpr int kPairGroup = 4;  // pairs 4i + j: channels 8i + j and 8i + 4 + j
     static constexpr bool kBiased = true;
     __device__ static int ca(int p) { return 8 * (p >> 2) + (p & 3); }
@@ -191,7 +190,6 @@ template <>
 struct KUnpack<2> {
     static constexpr bool kBiased = false;
     static constexpr int kPairGroup = 8;  // pairs 8i + j: channels 16i + j and 16i + 8 + j
-    static constexpr int kSliceBytes = 8;
     __device__ static int ca(int p) { return 16 * (p >> 3) + (p & 7); }
     __device__ static int cb(int p) { return ca(p) + 8; }
     __device__ static void run(const uint8_t* row, int t, uint32_t (&pr)[16]) {
@@ -235,7 +233,6 @@ template <>
 struct KUnpack<3> {
     static constexpr bool kBiased = false;
     static constexpr int kPairGroup = 8;  // pairs 8i + j: channels 16i + j and 16i + 8 + j
-    static constexpr int kSliceBytes = 8;  // low 2-bit plane; plus 4 bytes of the high plane
     __device__ static int ca(int p) { return 16 * (p >> 3) + (p & 7); }
     __device__ static int cb(int p) { return ca(p) + 8; }
     __device__ static void run(const uint8_t* row, int t, uint32_t (&pr)[16]) {
@@ -420,7 +417,7 @@ __device__ __forceinline__ uint32_t split_h2(float x) {
 // [m (log2 units), l, pad, pad, acc[D] (original domain)] per head
 // (part_stride floats).
 template <int D, int BITS, int MODE, bool HAD, int GP>
-__global__ void __launch_bounds__(kNW * 32) decode_mma_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kNW * 32, (BITS == 3) ? 3 : 0) decode_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "tensor-core decode is built for head dim 128");
     using SL = SlotLayout<D, BITS, MODE>;
     using SM = MmaSmem<D, BITS, MODE, GP>;

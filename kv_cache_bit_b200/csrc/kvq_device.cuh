@@ -417,13 +417,15 @@ template <int BITS, int W>
 __device__ __forceinline__ void pairv_words(int t, const uint32_t (&w)[W], uint32_t (&v)[W]) {
     static_assert(W % 2 == 0, "even number of words per row");
     const bool odd = (t & 1) != 0;
+    // (row 2k unit, row 2k + 1 unit) from (own word, partner's word): the
+    // even thread holds row 2k, the odd one row 2k + 1
+    const uint32_t sel_lo = odd ? 0x1054u : 0x5410u, sel_hi = odd ? 0x3276u : 0x7632u;
 #pragma unroll
     for (int j = 0; j < W / 2; ++j) {
+        const uint32_t own = odd ? w[W / 2 + j] : w[j];  // units 2j, 2j + 1 of this half
         const uint32_t p = __shfl_xor_sync(0xffffffffu, odd ? w[j] : w[W / 2 + j], 1);
-        const uint32_t r0 = odd ? p : w[j];               // row 2k: units 2j, 2j + 1 of this half
-        const uint32_t r1 = odd ? w[W / 2 + j] : p;       // row 2k + 1
-        v[2 * j] = prmt32(r0, r1, 0x5410u);
-        v[2 * j + 1] = prmt32(r0, r1, 0x7632u);
+        v[2 * j] = prmt32(own, p, sel_lo);
+        v[2 * j + 1] = prmt32(own, p, sel_hi);
     }
     if constexpr (BITS == 4) {
         static_assert(W == 16, "INT4 rows of head dim 128: four 16-byte chunks per half");
