@@ -28,7 +28,7 @@
  *  [P4] "Activation-guided compensation and orthogonal residuals" abstract:
  *       randomized Hadamard rotation with random sign patterns.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *  - block = 128 tokens; pchan scale = max over the block's tokens, per channel;
  *  - sums (norms, NSN means) are fp32 pairwise (recursive halving) sums;
  *  - codes = round-half-even of the exact product u * (1/sigma16), clamped;
