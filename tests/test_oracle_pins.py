@@ -7,6 +7,11 @@ fp64, published known-answer values, hand-worked layouts, or an invariant the
 pages state.  A plausible slip in the oracle (a dropped term, a wrong sign or
 index, a transposed operand, the L_{-1} "norm" the nsep+pchan post warns
 about) fails at least one of them.
+
+Page tags: [P1] the "KV cache INT4 quantization ... nsep+pchan" post,
+section "Fix (nsep+pchan)"; [P2] the "Rotated Runtime Smooth" analysis,
+master equation and symbol list; [P3] the "NSNQuant" explainer, section
+"Method: 1. Normalize-Shift-Normalize".
 """
 import math
 import os
