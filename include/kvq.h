@@ -169,8 +169,8 @@ kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache,
 
 /* Workspace bytes kvq_decode_attention needs for this cache and q_heads
    (partial softmax states of the sequence splits); 0 on invalid arguments.
-   The workspace must be zero-filled once when it is allocated: the decode
-   call leaves its counters at zero again when it completes. */
+   Each call writes every partial state it reads, so the workspace needs no
+   initialization. */
 size_t kvq_decode_workspace_bytes(const kvq_config* cfg, const kvq_cache* cache, int32_t q_heads);
 
 /*
@@ -185,8 +185,8 @@ size_t kvq_decode_workspace_bytes(const kvq_config* cfg, const kvq_cache* cache,
  *         q_heads / kv_heads <= 8
  *   scale softmax scale; <= 0 selects 1/sqrt(head_dim)
  *   out   fp32 [B][q_heads][head_dim]; len == 0 gives zeros
- *   ws    workspace of at least kvq_decode_workspace_bytes(), zero-filled
- *         when first allocated; calls that share a workspace must not
+ *   ws    workspace of at least kvq_decode_workspace_bytes() (contents
+ *         need no initialization); calls that share a workspace must not
  *         overlap in time
  * Errors: INVALID_ARG; WORKSPACE; UNSUPPORTED; CUDA.
  */
