@@ -91,6 +91,9 @@ DECODE_CASES = [
     ("nsn", 128, 4, 1, 2, 4, 256, 0),
     ("nsep+pchan", 128, 2, 1, 2, 16, 256, 0),     # g = 8
     ("nsep+pchan", 64, 3, 1, 2, 2, 128, 1),
+    # rotation with one and two query heads per kv head (idle fragment columns)
+    ("rht+nsep+pchan", 128, 4, 2, 2, 2, 256, 7),
+    ("nsn+hadamard", 128, 2, 1, 2, 4, 256, 0),
     # rotation with two n-tiles of query heads (G = 6 and 8)
     ("rht+nsep+pchan", 128, 4, 1, 2, 12, 384, 9),
     ("nsn+hadamard", 128, 4, 1, 1, 8, 256, 3),
