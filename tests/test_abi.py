@@ -123,6 +123,10 @@ def test_host_side_rejections(kvq):
     assert L.kvq_decode_attention(by(cfg), by(cache), A, 8, 0.0, A, None, need, None) == WS
     assert L.kvq_decode_attention(by(cfg), by(cache), A, 3, 0.0, A, A, need, None) == INV
     assert L.kvq_decode_attention(by(cfg), by(cache), A, 18, 0.0, A, A, 1 << 30, None) == UNS
+    # device pointers must be 16-byte aligned: query, output, workspace
+    assert L.kvq_decode_attention(by(cfg), by(cache), A + 8, 8, 0.0, A, A, need, None) == INV
+    assert L.kvq_decode_attention(by(cfg), by(cache), A, 8, 0.0, A + 4, A, need, None) == INV
+    assert L.kvq_decode_attention(by(cfg), by(cache), A, 8, 0.0, A, A + 4, need, None) == WS
     # dequantize ranges
     c300 = _fake_cache(kvq, length=200)
     assert L.kvq_dequantize(by(cfg), by(c300), 2, 0, 128, A, None) == INV
