@@ -152,8 +152,9 @@ struct KUnpack;
 // subtraction gives q = e - 8.  A high nibble (bits 4..7 of its byte) OR-ed
 // into 1024 reads 1024 + 16 e = 16 (q + 72) and is used in that biased form,
 // one LOP3 per pair with no fp16 arithmetic (kBiased): the kernel scales the
-// other operand of those channels by 1/16 and removes the bias with one MMA
-// against a constant A of -1152 = -16 * 72.
+// other operand of those channels by 1/16 and removes the bias 1152 = 16 * 72
+// times the sum of that operand: for the scores with one MMA against a
+// constant A of -1152 per block, for the values from the unit's sum of P'.
 constexpr float kBiasA = -1152.0f;
 
 template <>
@@ -416,8 +417,12 @@ __device__ __forceinline__ uint32_t split_h2(float x) {
 // Partial state of a (warp, pair) segment goes to slot part_slot() of a.part:
 // [m (log2 units), l, pad, pad, acc[D] (original domain)] per head
 // (part_stride floats).
+// The NSN and INT3 instantiations with one n-tile of query heads are held to
+// three resident CTAs per SM (168 registers), where the register allocator
+// otherwise spills or settles for fewer CTAs; the others are left to it.
 template <int D, int BITS, int MODE, bool HAD, int GP>
-__global__ void __launch_bounds__(kNW * 32, (BITS == 3) ? 3 : 0) decode_mma_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP == 4) ? 3 : 0)
+    decode_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "tensor-core decode is built for head dim 128");
     using SL = SlotLayout<D, BITS, MODE>;
     using SM = MmaSmem<D, BITS, MODE, GP>;
@@ -759,10 +764,10 @@ __global__ void __launch_bounds__(kNW * 32, (BITS == 3) ? 3 : 0) decode_mma_kern
                 }
                 // ---- P' = p * nu (scaled) and the values, tile by tile
                 float dv[NT][8][4];  // set by the first tile's MMAs
-                float vbias[NT][2];  // -1152 * sum of the unit's P' (hi, lo columns)
+                float psum[NT];  // this thread's rows of the unit's sum of P' (biased V codes)
                 float lsum[NT], bsum[NT];
 #pragma unroll
-                for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; }
+                for (int n = 0; n < NT; ++n) { lsum[n] = 0.0f; bsum[n] = 0.0f; psum[n] = 0.0f; }
                 uint32_t bpa[4][NT][2];
 #pragma unroll
                 for (int m4 = 0; m4 < 4; ++m4) {
@@ -782,7 +787,9 @@ __global__ void __launch_bounds__(kNW * 32, (BITS == 3) ? 3 : 0) decode_mma_kern
                             const float p = fast_exp2(l2[m4][n][r] - m_ref[n]);
                             lsum[n] += p;
                             if constexpr (MODE == kNsn) bsum[n] += p * s1o;
-                            bpa[m4][n][r] = movmatrix_t(split_h2(p * nu));
+                            const float x_ = p * nu;
+                            if constexpr (VB) psum[n] += x_;
+                            bpa[m4][n][r] = movmatrix_t(split_h2(x_));
                         }
                     }
                 }
@@ -795,20 +802,6 @@ __global__ void __launch_bounds__(kNW * 32, (BITS == 3) ? 3 : 0) decode_mma_kern
                     // the tile) for va and 8 + 2t, 9 + 2t (pair 4 + t) for vb
                     VUnpack<BITS>::run(vbase + t * 2 * SL::kRB, t, g, va);
                     VUnpack<BITS>::run(vbase + (4 + t) * 2 * SL::kRB, t, g, vb);
-                    if constexpr (VB) {
-                        // every row of this product is the same: carry one
-#pragma unroll
-                        for (int n = 0; n < NT; ++n) {
-                            float r4[4];
-                            if (m4 == 0)
-                                mma16816_z(r4, kBiasH2, kBiasH2, kBiasH2, kBiasH2, bp[n][0], bp[n][1]);
-                            else
-                                mma16816_c(r4, kBiasH2, kBiasH2, kBiasH2, kBiasH2, bp[n][0], bp[n][1], vbias[n][0],
-                                           vbias[n][1]);
-                            vbias[n][0] = r4[0];
-                            vbias[n][1] = r4[1];
-                        }
-                    }
 #pragma unroll
                     for (int tc = 0; tc < 8; ++tc) {
 #pragma unroll
@@ -829,7 +822,13 @@ __global__ void __launch_bounds__(kNW * 32, (BITS == 3) ? 3 : 0) decode_mma_kern
                 // removed and 1/16 goes into their scale
                 float vbs[NT];
 #pragma unroll
-                for (int n = 0; n < NT; ++n) vbs[n] = VB ? vbias[n][0] + vbias[n][1] : 0.0f;
+                for (int n = 0; n < NT; ++n) {
+                    if constexpr (VB) {
+#pragma unroll
+                        for (int o = 4; o < 32; o <<= 1) psum[n] += __shfl_xor_sync(0xffffffffu, psum[n], o);
+                    }
+                    vbs[n] = VB ? kBiasA * psum[n] : 0.0f;
+                }
                 const float pinv_v = VB ? pinv * 0.0625f : pinv;
 #pragma unroll
                 for (int tc = 0; tc < 8; ++tc) {
