@@ -31,8 +31,12 @@
  *  - Every argument is checked on the host before anything is enqueued; a
  *    failed check returns an error and changes no state.  Errors reported by
  *    the CUDA runtime at launch are returned as KVQ_ERR_CUDA.
- *  - The library holds no global state; calls on distinct caches may be made
- *    from several host threads.
+ *  - The library's global state is small and per device: a sticky device
+ *    error word (kvq_read_device_errors), per-device flags recording which
+ *    kernel attributes have been set, and the fixed scratch array of
+ *    kvq_decode_attention_noalloc.  Calls on distinct caches may be made from
+ *    several host threads; kvq_decode_attention_noalloc calls that overlap on
+ *    the GPU race on the shared scratch (see there).
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -143,8 +147,10 @@ kvq_status kvq_make_signs(uint64_t seed, int32_t head_dim, int8_t* host_out);
  * tokens, qmax = 2^(N-1)-1).
  *   k, v   fp16 [B][H][ntok][head_dim], contiguous
  *   t0     multiple of 128; ntok > 0 and a multiple of 128
- * Per (b, h, block, tensor) one CTA reads the 128 x head_dim tile once and
- * writes codes, per-token parameters and per-block channel scales/means.
+ * A persistent grid (a few CTAs per SM) takes the (b, h, block, tensor)
+ * tiles in turn; each tile of 128 x head_dim fp16 values is read from HBM
+ * once and its codes, per-token parameters and per-block channel
+ * scales/means are written once.
  * On success len = max(len, t0 + ntok).
  * Errors: INVALID_ARG (null/misaligned pointers, t0 or ntok not multiples of
  * 128, or a range that overlaps residual tokens that are still held, i.e.
@@ -233,9 +239,9 @@ kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache* 
 /*
  * Read (and, if clear != 0, reset) the sticky device error word of the
  * current device: bit 0 = a kernel gave up waiting for a TMA tile, bit 1 = a
- * kernel gave up waiting on a barrier.  Kernels that give up write no
- * results.  This word is the library's only device-global state.  HOST call;
- * synchronizes the device.  Errors: INVALID_ARG (host_out NULL); CUDA.
+ * kernel gave up waiting on a barrier.  Kernels that give up leave the
+ * results of that call undefined.  HOST call; synchronizes the device.
+ * Errors: INVALID_ARG (host_out NULL); CUDA.
  */
 kvq_status kvq_read_device_errors(uint32_t* host_out, int32_t clear);
 

@@ -58,6 +58,7 @@ def lib():
         L.ko_quantize_block.argtypes = [_P, _P, _P, _P, _P, _P]
         L.ko_dequantize_block.argtypes = [_P, _P, _P, _P, _P, _P]
         L.ko_quantize_slice.argtypes = [_P, _P, ctypes.c_long, ctypes.c_long, _P, _P, _P, _P]
+        L.ko_quantize_slice_y.argtypes = [_P, _P, ctypes.c_long, ctypes.c_long, _P, _P, _P, _P, _P]
         L.ko_dequantize_slice.argtypes = [_P, _P, _P, _P, _P, ctypes.c_long, ctypes.c_long, _P]
         L.ko_attention_f64.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_long, _P, _P, _P,
                                        ctypes.c_double, _P]
@@ -206,6 +207,38 @@ def quantize_into(cfg: Cfg, x16: np.ndarray, cache: dict, t0: int = 0, threads: 
     with _pool(threads) as ex:
         list(ex.map(one, [(b, h) for b in range(B) for h in range(H)]))
     return cache
+
+
+def quantize_products(cfg: Cfg, x16: np.ndarray, cache: dict, t0: int = 0, threads: int = 1) -> np.ndarray:
+    """Quantize like quantize_into and return the exact pre-rounding
+    product u * (1/sigma16) of every code, float64 [B, H, n, d]: each code is
+    clamp(round-half-even(y)).  Used to tell a rounding half-point from a
+    real disagreement."""
+    x16 = np.ascontiguousarray(x16, dtype=np.uint16)
+    B, H, n, d = x16.shape
+    assert d == cfg.d and n % T == 0 and t0 % T == 0
+    y = np.empty((B, H, n, d), np.float64)
+    c = cfg.c()
+    L = lib()
+
+    def one(bh):
+        b, h = bh
+        L.ko_quantize_slice_y(ctypes.byref(c), _ptr(x16[b, h]), t0, n,
+                              _ptr(cache["codes"][b, h]),
+                              None if cache["tok"] is None else _ptr(cache["tok"][b, h]),
+                              None if cache["chan"] is None else _ptr(cache["chan"][b, h]),
+                              None if cache["off"] is None else _ptr(cache["off"][b, h]),
+                              _ptr(y[b, h]))
+
+    with _pool(threads) as ex:
+        list(ex.map(one, [(b, h) for b in range(B) for h in range(H)]))
+    return y
+
+
+def half_point_distance(y: np.ndarray) -> np.ndarray:
+    """Distance of |y| from the nearest rounding half-point k + 1/2."""
+    a = np.abs(np.asarray(y, np.float64))
+    return np.abs(a - np.floor(a) - 0.5)
 
 
 def quantize(cfg: Cfg, x16: np.ndarray, S_max: Optional[int] = None, threads: int = 1) -> dict:

@@ -216,8 +216,11 @@ static int ko_code(float u, float inv, int qmax)
 /*   chan  [d] fp16 bits per-channel scale (PER_CHANNEL)               */
 /*   off   [d] fp16 bits per-channel mean (NSN)                        */
 /* ------------------------------------------------------------------ */
-void ko_quantize_block(const ko_cfg* cfg, const uint16_t* x, uint8_t* codes,
-                       uint16_t* tok, uint16_t* chan, uint16_t* off)
+/* y (optional, [T][d] doubles): the exact product u * inv that each code
+   rounds; it exposes the value the codes are taken from and changes nothing
+   else. */
+static void ko_quantize_block_impl(const ko_cfg* cfg, const uint16_t* x, uint8_t* codes,
+                                   uint16_t* tok, uint16_t* chan, uint16_t* off, double* y)
 {
     const int d = cfg->d, T = KO_T, qmax = ko_qmax(cfg->bits);
     const unsigned fl = cfg->flags;
@@ -286,7 +289,10 @@ void ko_quantize_block(const ko_cfg* cfg, const uint16_t* x, uint8_t* codes,
             chan[c] = ko_f32_to_f16(m / (float)qmax);
             float sf = ko_f16_to_f32(chan[c]);
             float inv = sf > 0.0f ? 1.0f / sf : 0.0f;
-            for (int t = 0; t < T; t++) q[t * d + c] = (int8_t)ko_code(w[t * d + c], inv, qmax);
+            for (int t = 0; t < T; t++) {
+                q[t * d + c] = (int8_t)ko_code(w[t * d + c], inv, qmax);
+                if (y) y[t * d + c] = (double)w[t * d + c] * (double)inv;
+            }
         }
     } else {
         for (int t = 0; t < T; t++) {
@@ -296,13 +302,22 @@ void ko_quantize_block(const ko_cfg* cfg, const uint16_t* x, uint8_t* codes,
             tok[t * ntok + ntok - 1] = s16;
             float sf = ko_f16_to_f32(s16);
             float inv = sf > 0.0f ? 1.0f / sf : 0.0f;
-            for (int c = 0; c < d; c++) q[t * d + c] = (int8_t)ko_code(w[t * d + c], inv, qmax);
+            for (int c = 0; c < d; c++) {
+                q[t * d + c] = (int8_t)ko_code(w[t * d + c], inv, qmax);
+                if (y) y[t * d + c] = (double)w[t * d + c] * (double)inv;
+            }
         }
     }
 
     const int rb = ko_row_bytes(d, cfg->bits);
     for (int t = 0; t < T; t++) ko_pack_row(q + t * d, d, cfg->bits, codes + (size_t)t * rb);
     free(w); free(ks); free(q);
+}
+
+void ko_quantize_block(const ko_cfg* cfg, const uint16_t* x, uint8_t* codes,
+                       uint16_t* tok, uint16_t* chan, uint16_t* off)
+{
+    ko_quantize_block_impl(cfg, x, codes, tok, chan, off, NULL);
 }
 
 /* ------------------------------------------------------------------ */
@@ -365,17 +380,26 @@ int ko_dequantize_block(const ko_cfg* cfg, const uint8_t* codes, const uint16_t*
 /* Layouts per slice: x [ntok][d]; codes [S_max][row_bytes];           */
 /* tok [S_max][ntok]; chan, off [S_max/T][d].                          */
 /* ------------------------------------------------------------------ */
-void ko_quantize_slice(const ko_cfg* cfg, const uint16_t* x, long t0, long ntok,
-                       uint8_t* codes, uint16_t* tok, uint16_t* chan, uint16_t* off)
+/* y: NULL, or [ntok][d] doubles that receive the exact pre-rounding
+   product of every code (see ko_quantize_block_impl). */
+void ko_quantize_slice_y(const ko_cfg* cfg, const uint16_t* x, long t0, long ntok,
+                         uint8_t* codes, uint16_t* tok, uint16_t* chan, uint16_t* off, double* y)
 {
     const int d = cfg->d, rb = ko_row_bytes(d, cfg->bits), nt = ko_ntok(cfg->flags);
     for (long t = 0; t < ntok; t += KO_T) {
         long tb = t0 + t, blk = tb / KO_T;
-        ko_quantize_block(cfg, x + (size_t)t * d, codes + (size_t)tb * rb,
-                          tok ? tok + (size_t)tb * nt : NULL,
-                          chan ? chan + (size_t)blk * d : NULL,
-                          off ? off + (size_t)blk * d : NULL);
+        ko_quantize_block_impl(cfg, x + (size_t)t * d, codes + (size_t)tb * rb,
+                               tok ? tok + (size_t)tb * nt : NULL,
+                               chan ? chan + (size_t)blk * d : NULL,
+                               off ? off + (size_t)blk * d : NULL,
+                               y ? y + (size_t)t * d : NULL);
     }
+}
+
+void ko_quantize_slice(const ko_cfg* cfg, const uint16_t* x, long t0, long ntok,
+                       uint8_t* codes, uint16_t* tok, uint16_t* chan, uint16_t* off)
+{
+    ko_quantize_slice_y(cfg, x, t0, ntok, codes, tok, chan, off, NULL);
 }
 
 int ko_dequantize_slice(const ko_cfg* cfg, const uint8_t* codes, const uint16_t* tok,

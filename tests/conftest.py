@@ -25,3 +25,18 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Report the rounding half-point cases met by the GPU parity tests."""
+    try:
+        from tests.gpu_helpers import HALF_POINT_LOG
+    except Exception:
+        return
+    if not HALF_POINT_LOG:
+        return
+    n = sum(h for h, _ in HALF_POINT_LOG)
+    codes = sum(c for _, c in HALF_POINT_LOG)
+    terminalreporter.write_line(
+        f"GPU parity: {codes} codes compared with the oracle in {len(HALF_POINT_LOG)} comparisons; "
+        f"{n} differed, each at a rounding half-point (within 1e-6)")

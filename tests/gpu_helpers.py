@@ -50,14 +50,18 @@ def gpu_prefill(mode, d, bits, K, V, cap=None, ntok=None):
 
 
 def oracle_prefill(mode, d, bits, K, V, cap=None, ntok=None, threads=8):
+    """The oracle's caches of K and V.  Each cache dict also carries "y":
+    the exact pre-rounding product of every code of the quantized tokens
+    (float64 [B, H, ntok, d]), which tells a rounding half-point apart."""
     B, H, S, _ = K.shape
     ntok = S if ntok is None else ntok
     cfg = oracle_cfg(mode, d, bits)
     ck = oracle.empty_cache(cfg, B, H, cap or S)
     cv = oracle.empty_cache(cfg, B, H, cap or S)
+    ck["y"] = cv["y"] = None
     if ntok:
-        oracle.quantize_into(cfg, f16bits(K[:, :, :ntok]), ck, 0, threads)
-        oracle.quantize_into(cfg, f16bits(V[:, :, :ntok]), cv, 0, threads)
+        ck["y"] = oracle.quantize_products(cfg, f16bits(K[:, :, :ntok]), ck, 0, threads)
+        cv["y"] = oracle.quantize_products(cfg, f16bits(V[:, :, :ntok]), cv, 0, threads)
     return cfg, ck, cv
 
 
@@ -71,39 +75,62 @@ def fp16_ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> int:
     return int(np.max(np.abs(key(a_bits) - key(b_bits))))
 
 
-def compare_cache(gcache, ck, cv, d, bits, nq, bh_slice=slice(None)):
-    """Codes bit-exact, side parameters within 1 fp16 ulp.  Returns a dict of
-    mismatch counts (codes that differ must be neighbours; each one counts as
-    a half-point case)."""
+# A code may differ from the oracle's only where the exact product it rounds
+# lies within this distance of a rounding half-point.
+HALF_POINT_TOL = 1e-6
+
+# Half-point cases met by the GPU parity tests of this session, reported in
+# the pytest terminal summary (tests/conftest.py).
+HALF_POINT_LOG = []
+
+
+def compare_cache(gcache, ck, cv, d, bits, nq, bh_slice=slice(None), t0=0):
+    """Codes bit-exact except at rounding half-points, side parameters within
+    1 fp16 ulp.  ck / cv are oracle caches whose "y" holds the exact products
+    of the oracle's codes for tokens [t0, nq).  A code that differs from the
+    oracle's must be a neighbour whose product lies within HALF_POINT_TOL of
+    a half-point; such codes are counted ("half_points") and logged.
+    Returns a dict of counts and largest parameter differences in ulps."""
     rb = oracle.row_bytes(d, bits)
-    res = {"code_mismatch": 0, "tok_ulp": 0, "chan_ulp": 0, "off_ulp": 0, "codes": 0}
+    res = {"code_mismatch": 0, "half_points": 0, "tok_ulp": 0, "chan_ulp": 0, "off_ulp": 0, "codes": 0}
     nb = nq // T
     for i, oc in enumerate((ck, cv)):
-        g_codes = gcache.codes[i][bh_slice][:, :, :nq].cpu().numpy()
+        g_codes = gcache.codes[i][bh_slice][:, :, t0:nq].cpu().numpy()
         if i == 1 and pairv_applies(d):
             g_codes = pairv_to_rows(g_codes, bits)  # the library's V layout -> token-major rows
-        o_codes = oc["codes"][:, :, :nq]
+        o_codes = oc["codes"][:, :, t0:nq]
         if not np.array_equal(g_codes, o_codes):
             gq, _ = oracle.unpack_rows(g_codes.reshape(-1, rb), d, bits)
             oq, _ = oracle.unpack_rows(o_codes.reshape(-1, rb), d, bits)
             diff = gq.astype(int) - oq.astype(int)
             assert np.abs(diff).max() <= 1, "codes differ by more than one step"
-            res["code_mismatch"] += int(np.count_nonzero(diff))
+            y = oc.get("y")
+            assert y is not None, "codes differ and the oracle's products were not kept"
+            y = y[:, :, t0:nq].reshape(diff.shape)
+            bad = (diff != 0) & (oracle.half_point_distance(y) > HALF_POINT_TOL)
+            assert not bad.any(), f"{int(bad.sum())} code(s) differ away from a rounding half-point"
+            n = int(np.count_nonzero(diff))
+            res["code_mismatch"] += n
+            res["half_points"] += n
         res["codes"] += o_codes.size * 8 // bits
-        res["tok_ulp"] = max(res["tok_ulp"], fp16_ulp_diff(host16(gcache.tok[i][bh_slice][:, :, :nq]),
-                                                           oc["tok"][:, :, :nq]))
+        res["tok_ulp"] = max(res["tok_ulp"], fp16_ulp_diff(host16(gcache.tok[i][bh_slice][:, :, t0:nq]),
+                                                           oc["tok"][:, :, t0:nq]))
+        b0 = t0 // T
         if oc["chan"] is not None:
-            res["chan_ulp"] = max(res["chan_ulp"], fp16_ulp_diff(host16(gcache.chan[i][bh_slice][:, :, :nb]),
-                                                                 oc["chan"][:, :, :nb]))
+            res["chan_ulp"] = max(res["chan_ulp"], fp16_ulp_diff(host16(gcache.chan[i][bh_slice][:, :, b0:nb]),
+                                                                 oc["chan"][:, :, b0:nb]))
         if oc["off"] is not None:
-            res["off_ulp"] = max(res["off_ulp"], fp16_ulp_diff(host16(gcache.off[i][bh_slice][:, :, :nb]),
-                                                               oc["off"][:, :, :nb]))
+            res["off_ulp"] = max(res["off_ulp"], fp16_ulp_diff(host16(gcache.off[i][bh_slice][:, :, b0:nb]),
+                                                               oc["off"][:, :, b0:nb]))
+    HALF_POINT_LOG.append((res["half_points"], res["codes"]))
     return res
 
 
-def assert_cache_parity(res, max_half_point_frac=1e-5):
+def assert_cache_parity(res):
+    """fp16 side parameters within 1 ulp; every code difference was already
+    proven a half-point case by compare_cache."""
     assert res["tok_ulp"] <= 1 and res["chan_ulp"] <= 1 and res["off_ulp"] <= 1, res
-    assert res["code_mismatch"] <= max(1, int(max_half_point_frac * res["codes"])), res
+    assert res["code_mismatch"] == res["half_points"], res
 
 
 def gpu_decode(cfg, cache, q16: np.ndarray, scale: float = 0.0):
