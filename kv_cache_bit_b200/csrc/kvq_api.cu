@@ -207,7 +207,7 @@ struct QuantLaunch {
             if (!make_code_map(&mck, a.codes[0], crow, rb) || !make_code_map(&mcv, a.codes[1], crow, rb))
                 return KVQ_ERR_CUDA;
         }
-        constexpr int smem = quant_smem_bytes<D>();
+        constexpr int smem = quant_smem_bytes<D, MODE>();
         auto kern = quantize_kernel<D, BITS, MODE, HAD>;
         if (!ensure_smem<quantize_kernel<D, BITS, MODE, HAD>>(smem)) return KVQ_ERR_CUDA;
         int dev = 0, sms = 0, occ = 0;
@@ -231,7 +231,7 @@ struct AppendLaunch {
     cudaStream_t st;
     template <int D, int BITS, int MODE, bool HAD>
     kvq_status run() {
-        constexpr int smem = quant_smem_bytes<D>();
+        constexpr int smem = quant_smem_bytes<D, MODE>();
         if (!ensure_smem<append_kernel<D, BITS, MODE, HAD>>(smem)) return KVQ_ERR_CUDA;
         append_kernel<D, BITS, MODE, HAD><<<dim3(bh, 2), kT, a.slot == kT - 1 ? smem : 0, st>>>(a);
         return launch_status();

@@ -261,6 +261,20 @@ __device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
     return r;
 }
 
+// Lane-wise product rounded to fp32 on its own, as two scalar mul.rn.f32:
+// the assembler keeps an explicitly rounded scalar multiply separate, while
+// it may fuse a packed mul.rn.f32x2 with the add or subtract that consumes
+// it into one fused multiply-add (one rounding instead of two).  Every
+// product that feeds an add whose operands are not exact products uses this.
+__device__ __forceinline__ f2_t f2_mul_sep(f2_t a, f2_t b) {
+    f2_t r;
+    asm("{\n .reg .f32 a0, a1, b0, b1, r0, r1;\n mov.b64 {a0, a1}, %1;\n mov.b64 {b0, b1}, %2;\n"
+        " mul.rn.f32 r0, a0, b0;\n mul.rn.f32 r1, a1, b1;\n mov.b64 %0, {r0, r1};\n}"
+        : "=l"(r)
+        : "l"(a), "l"(b));
+    return r;
+}
+
 // Pairwise sum of squares over the pairs P[OFF .. OFF+N): lane 0 sums the
 // first half of the row, lane 1 the second, with the same recursive halving.
 // The volatile forms keep the depth-first order of the tree, so that the
@@ -275,18 +289,57 @@ __device__ __forceinline__ f2_t f2_add_ordered(f2_t a, f2_t b) {
     asm volatile("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
-template <int OFF, int N, int H2>
+// EXACT: the squares are exact in fp32 (values widened from fp16), so a
+// fused square-and-add rounds like the separate operations and the packed
+// multiply may be used; otherwise the squares are rounded on their own.
+template <int OFF, int N, int H2, bool EXACT>
 __device__ __forceinline__ f2_t pw_sumsq2(const f2_t (&P)[H2]) {
-    if constexpr (N == 1) return f2_mul_ordered(P[OFF], P[OFF]);
-    else return f2_add_ordered(pw_sumsq2<OFF, N / 2>(P), pw_sumsq2<OFF + N / 2, N / 2>(P));
+    if constexpr (N == 1) return EXACT ? f2_mul_ordered(P[OFF], P[OFF]) : f2_mul_sep(P[OFF], P[OFF]);
+    else return f2_add_ordered(pw_sumsq2<OFF, N / 2, H2, EXACT>(P), pw_sumsq2<OFF + N / 2, N / 2, H2, EXACT>(P));
 }
 
 // Pairwise sum of squares of the whole row: the top split of the halving
 // tree adds the two lanes.
-template <int H2>
+template <int H2, bool EXACT>
 __device__ __forceinline__ float row_sumsq(const f2_t (&P)[H2]) {
     float lo, hi;
-    f2_unpack(pw_sumsq2<0, H2>(P), lo, hi);
+    f2_unpack(pw_sumsq2<0, H2, H2, EXACT>(P), lo, hi);
+    return __fadd_rn(lo, hi);
+}
+
+// x_lo^2 + x_hi^2 of the two fp16 values of a word, rounded once to fp32:
+// the square of an fp16 value is exact in fp32, so two mixed-precision fused
+// multiply-adds (fp16 factors, fp32 addend) give exactly the fp32 sum of the
+// two exact squares.
+__device__ __forceinline__ float sumsq_h2(uint32_t w) {
+    float r;
+    asm volatile(
+        "{\n .reg .b16 l, h;\n .reg .f32 s;\n mov.b32 {l, h}, %1;\n"
+        " fma.rn.f32.f16 s, l, l, 0f00000000;\n fma.rn.f32.f16 %0, h, h, s;\n}"
+        : "=f"(r)
+        : "r"(w));
+    return r;
+}
+
+// The pairwise sum of squares of pw_sumsq2 taken straight from the raw fp16
+// row (chunk q = channels 8q .. 8q + 7): node OFF of the level above the
+// squares sums channels 2 OFF, 2 OFF + 1 of the low half (lane 0) and of the
+// high half (lane 1).
+template <int OFF, int N, int D>
+__device__ __forceinline__ f2_t raw_pw_sumsq(const uint4 (&raw)[D / 8]) {
+    if constexpr (N == 1) {
+        const uint32_t* lo = reinterpret_cast<const uint32_t*>(&raw[OFF / 4]);
+        const uint32_t* hi = reinterpret_cast<const uint32_t*>(&raw[D / 16 + OFF / 4]);
+        return f2_pack(sumsq_h2(lo[OFF % 4]), sumsq_h2(hi[OFF % 4]));
+    } else {
+        return f2_add_ordered(raw_pw_sumsq<OFF, N / 2, D>(raw), raw_pw_sumsq<OFF + N / 2, N / 2, D>(raw));
+    }
+}
+
+template <int D>
+__device__ __forceinline__ float raw_row_sumsq(const uint4 (&raw)[D / 8]) {
+    float lo, hi;
+    f2_unpack(raw_pw_sumsq<0, D / 4, D>(raw), lo, hi);
     return __fadd_rn(lo, hi);
 }
 
@@ -372,16 +425,45 @@ struct QuantSmem {
     // fp16 input tile: 64-channel boxes of 128 rows x 128 bytes, 16-byte
     // chunk c of row t stored at chunk c ^ (t & 7) (the TMA 128-byte swizzle)
     const uint8_t* tile;
-    // fp32 [128][D] transpose buffer in pair order, in two halves: pairs
-    // [0, D/4) of every row in red_lo, pairs [D/4, D/2) in red_hi; 16-byte
-    // chunk k of a half row t stored at chunk k ^ (t & (D/8 - 1))
+    // NSN: fp32 [128][D] buffer of the rows in pair order, in two halves:
+    // pairs [0, D/4) of every row in red_lo, pairs [D/4, D/2) in red_hi;
+    // 16-byte chunk k of a half row t stored at chunk k ^ (t & (D/8 - 1))
     float* red_lo;
     float* red_hi;
     float* vec;      // [D] a per-channel vector in pair order (means, reciprocal scales)
-    float* gpart;    // [4 KB] per-token-group partial sums / maxima
+    float* gpart;    // [4 KB] per-token-group partial sums (NSN means), then per-warp maxima
     float* tokv;     // [128] a per-token scalar (NSN 1/||x|| * sqrt(d))
     uint32_t* sgn2;  // [D/2] fp16x2 sign masks of channels (2i, 2i+1)
 };
+
+// Widen 8 fp16 channels of the low half (lo) and the matching 8 of the high
+// half (hi) into pairs P[8q .. 8q+8), after the rotation's sign flips when
+// SIGNS (the plain Hadamard transform has none).
+template <int D, bool SIGNS>
+__device__ __forceinline__ void widen_chunk(uint4 lo, uint4 hi, int q, const QuantSmem<D>& sm, f2_t (&P)[D / 2]) {
+    if constexpr (SIGNS) {
+        const uint4 ml = reinterpret_cast<const uint4*>(sm.sgn2)[q];
+        const uint4 mh = reinterpret_cast<const uint4*>(sm.sgn2)[D / 16 + q];
+        lo.x ^= ml.x; lo.y ^= ml.y; lo.z ^= ml.z; lo.w ^= ml.w;
+        hi.x ^= mh.x; hi.y ^= mh.y; hi.z ^= mh.z; hi.w ^= mh.w;
+    }
+    const __half2* hl = reinterpret_cast<const __half2*>(&lo);
+    const __half2* hh = reinterpret_cast<const __half2*>(&hi);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 a = __half22float2(hl[i]), b = __half22float2(hh[i]);
+        P[8 * q + 2 * i] = f2_pack(a.x, b.x);
+        P[8 * q + 2 * i + 1] = f2_pack(a.y, b.y);
+    }
+}
+
+// The row as pairs P[j] = (channel j, channel j + D/2) from its raw fp16
+// chunks (chunk q = channels 8q .. 8q + 7).
+template <int D, bool SIGNS>
+__device__ __forceinline__ void widen_row(const uint4 (&raw)[D / 8], const QuantSmem<D>& sm, f2_t (&P)[D / 2]) {
+#pragma unroll
+    for (int q = 0; q < D / 16; ++q) widen_chunk<D, SIGNS>(raw[q], raw[D / 16 + q], q, sm, P);
+}
 
 // V code rows of head dim 128 are stored pair-interleaved, the layout the
 // decode kernel's value operand wants (two tokens' codes of one channel in
@@ -468,20 +550,24 @@ __device__ __forceinline__ void store_codes(const QuantOut& out, int t, const ui
     store_words<L::kWords>(out.codes + (size_t)t * L::kBytes, w);
 }
 
-template <int D>
-__device__ __forceinline__ void store_pair_row(float* red, const f2_t (&P)[D / 2], int t) {
-    constexpr int NCH = D / 4;  // 16-byte chunks per row
-    char* row = reinterpret_cast<char*>(red) + (size_t)t * D * 4;
-#pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-        const int pk = k ^ (t & (NCH - 1));
-        *reinterpret_cast<ulonglong2*>(row + pk * 16) = make_ulonglong2(P[2 * k], P[2 * k + 1]);
-    }
-}
-
 // Sign of channel c of the rotation as an fp16 sign-bit mask.
 __device__ __forceinline__ uint16_t sign16(const uint32_t* sgn2, int c) {
     return (uint16_t)((sgn2[c >> 1] >> ((c & 1) * 16)) & 0x8000u);
+}
+
+// 8-byte shared-memory load kept in program order (volatile), so that a loop
+// of them does not have all its loads hoisted ahead of their uses.
+__device__ __forceinline__ f2_t lds_f2(uint32_t addr) {
+    f2_t r;
+    asm volatile("ld.shared.b64 %0, [%1];" : "=l"(r) : "r"(addr));
+    return r;
+}
+
+// max over the warp's lanes of |x| (exact: a comparison, no rounding).
+__device__ __forceinline__ float warp_max_abs(float x) {
+    float r;
+    asm volatile("redux.sync.max.abs.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+    return r;
 }
 
 // Offset-binary code words of one pair: lanes of fma(x, inv, kC) (see
@@ -509,7 +595,11 @@ __device__ __forceinline__ uint32_t pack_half(const uint32_t* e) {
 }
 
 // Codes of the row held in registers (reciprocal scales in pair order in
-// vec), packed group by group so that few code words are live at once.
+// vec), packed as they are produced: a group of GP pairs gives GP codes of
+// the low half (channels j ..) and GP of the high half (channels j + D/2 ..),
+// folded at once into half-words (INT4 / INT2, and the 2-bit plane of INT3)
+// or bytes (the bit plane of INT3), so that few code words are live while
+// most of the row still is.
 template <int D, int BITS, bool CLAMP>
 __device__ __forceinline__ void codes_from_regs(const f2_t (&P)[D / 2], const float* vec,
                                                 uint32_t (&w)[RowLayout<D, BITS>::kWords]) {
@@ -517,8 +607,9 @@ __device__ __forceinline__ void codes_from_regs(const f2_t (&P)[D / 2], const fl
     constexpr int H2 = D / 2;
     constexpr float kQ = (float)L::kQmax;
     constexpr float kC = 12582912.0f + (float)L::kOff;
-    constexpr int GP = (BITS == 4) ? 8 : (BITS == 2 ? 16 : (H2 < 32 ? H2 : 32));
+    constexpr int GP = (BITS == 4) ? 4 : 8;  // pairs per group: one half-word of codes per half
     const f2_t* iv = reinterpret_cast<const f2_t*>(vec);
+    uint32_t pend_lo = 0, pend_hi = 0;  // the first half-words of the words being built
 #pragma unroll
     for (int q = 0; q < H2 / GP; ++q) {
         uint32_t lo[GP], hi[GP];
@@ -528,38 +619,51 @@ __device__ __forceinline__ void codes_from_regs(const f2_t (&P)[D / 2], const fl
             code_pair<CLAMP>(P[q * GP + i], r.x, kQ, kC, lo[i], hi[i]);
             code_pair<CLAMP>(P[q * GP + i + 1], r.y, kQ, kC, lo[i + 1], hi[i + 1]);
         }
+        uint32_t hl, hh;  // this group's half-words (16 bits of codes in the low half)
         if constexpr (BITS == 4) {
-            w[q] = prmt32(pack_half<4, 4>(lo), pack_half<4, 4>(lo + 4), 0x5410u);
-            w[H2 / 8 + q] = prmt32(pack_half<4, 4>(hi), pack_half<4, 4>(hi + 4), 0x5410u);
+            hl = pack_half<4, 4>(lo);
+            hh = pack_half<4, 4>(hi);
         } else if constexpr (BITS == 2) {
-            w[q] = prmt32(pack_half<8, 2>(lo), pack_half<8, 2>(lo + 8), 0x5410u);
-            w[H2 / 16 + q] = prmt32(pack_half<8, 2>(hi), pack_half<8, 2>(hi + 8), 0x5410u);
+            hl = pack_half<8, 2>(lo);
+            hh = pack_half<8, 2>(hi);
         } else {
+            // the 2-bit plane (e & 3) and the bit plane (bit 2 of e)
+            hl = 0; hh = 0;
+            uint32_t bl = 0, bh = 0;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const uint32_t* e = half ? hi : lo;
-                const int c0 = half * H2 + q * GP;
-#pragma unroll
-                for (int m = 0; m < GP / 16; ++m) {
-                    uint32_t v = 0;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v |= (e[16 * m + i] & 3u) << (2 * i);
-                    w[c0 / 16 + m] = v;
-                }
-                static_assert(GP == 32, "one bit-plane word per run");
-                uint32_t b = 0;
-#pragma unroll
-                for (int i = 0; i < GP; ++i) b |= ((e[i] >> 2) & 1u) << i;
-                w[D / 16 + c0 / 32] = b;
+            for (int i = 0; i < GP; ++i) {
+                hl |= (lo[i] & 3u) << (2 * i);
+                hh |= (hi[i] & 3u) << (2 * i);
+                bl |= ((lo[i] >> 2) & 1u) << i;
+                bh |= ((hi[i] >> 2) & 1u) << i;
             }
+            constexpr int BP = D / 16;  // first word of the bit plane
+            const int sh = 8 * (q & 3);
+            if ((q & 3) == 0) {
+                w[BP + q / 4] = bl;
+                w[BP + H2 / 32 + q / 4] = bh;
+            } else {
+                w[BP + q / 4] |= bl << sh;
+                w[BP + H2 / 32 + q / 4] |= bh << sh;
+            }
+        }
+        // two groups make a word: 8 INT4 codes, 16 INT2 codes or 16 2-bit fields
+        constexpr int WH = (BITS == 4) ? H2 / 8 : H2 / 16;  // words of the low half
+        if (q & 1) {
+            w[q / 2] = prmt32(pend_lo, hl, 0x5410u);
+            w[WH + q / 2] = prmt32(pend_hi, hh, 0x5410u);
+        } else {
+            pend_lo = hl;
+            pend_hi = hh;
         }
     }
 }
 
-// Quantize the 128 token rows of one block.  Thread t (0..127) holds row t
-// as pairs P[j] = (x[j], x[j + D/2]) in fp32 (widened from fp16), with the
-// rotation signs already applied under HADAMARD; all 128 threads of the CTA
-// call this.
+// Quantize the 128 token rows of one block.  Thread t (0..127) passes row t
+// as its raw fp16 chunks (chunk q = channels 8q .. 8q + 7, without the
+// rotation's signs) and works on it as pairs P[j] = (x[j], x[j + D/2]) in
+// fp32, with the signs applied (SIGNS) when the pairs are formed; all 128
+// threads of the CTA call this.
 //   nsep:  n = ||x||, u = H(s (.) x) * (c0 / n)
 //   NSN:   s1 = ||x|| rsqd, a = x (sqd / ||x||), o = block mean of a (fp16),
 //          b = a - o, s2 = ||b|| rsqd, u = H(s (.) b) * (c0 / ||b||)
@@ -569,100 +673,115 @@ __device__ __forceinline__ void codes_from_regs(const f2_t (&P)[D / 2], const fl
 // rne(u * (1/sigma)) clamped.  Sign flips commute exactly with every step
 // up to the rotation (means, norms, fp16 rounding are all sign-symmetric),
 // which is why they can be applied when the row is loaded; the stored
-// offsets are flipped back.  done() is called by every thread right after
-// the barrier that follows the last read of the fp16 tile and of the
-// transpose buffer.
-template <int D, int BITS, int MODE, bool HAD, typename Done>
-__device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, const QuantSmem<D>& sm,
-                                              const QuantOut& out, const float rsqd, const float sqd, Done done) {
+// offsets are flipped back.  out gives the block's output pointers
+// (built where they are used, to keep registers free).  The fp16 tile is
+// last read before the barrier that publishes the NSN means; codes are
+// staged (QuantOut::stage) only after a later barrier, so the staging tile
+// may overlay the fp16 tile.
+template <int D, int BITS, int MODE, bool HAD, bool SIGNS, typename Pre, typename Post>
+__device__ __forceinline__ void quantize_rows(uint4 (&raw)[D / 8], const int t, const QuantSmem<D>& sm,
+                                              const QuantOut& out, const float rsqd, const float sqd,
+                                              Pre before_spill, Post after_means) {
     using L = RowLayout<D, BITS>;
     constexpr int H2 = D / 2;
     const float c0 = HAD ? rsqd : 1.0f;
     float kscale = 1.0f;
+    f2_t P[H2];
 
     if constexpr (MODE == kNsn) {
-        const float n1 = __fsqrt_rn(row_sumsq<H2>(P));
+        const float n1 = __fsqrt_rn(raw_row_sumsq<D>(raw));
         const float s1 = __fmul_rn(n1, rsqd);
         const float r1 = n1 > 0.0f ? __fdiv_rn(sqd, n1) : 0.0f;
-        sm.tokv[t] = r1;
+        // a = x * r1, with the rotation's signs when SIGNS
+        widen_row<D, SIGNS>(raw, sm, P);
         const f2_t R1 = f2_pack(r1, r1);
 #pragma unroll
-        for (int j = 0; j < H2; ++j) P[j] = f2_mul(P[j], R1);
+        for (int j = 0; j < H2; ++j) P[j] = f2_mul_sep(P[j], R1);
+        before_spill();
+        __syncthreads();  // every row has been read from the tile region
+        {
+            // the rows of a into the transposed buffer
+            constexpr int NCH2 = D / 8;  // 16-byte chunks (two pairs) per half row
+            char* lo = reinterpret_cast<char*>(sm.red_lo) + (size_t)t * (D / 2) * 4;
+            char* hi = reinterpret_cast<char*>(sm.red_hi) + (size_t)t * (D / 2) * 4;
+#pragma unroll
+            for (int k = 0; k < 2 * NCH2; ++k) {
+                const int pk = (k % NCH2) ^ (t & (NCH2 - 1));
+                *reinterpret_cast<ulonglong2*>((k < NCH2 ? lo : hi) + pk * 16) = make_ulonglong2(P[2 * k], P[2 * k + 1]);
+            }
+        }
         __syncthreads();
         {
-            // block means of a = x * r1 straight from the fp16 tile (the
-            // unsigned values; the same products as the rows'): thread t
-            // sums the 8 channels of chunk column kc8 over the TGc tokens of
-            // group gc in the pairwise (binary-counter) order
-            constexpr int NKC = D / 8, NGC = kT / NKC, TGC = kT / NGC;
-            static_assert(NGC * D * 4 <= kGpartBytes, "group sums fit the partials buffer");
-            const int kc8 = t % NKC, gc = t / NKC;
-            const uint8_t* colp = sm.tile + (kc8 / 8) * (kT * 128);
-            const int ck = kc8 % 8;
-            f2_t acc[4][6];
+            // block means: thread t sums chunk column kc (pairs 2 kc, 2 kc + 1)
+            // over the TG tokens of group g in the pairwise (binary-counter)
+            // order; the NG group sums meet in the top levels of the tree
+            constexpr int NCH2 = D / 8, NCH = 2 * NCH2, TG = NCH, NG = kT / TG;
+            static_assert(NG * D * 4 <= kGpartBytes, "group sums fit the partials buffer");
+            constexpr int LV = (TG == 32) ? 5 : 4;  // log2 TG
+            const int kc = t % NCH, g = t / NCH;
+            const char* base = reinterpret_cast<const char*>(kc < NCH2 ? sm.red_lo : sm.red_hi) +
+                               (size_t)g * TG * (D / 2) * 4;
+            const int kh = kc % NCH2;
+            f2_t acc[2][LV];
+            f2_t cur[2];
 #pragma unroll
-            for (int i = 0; i < TGC; ++i) {
-                const int tt = gc * TGC + i;
-                const uint4 raw = *reinterpret_cast<const uint4*>(colp + tt * 128 + ((ck ^ (tt & 7)) << 4));
-                const float rt = sm.tokv[tt];
-                const f2_t RT = f2_pack(rt, rt);
-                const __half2* hp = reinterpret_cast<const __half2*>(&raw);
-                f2_t cur[4];
+            for (int i = 0; i < TG; ++i) {
+                const int tt = g * TG + i;
+                const ulonglong2 x =
+                    *reinterpret_cast<const ulonglong2*>(base + (size_t)i * (D / 2) * 4 + ((kh ^ (tt & (NCH2 - 1))) << 4));
+                cur[0] = x.x;
+                cur[1] = x.y;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 x = __half22float2(hp[e]);
-                    cur[e] = f2_mul(f2_pack(x.x, x.y), RT);
-                }
-#pragma unroll
-                for (int l = 0; l < 6; ++l) {
+                for (int l = 0; l < LV; ++l) {
                     if ((i >> l) & 1) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) cur[e] = f2_add(acc[e][l], cur[e]);
+                        cur[0] = f2_add(acc[0][l], cur[0]);
+                        cur[1] = f2_add(acc[1][l], cur[1]);
                     } else {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[e][l] = cur[e];
+                        acc[0][l] = cur[0];
+                        acc[1][l] = cur[1];
                         break;
                     }
                 }
-                if (i == TGC - 1) {
-                    f2_t* gp = reinterpret_cast<f2_t*>(sm.gpart) + (gc * D + 8 * kc8) / 2;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) gp[e] = cur[e];
-                }
             }
+            // cur: the sum over the group (pair order index 4 kc .. 4 kc + 3)
+            *reinterpret_cast<ulonglong2*>(sm.gpart + g * D + 4 * kc) = make_ulonglong2(cur[0], cur[1]);
         }
         __syncthreads();
         if (t < D) {
-            // the group sums meet in the top levels of the pairwise tree
-            constexpr int NGC = kT / (D / 8);
-            float g[NGC];
+            // pair-order index t: channel c = pair t >> 1 of half t & 1
+            constexpr int NG = kT / (D / 4);
+            float gs[NG];
 #pragma unroll
-            for (int k = 0; k < NGC; ++k) g[k] = sm.gpart[k * D + t];
+            for (int k = 0; k < NG; ++k) gs[k] = sm.gpart[k * D + t];
 #pragma unroll
-            for (int w = 1; w < NGC; w *= 2) {
+            for (int w = 1; w < NG; w *= 2) {
 #pragma unroll
-                for (int k = 0; k < NGC; k += 2 * w) g[k] = __fadd_rn(g[k], g[k + w]);
+                for (int k = 0; k < NG; k += 2 * w) gs[k] = __fadd_rn(gs[k], gs[k + w]);
             }
-            const __half o16 = __float2half_rn(__fmul_rn(g[0], 1.0f / 128.0f));
-            out.off[t] = o16;
-            // the rows carry the rotation's signs: subtract s_c * o there
-            float ov = __half2float(o16);
-            if constexpr (HAD) ov = sign16(sm.sgn2, t) ? -ov : ov;
-            sm.vec[2 * (t % H2) + t / H2] = ov;
+            // the mean of the signed rows; the stored mean is of the unsigned
+            // ones (a sign flip commutes exactly with the sum and the rounding)
+            const __half o16 = __float2half_rn(__fmul_rn(gs[0], 1.0f / 128.0f));
+            const int c = (t >> 1) + (t & 1) * H2;
+            out.off[c] = (SIGNS && sign16(sm.sgn2, c)) ? __hneg(o16) : o16;
+            sm.vec[t] = __half2float(o16);
         }
         __syncthreads();
-        const f2_t* mv = reinterpret_cast<const f2_t*>(sm.vec);
+        after_means();  // the transposed buffer is free again
+        // b = a - s (.) o
+        const uint32_t mv = smem_u32(sm.vec);
 #pragma unroll
-        for (int j = 0; j < H2; ++j) P[j] = f2_sub(P[j], mv[j]);
-        const float n2 = __fsqrt_rn(row_sumsq<H2>(P));
+        for (int j = 0; j < H2; ++j) P[j] = f2_sub(P[j], lds_f2(mv + 8 * j));
+        const float n2 = __fsqrt_rn(row_sumsq<H2, false>(P));
         const float s2 = __fmul_rn(n2, rsqd);
         kscale = n2 > 0.0f ? __fdiv_rn(c0, n2) : 0.0f;
         reinterpret_cast<__half2*>(out.tok)[t] = __halves2half2(__float2half_rn(s1), __float2half_rn(s2));
     } else if constexpr (MODE == kNsep) {
-        const float n = __fsqrt_rn(row_sumsq<H2>(P));
+        widen_row<D, SIGNS>(raw, sm, P);
+        const float n = __fsqrt_rn(row_sumsq<H2, true>(P));
         out.tok[t] = __float2half_rn(n);
         kscale = n > 0.0f ? __fdiv_rn(c0, n) : 0.0f;
     } else {
+        widen_row<D, SIGNS>(raw, sm, P);
         kscale = c0;
     }
 
@@ -676,8 +795,7 @@ __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, con
     constexpr float kQ = (float)L::kQmax;
     constexpr float kC = 12582912.0f + (float)L::kOff;  // 1.5 * 2^23 + offset
     if constexpr (MODE == kNaive) {
-        __syncthreads();
-        done();
+        __syncthreads();  // every row has been read from the tile the codes are staged over
         uint32_t cw[D];
         float m = 0.0f;
 #pragma unroll
@@ -704,47 +822,27 @@ __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, con
         pack_codes<D, BITS>(cw, w);
         store_codes<D, BITS>(out, t, w);
     } else {
-        // per-channel absmax over the block through the transpose buffer:
-        // thread t takes chunk column kc (two pairs) of the TG tokens of group g
-        constexpr int NCH = D / 4, NCH2 = D / 8, TG = NCH, NG = kT / TG;
-        static_assert(NG * D * 4 <= kGpartBytes, "group maxima fit the partials buffer");
-        const int kc = t % NCH, g = t / NCH;
-        {
-            char* lo = reinterpret_cast<char*>(sm.red_lo) + (size_t)t * (D / 2) * 4;
-            char* hi = reinterpret_cast<char*>(sm.red_hi) + (size_t)t * (D / 2) * 4;
+        // per-channel absmax over the block: one redux per channel and warp
+        // gives the max over the warp's 32 tokens to every lane; lane k
+        // stores the four values of pairs 2k, 2k + 1 (pair order)
+        const int lane = t & 31, warp = t >> 5;
+        float* wm = sm.gpart + warp * D;
+        static_assert(4 * D * 4 <= kGpartBytes, "warp maxima fit the partials buffer");
 #pragma unroll
-            for (int k = 0; k < NCH; ++k) {
-                const int pk = (k % NCH2) ^ (t & (NCH2 - 1));
-                *reinterpret_cast<ulonglong2*>((k < NCH2 ? lo : hi) + pk * 16) = make_ulonglong2(P[2 * k], P[2 * k + 1]);
-            }
-        }
-        __syncthreads();
-        {
-            const char* base = reinterpret_cast<const char*>(kc < NCH2 ? sm.red_lo : sm.red_hi) +
-                               (size_t)g * TG * (D / 2) * 4;
-            const int kh = kc % NCH2;
-            float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
-#pragma unroll 4
-            for (int i = 0; i < TG; ++i) {
-                const int tt = g * TG + i;
-                const float4 x =
-                    *reinterpret_cast<const float4*>(base + (size_t)i * (D / 2) * 4 + ((kh ^ (tt & (NCH2 - 1))) << 4));
-                m0 = fmaxf(m0, fabsf(x.x));
-                m1 = fmaxf(m1, fabsf(x.y));
-                m2 = fmaxf(m2, fabsf(x.z));
-                m3 = fmaxf(m3, fabsf(x.w));
-            }
-            // group maxima in pair order: [group][pair-order index of the row]
-            reinterpret_cast<float4*>(sm.gpart)[g * NCH + kc] = make_float4(m0, m1, m2, m3);
+        for (int j = 0; j < H2; j += 2) {
+            float a0, b0, a1, b1;
+            f2_unpack(P[j], a0, b0);
+            f2_unpack(P[j + 1], a1, b1);
+            const float r0 = warp_max_abs(a0), r1 = warp_max_abs(b0);
+            const float r2 = warp_max_abs(a1), r3 = warp_max_abs(b1);
+            if (lane == ((j >> 1) & 31)) *reinterpret_cast<float4*>(wm + 2 * j) = make_float4(r0, r1, r2, r3);
         }
         __syncthreads();
         int clamp = 0;
         if (t < D) {
             // t indexes the pair-order vector: pair t >> 1, lane t & 1
             const int c = (t >> 1) + (t & 1) * H2;
-            float m = 0.0f;
-#pragma unroll
-            for (int gg = 0; gg < NG; ++gg) m = fmaxf(m, sm.gpart[gg * D + t]);
+            const float m = fmaxf(fmaxf(sm.gpart[t], sm.gpart[D + t]), fmaxf(sm.gpart[2 * D + t], sm.gpart[3 * D + t]));
             const __half s16 = __float2half_rn(__fdiv_rn(m, kQ));
             out.chan[c] = s16;
             const float sf = __half2float(s16);
@@ -755,7 +853,6 @@ __device__ __forceinline__ void quantize_rows(f2_t (&P)[D / 2], const int t, con
             clamp = __fmaf_rn(m, inv, -(kQ + 0.5f)) >= 0.0f;
         }
         const int any_clamp = __syncthreads_or(clamp);
-        done();
         uint32_t w[L::kWords];
         if (!any_clamp) codes_from_regs<D, BITS, false>(P, sm.vec, w);
         else codes_from_regs<D, BITS, true>(P, sm.vec, w);

@@ -21,29 +21,48 @@ struct QuantArgs {
     float rsqd, sqd; // (float)(1/sqrt(d)), (float)sqrt(d)
 };
 
-// Shared memory of a quantizer CTA: three regions of one fp16 tile each
-// (128 x D x 2 bytes, which is also half of the fp32 transpose buffer), the
-// small vectors and three mbarriers.
+// Shared memory of a quantizer CTA: tile-sized regions (128 x D x 2
+// bytes; a region also stages a tile's codes for the TMA store once the tile
+// has been read), the small vectors and one mbarrier per region.  NSN uses
+// three regions: two of them hold the block's fp32 rows for the means (the
+// transposed buffer) while the third receives the next tile.
+template <int MODE>
+__host__ __device__ constexpr int quant_regions() {
+    return MODE == kNsn ? 3 : 2;
+}
+
 template <int D>
 __host__ __device__ constexpr int quant_region_bytes() {
     return kT * D * 2;
 }
 
-template <int D>
+template <int D, int MODE>
 __host__ __device__ constexpr int quant_smem_bytes() {
-    // 1024 B alignment slack + 3 regions + vec + group partials + token vector + sign masks + mbarriers
-    return 1024 + 3 * quant_region_bytes<D>() + D * 4 + kGpartBytes + kT * 4 + D * 4 + 3 * 8;
+    // 1024 B alignment slack + regions + vec + group partials + token vector + sign masks + mbarriers
+    return 1024 + quant_regions<MODE>() * quant_region_bytes<D>() + D * 4 + kGpartBytes + kT * 4 + D * 4 +
+           quant_regions<MODE>() * 8;
 }
 
-template <int D>
+// Resident quantizer CTAs per SM the register budget is set for: a thread
+// holds a whole row of D fp32 values.  Under NSN that row stays live
+// through the block means as well, and the rotated INT3 codes need more
+// registers than three CTAs leave; those run two CTAs per SM.
+template <int D, int BITS, int MODE, bool HAD>
+__host__ __device__ constexpr int quant_min_ctas() {
+    return D == 128 ? ((MODE == kNsn || (HAD && BITS == 3)) ? 2 : 3) : 4;
+}
+
+template <int D, int MODE>
 __device__ __forceinline__ QuantSmem<D> carve_quant_smem(uint8_t* base, uint64_t*& bar, uint8_t*& regions) {
-    uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023));
+    // 1024-byte alignment (TMA 128-byte swizzle) by an offset from the base,
+    // so that the pointers stay known to address shared memory
+    uint8_t* p = base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
     QuantSmem<D> sm;
     regions = p;
     sm.tile = p;
-    sm.red_lo = reinterpret_cast<float*>(p + quant_region_bytes<D>());
-    sm.red_hi = reinterpret_cast<float*>(p + 2 * quant_region_bytes<D>());
-    p += 3 * quant_region_bytes<D>();
+    sm.red_lo = reinterpret_cast<float*>(p);
+    sm.red_hi = reinterpret_cast<float*>(p + quant_region_bytes<D>());
+    p += quant_regions<MODE>() * quant_region_bytes<D>();
     sm.vec = reinterpret_cast<float*>(p);
     p += D * 4;
     sm.gpart = reinterpret_cast<float*>(p);
@@ -85,52 +104,47 @@ __device__ __forceinline__ void load_signs(const QuantArgs& a, const QuantSmem<D
     }
 }
 
-// Widen 8 fp16 channels of the low half (lo) and the matching 8 of the high
-// half (hi) into pairs P[8q .. 8q+8), after the rotation's sign flips.
-template <int D, bool HAD>
-__device__ __forceinline__ void widen_chunk(uint4 lo, uint4 hi, int q, const QuantSmem<D>& sm, f2_t (&P)[D / 2]) {
-    if constexpr (HAD) {
-        const uint4 ml = reinterpret_cast<const uint4*>(sm.sgn2)[q];
-        const uint4 mh = reinterpret_cast<const uint4*>(sm.sgn2)[D / 16 + q];
-        lo.x ^= ml.x; lo.y ^= ml.y; lo.z ^= ml.z; lo.w ^= ml.w;
-        hi.x ^= mh.x; hi.y ^= mh.y; hi.z ^= mh.z; hi.w ^= mh.w;
-    }
-    const __half2* hl = reinterpret_cast<const __half2*>(&lo);
-    const __half2* hh = reinterpret_cast<const __half2*>(&hi);
+// Row t of the tile as its raw fp16 chunks (chunk q = channels 8q .. 8q + 7).
+template <int D>
+__device__ __forceinline__ void load_tile_raw(const uint8_t* tile, int t, uint4 (&raw)[D / 8]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 a = __half22float2(hl[i]), b = __half22float2(hh[i]);
-        P[8 * q + 2 * i] = f2_pack(a.x, b.x);
-        P[8 * q + 2 * i + 1] = f2_pack(a.y, b.y);
+    for (int q = 0; q < D / 8; ++q) {
+        const int c = 8 * q;
+        raw[q] = *reinterpret_cast<const uint4*>(tile + (c / 64) * (kT * 128) + t * 128 + ((((c % 64) / 8) ^ (t & 7)) << 4));
     }
 }
 
 // Persistent quantizer: CTA c takes the work items c, c + gridDim.x, ... of
-// the list (batch * head, block, tensor).  Three tile-sized regions rotate:
-// item i's fp16 tile arrives by TMA in region i % 3 (64-channel boxes with
-// 128-byte swizzle, chunk c of row t at chunk c ^ (t & 7)) while item i - 1
-// is quantized; once item i has read its tile, that region and the free one
-// form its fp32 transpose buffer, and when the transpose buffer has been read
-// the free region takes item i + 2.
+// the list (batch * head, block, tensor).  NR = quant_regions regions
+// rotate: item i's fp16 tile arrives by TMA in region i % NR (64-channel
+// boxes with 128-byte swizzle, chunk c of row t at chunk c ^ (t & 7)) while
+// earlier items are quantized, and once its rows have been read the region
+// stages item i's codes for a TMA store.  With two regions, region (i + 1)
+// % 2 takes item i + 2 at the start of item i + 1 (when the store has read
+// the staging tile).  With three (NSN), regions i % 3 and (i + 2) % 3 hold
+// the block's fp32 rows for the means, after which region (i + 2) % 3 takes
+// item i + 2.  A thread owns one token row (D fp32 values in registers),
+// and the register budget is set for quant_min_ctas resident CTAs per SM.
 template <int D, int BITS, int MODE, bool HAD>
-__global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ CUtensorMap map_k,
-                                                       const __grid_constant__ CUtensorMap map_v,
-                                                       const __grid_constant__ CUtensorMap map_ck,
-                                                       const __grid_constant__ CUtensorMap map_cv, QuantArgs a) {
+__global__ void __launch_bounds__(128, (quant_min_ctas<D, BITS, MODE, HAD>())) quantize_kernel(
+    const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+    const __grid_constant__ CUtensorMap map_ck, const __grid_constant__ CUtensorMap map_cv, QuantArgs a) {
     // INT4 / INT2 code rows leave through a TMA store of a swizzled staging
     // tile (the region just read), so that each warp writes whole lines
     constexpr bool kTmaStore = (BITS == 4 && D * BITS / 8 == 64) || (BITS == 2 && D * BITS / 8 == 32);
+    constexpr int NR = quant_regions<MODE>();
     extern __shared__ uint8_t smem_raw[];
     const int t = threadIdx.x;
-    uint64_t* bar;  // [3]
+    uint64_t* bar;  // [NR]
     uint8_t* regions;
-    QuantSmem<D> sm = carve_quant_smem<D>(smem_raw, bar, regions);
+    QuantSmem<D> sm = carve_quant_smem<D, MODE>(smem_raw, bar, regions);
     constexpr uint32_t kTileBytes = quant_region_bytes<D>();
     const int nblk = a.ntok / kT;
     const int nitems = nblk * a.bh * 2;  // < 2^31, checked on the host
+    const bool signs = HAD && a.signs != nullptr;
 
     if (t == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < NR; ++i) mbar_init(&bar[i], 1);
         fence_mbar_init();
     }
     load_signs<D, HAD>(a, sm, t);
@@ -158,56 +172,62 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __grid_constant__ C
     int it = 0;
     uint32_t phases = 0;  // bit k: parity of the next completion of region k
     for (; w < nitems; w += stride, ++it) {
-        const int reg = it % 3;
+        const int reg = it % NR;
+        if (NR == 2 && it > 0 && t == 0) {
+            // the previous item's region: free once its code store has read
+            // the staging tile; it takes the next item
+            if (kTmaStore) bulk_wait_read();
+            if (w + stride < nitems) {
+                fence_proxy_async_smem();
+                issue(w + stride, reg ^ 1);
+            }
+        }
         const bool landed = mbar_wait(&bar[reg], (phases >> reg) & 1, 1u << 24);
-        if (kTmaStore && t == 0) bulk_wait_read();  // the last code store has read its staging tile
         if (__syncthreads_or(!landed)) {
             if (t == 0) report_error(kErrTmaTimeout);
             break;
         }
         phases ^= 1u << reg;
-        const uint8_t* tile = regions + reg * kTileBytes;
-        const int spare = (it + 2) % 3;
+        uint8_t* tile = regions + reg * kTileBytes;
         sm.tile = tile;
-        sm.red_lo = reinterpret_cast<float*>(regions + reg * kTileBytes);
+        const int spare = (reg + 2) % NR;  // NSN: the region of the item after next
+        sm.red_lo = reinterpret_cast<float*>(tile);
         sm.red_hi = reinterpret_cast<float*>(regions + spare * kTileBytes);
         const int tensor = w & 1;
         const int r = w >> 1;
         const int bh = r / nblk, blk = r - bh * nblk;
-        // row t as pairs (channel j, channel j + D/2)
-        f2_t P[D / 2];
-#pragma unroll
-        for (int q = 0; q < D / 16; ++q) {
-            const int cl = 8 * q, ch = D / 2 + 8 * q;
-            const uint8_t* rl = tile + (cl / 64) * (kT * 128) + t * 128;
-            const uint8_t* rh = tile + (ch / 64) * (kT * 128) + t * 128;
-            const uint4 lo = *reinterpret_cast<const uint4*>(rl + ((((cl % 64) / 8) ^ (t & 7)) << 4));
-            const uint4 hi = *reinterpret_cast<const uint4*>(rh + ((((ch % 64) / 8) ^ (t & 7)) << 4));
-            widen_chunk<D, HAD>(lo, hi, q, sm, P);
-        }
-        if constexpr (MODE != kNsn) __syncthreads();  // the tile region becomes transpose buffer
-        const int wn = w + 2 * stride;
+        uint4 raw[D / 8];
+        load_tile_raw<D>(tile, t, raw);
         QuantOut out = quant_out<D, BITS, MODE, HAD>(a, tensor, bh, a.blk0 + blk);
-        if constexpr (kTmaStore) out.stage = regions + reg * kTileBytes;
-        quantize_rows<D, BITS, MODE, HAD>(P, t, sm, out, a.rsqd, a.sqd, [&] {
-            if (t == 0 && wn < nitems) {
+        if constexpr (kTmaStore) out.stage = tile;
+        // NSN: the spare region is written once the previous item's code store
+        // has read it, and takes item w + 2 stride after the means
+        auto before_spill = [&] {
+            if (NR == 3 && kTmaStore && t == 0) bulk_wait_read();
+        };
+        auto after_means = [&] {
+            if (NR == 3 && t == 0 && w + 2 * stride < nitems) {
                 fence_proxy_async_smem();
-                issue(wn, spare);
+                issue(w + 2 * stride, spare);
             }
-        });
-        __syncthreads();  // the next item's row loads reuse the shared vectors; codes staged
+        };
+        if (signs) quantize_rows<D, BITS, MODE, HAD, true>(raw, t, sm, out, a.rsqd, a.sqd, before_spill, after_means);
+        else quantize_rows<D, BITS, MODE, HAD, false>(raw, t, sm, out, a.rsqd, a.sqd, before_spill, after_means);
+        __syncthreads();  // codes staged; the next item's rows reuse the shared vectors
         if (kTmaStore && t == 0) {
-            tma_store_2d(tensor ? &map_cv : &map_ck, 0, bh * a.cap + (a.blk0 + blk) * kT, out.stage);
+            tma_store_2d(tensor ? &map_cv : &map_ck, 0, bh * a.cap + (a.blk0 + blk) * kT, tile);
             bulk_commit();
         }
     }
     if (kTmaStore && t == 0) bulk_wait_read();
-    // after an early exit, the copies still in flight (items w and w + stride)
-    // land before the CTA ends
+    // after an early exit, the copies still in flight land before the CTA
+    // ends: items w and w + stride (both issued by then), and under NSN item
+    // w + 2 stride when item w - stride issued it
     if (t == 0 && w < nitems) {
-        for (int k = 0; k < 2; ++k) {
-            const int reg = (it + k) % 3;
-            if (w + k * stride < nitems) mbar_wait(&bar[reg], (phases >> reg) & 1, 1u << 24);
+        for (int k = 0; k < NR; ++k) {
+            const int reg = (it + k) % NR;
+            const bool issued = k < 2 || it > 0;
+            if (issued && w + k * stride < nitems) mbar_wait(&bar[reg], (phases >> reg) & 1, 1u << 24);
         }
     }
 }
@@ -237,26 +257,20 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
     }
     extern __shared__ uint8_t smem_raw[];
     uint64_t* bar;
-    uint8_t* tile;
-    QuantSmem<D> sm = carve_quant_smem<D>(smem_raw, bar, tile);
+    uint8_t* regions;
+    QuantSmem<D> sm = carve_quant_smem<D, MODE>(smem_raw, bar, regions);
     load_signs<D, HAD>(a.q, sm, t);
     __syncthreads();
     const __half* src = (t == kT - 1) ? xn : res + (size_t)t * D;
-    f2_t P[D / 2];
+    uint4 raw[D / 8];
 #pragma unroll
-    for (int q = 0; q < D / 16; ++q) {
-        const uint4 lo = reinterpret_cast<const uint4*>(src)[q];
-        const uint4 hi = reinterpret_cast<const uint4*>(src)[D / 16 + q];
-        if constexpr (MODE == kNsn) {
-            // the fp16 tile in the quantize kernel's layout, for the block means
-            const int cl = 8 * q, ch = D / 2 + 8 * q;
-            *reinterpret_cast<uint4*>(tile + (cl / 64) * (kT * 128) + t * 128 + ((((cl % 64) / 8) ^ (t & 7)) << 4)) = lo;
-            *reinterpret_cast<uint4*>(tile + (ch / 64) * (kT * 128) + t * 128 + ((((ch % 64) / 8) ^ (t & 7)) << 4)) = hi;
-        }
-        widen_chunk<D, HAD>(lo, hi, q, sm, P);
-    }
+    for (int q = 0; q < D / 8; ++q) raw[q] = reinterpret_cast<const uint4*>(src)[q];
     const QuantOut out = quant_out<D, BITS, MODE, HAD>(a.q, tensor, bh, a.blk);
-    quantize_rows<D, BITS, MODE, HAD>(P, t, sm, out, a.q.rsqd, a.q.sqd, [] {});
+    auto none = [] {};
+    if (HAD && a.q.signs != nullptr)
+        quantize_rows<D, BITS, MODE, HAD, true>(raw, t, sm, out, a.q.rsqd, a.q.sqd, none, none);
+    else
+        quantize_rows<D, BITS, MODE, HAD, false>(raw, t, sm, out, a.q.rsqd, a.q.sqd, none, none);
 }
 
 struct DequantArgs {
