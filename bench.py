@@ -147,14 +147,16 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ oracle sample
 
-def run_oracle_sample(w, mode, bits, pairs, threads, decode_seconds):
+def run_oracle_sample(w, mode, bits, pairs, threads, decode_seconds, data=None):
     """The CPU oracle over `pairs` (batch row, kv head) slices of the
     workload: quantize of the prefill (K and V), then decode steps over the
     quantized cache (each one dequantize + fp64 attention of the slices'
     query heads with a fresh query) until about `decode_seconds` of decode
-    work.  Returns (bytes, seconds, decode steps, quantize seconds): the
-    algorithmic bytes of the quantize and of every decode step, with the
-    same accounting as the GPU path."""
+    work.  `data` = (K, V) fp16 [pairs, 1, S, d] of those slices (else they
+    are drawn here).  Returns (bytes, seconds, decode steps, quantize seconds,
+    oracle state): the algorithmic bytes of the quantize and of every decode
+    step, with the same accounting as the GPU path, and the oracle's caches
+    with the exact products of their codes (for the parity sample)."""
     import oracle
     names, seeded = synth.MODES[mode]
     flags = flags_of(mode)
@@ -162,14 +164,19 @@ def run_oracle_sample(w, mode, bits, pairs, threads, decode_seconds):
                      signs=oracle.make_signs(synth.SIGN_SEED, w.d) if seeded else None)
     G = w.Hq // w.Hkv
     ws = w.scaled(B=max(1, (pairs + w.Hkv - 1) // w.Hkv))
-    K, V = synth.kv(ws)
-    Kb = K.reshape(-1, 1, w.S, w.d)[:pairs]
-    Vb = V.reshape(-1, 1, w.S, w.d)[:pairs]
+    if data is None:
+        K, V = synth.kv(ws)
+        Kb = K.reshape(-1, 1, w.S, w.d)[:pairs]
+        Vb = V.reshape(-1, 1, w.S, w.d)[:pairs]
+    else:
+        Kb, Vb = data
     k16 = np.ascontiguousarray(Kb).view(np.uint16)
     v16 = np.ascontiguousarray(Vb).view(np.uint16)
+    ck = oracle.empty_cache(cfg, pairs, 1, w.S)
+    cv = oracle.empty_cache(cfg, pairs, 1, w.S)
     t0 = time.perf_counter()
-    ck = oracle.quantize(cfg, k16, threads=threads)
-    cv = oracle.quantize(cfg, v16, threads=threads)
+    yk = oracle.quantize_products(cfg, k16, ck, 0, threads)
+    yv = oracle.quantize_products(cfg, v16, cv, 0, threads)
     tq = time.perf_counter() - t0
     qsteps = synth.queries(ws, steps=256)
     td, n = 0.0, 0
@@ -183,7 +190,62 @@ def run_oracle_sample(w, mode, bits, pairs, threads, decode_seconds):
         n += 1
     nbytes = (accounting.quantize_bytes(w.d, bits, flags, pairs, 1, w.S)
               + n * accounting.decode_bytes(w.d, bits, flags, pairs, 1, G, w.S))
-    return nbytes, tq + td, n, tq
+    return nbytes, tq + td, n, tq, (cfg, ck, cv, yk, yv)
+
+
+def sampled_parity(w, bits, state, cache, pairs):
+    """The GPU cache's prefill blocks of the first `pairs` (batch row, kv
+    head) slices against the oracle's: codes bit-exact except at rounding
+    half-points (each difference is proven to be one: the oracle's exact
+    product lies within 1e-6 of k + 1/2), fp16 side parameters compared in
+    ulps."""
+    import oracle
+    cfg, ck, cv, yk, yv = state
+    rb = oracle.row_bytes(w.d, bits)
+    res = {"slices": pairs, "tokens_per_slice": w.S, "codes_compared": 0, "code_mismatches": 0,
+           "half_point_cases": 0, "non_half_point_mismatches": 0, "max_param_ulp": 0}
+
+    def ulps(a, b):
+        key = lambda x: np.where(x.astype(np.int32) & 0x8000, -(x.astype(np.int32) & 0x7FFF), x.astype(np.int32))
+        return int(np.max(np.abs(key(a) - key(b)))) if a.size else 0
+
+    for i, (oc, y) in enumerate(((ck, yk), (cv, yv))):
+        g = cache.codes[i].reshape(-1, cache.codes[i].shape[2], rb)[:pairs, :w.S].cpu().numpy()
+        if i == 1 and w.d == 128:
+            g = pairv_rows(g, bits)
+        gq, _ = oracle.unpack_rows(g.reshape(-1, rb), w.d, bits)
+        oq, _ = oracle.unpack_rows(oc["codes"].reshape(-1, rb), w.d, bits)
+        diff = gq.astype(np.int32) - oq.astype(np.int32)
+        bad = diff != 0
+        hp = oracle.half_point_distance(y.reshape(diff.shape)) <= 1e-6
+        res["codes_compared"] += int(diff.size)
+        res["code_mismatches"] += int(bad.sum())
+        res["half_point_cases"] += int((bad & hp).sum())
+        res["non_half_point_mismatches"] += int((bad & ~hp).sum()) + int((np.abs(diff) > 1).sum())
+        for name in ("tok", "chan", "off"):
+            gt = getattr(cache, name)[i]
+            if gt is None or oc[name] is None:
+                continue
+            n_ = oc[name].shape[2]
+            gv = gt.reshape(-1, gt.shape[2], gt.shape[3])[:pairs, :n_].cpu().numpy().view(np.uint16)
+            res["max_param_ulp"] = max(res["max_param_ulp"], ulps(gv, oc[name].reshape(gv.shape)))
+    return res
+
+
+def pairv_rows(codes, bits):
+    """Pair-interleaved V code rows of head dim 128 (the library's layout,
+    include/kvq.h) -> token-major rows, as the oracle stores them."""
+    *lead, n, rb = codes.shape
+    x = codes.reshape(*lead, n // 2, 2 * rb)
+    if bits == 4:
+        nch = 2 * rb // 16
+        ch = x.reshape(*lead, n // 2, nch, 16)
+        k = np.arange(n // 2)[:, None]
+        idx = np.arange(nch)[None, :] ^ (2 * (k & 1))
+        ch = np.take_along_axis(ch, np.broadcast_to(idx[..., None], ch.shape), axis=-2)
+        x = ch.reshape(*lead, n // 2, 2 * rb)
+    w4 = x.reshape(*lead, n // 2, rb // 2, 2, 2)
+    return np.ascontiguousarray(np.swapaxes(w4, -3, -2)).reshape(*lead, n, rb)
 
 
 def oracle_sample_text(w, pairs, n, secs):
@@ -251,7 +313,7 @@ def run_reference(args, rank: int, world: int):
         run_oracle_sample(w, MODE, BITS, pairs, threads, 1.0)
     tot_b, tot_s, tot_n = 0.0, 0.0, 0
     for _ in range(args.steps):
-        nb, secs, n, _ = run_oracle_sample(w, MODE, BITS, pairs, threads, 4.0)
+        nb, secs, n, _, _ = run_oracle_sample(w, MODE, BITS, pairs, threads, 4.0)
         tot_b += nb
         tot_s += secs
         tot_n += n
@@ -406,10 +468,14 @@ def run_ours(args, rank: int, world: int):
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
+        # the oracle on the first slices of this run's own prefill, timed,
+        # then (untimed) compared with the GPU cache of the same slices
         pairs = max(1, min(host_cores(), 32))
-        nb, secs, n, _ = run_oracle_sample(w, MODE, BITS, pairs, pairs, 12.0)
+        data = (K.reshape(-1, 1, w.S, w.d)[:pairs], V.reshape(-1, 1, w.S, w.d)[:pairs])
+        nb, secs, n, _, state = run_oracle_sample(w, MODE, BITS, pairs, pairs, 12.0, data)
         line["cpu_baseline"] = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": pairs, "kind": "oracle",
                                 "sample": oracle_sample_text(w, pairs, n, secs)}
+        line["parity"] = sampled_parity(w, BITS, state, cache, pairs)
     print(json.dumps(line), flush=True)
     return 0
 

@@ -212,6 +212,34 @@ kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t
                           int64_t t0, int64_t ntok, float* out, void* stream);
 
 /*
+ * Sign-pattern selection for the randomized Hadamard rotation
+ * ("Activation-guided compensation and orthogonal residuals" abstract:
+ * sampling several random sign patterns improves the choice of the
+ * transform; random signs keep persistent outlier channels from adding up).
+ * Quantizes a sample with each candidate sign vector exactly as
+ * kvq_quantize_block does (cfg.signs is ignored), rebuilds it as
+ * kvq_dequantize does, and measures the reconstruction error
+ *   err[k] = sum over the sample's blocks, in order, of the pairwise sum
+ *            over the block's tokens of the pairwise sum over channels of
+ *            (x_hat - x)^2, in fp64;
+ * best = the index of the smallest err (the lowest index among equal ones).
+ *   cfg     flags with KVQ_HADAMARD (nsep+pchan or NSN); head_dim, bits as usual
+ *   x       fp16 [n_blocks][128][head_dim], the sample (for instance the
+ *           first block of every (batch, kv head) slice of a prefill)
+ *   signs   int8 [n_cand][head_dim] of +-1 (e.g. kvq_make_signs of n_cand
+ *           seeds, copied to the device), 1 <= n_cand <= KVQ_SELECT_MAX_CANDIDATES
+ *   err     fp64 [n_cand] out;  best  int32 [1] out
+ *   ws      workspace of kvq_select_signs_workspace_bytes(n_cand, n_blocks)
+ *           bytes (the per-block errors; needs no initialization)
+ * Errors: INVALID_ARG; UNSUPPORTED (no HADAMARD flag, or the naive mode);
+ * WORKSPACE; CUDA.
+ */
+#define KVQ_SELECT_MAX_CANDIDATES 256
+size_t kvq_select_signs_workspace_bytes(int32_t n_cand, int64_t n_blocks);
+kvq_status kvq_select_signs(const kvq_config* cfg, const uint16_t* x, int64_t n_blocks, const int8_t* signs,
+                            int32_t n_cand, double* err, int32_t* best, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Decode attention that allocates nothing and needs no caller workspace.
  * The pages have no counterpart to this call; it exists for callers that are
  * handed only their input and output buffers and cannot allocate device

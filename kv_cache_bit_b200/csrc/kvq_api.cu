@@ -249,6 +249,28 @@ struct DequantLaunch {
     }
 };
 
+struct SelectLaunch {
+    SelectArgs a;
+    int n_cand;
+    double* err;
+    int* best;
+    cudaStream_t st;
+    template <int D, int BITS, int MODE, bool HAD>
+    kvq_status run() {
+        if constexpr (!HAD || MODE == kNaive) {
+            return KVQ_ERR_UNSUPPORTED;
+        } else {
+            constexpr int smem = select_smem_bytes<D, BITS, MODE>();
+            if (!ensure_smem<select_signs_kernel<D, BITS, MODE>>(smem)) return KVQ_ERR_CUDA;
+            select_signs_kernel<D, BITS, MODE><<<dim3(a.n_blocks, n_cand), kT, smem, st>>>(a);
+            kvq_status s = launch_status();
+            if (s != KVQ_OK) return s;
+            select_reduce_kernel<<<1, 256, 0, st>>>(a.part, a.n_blocks, n_cand, err, best);
+            return launch_status();
+        }
+    }
+};
+
 template <int D, int BITS, int MODE, bool HAD, int GP>
 kvq_status launch_decode_mma(DecodeArgs a, int bh, cudaStream_t st) {
     constexpr int smem = mma_smem_bytes<D, BITS, MODE, GP>();
@@ -456,6 +478,36 @@ kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, c
     return dispatch(cfg->head_dim, cfg->bits, mi, L);
 }
 
+size_t kvq_select_signs_workspace_bytes(int32_t n_cand, int64_t n_blocks) {
+    if (n_cand < 1 || n_cand > KVQ_SELECT_MAX_CANDIDATES || n_blocks < 1 || n_blocks > INT32_MAX) return 0;
+    return (size_t)n_cand * (size_t)n_blocks * sizeof(double);
+}
+
+kvq_status kvq_select_signs(const kvq_config* cfg, const uint16_t* x, int64_t n_blocks, const int8_t* signs,
+                            int32_t n_cand, double* err, int32_t* best, void* ws, size_t ws_bytes, void* stream) {
+    ModeInfo mi;
+    kvq_status s = check_cfg(cfg, &mi);
+    if (s != KVQ_OK) return s;
+    if (!mi.had || mi.mode == kNaive) return KVQ_ERR_UNSUPPORTED;
+    if (!ok_ptr(x) || !ok_ptr(signs) || !ok_ptr(err) || !ok_ptr(best)) return KVQ_ERR_INVALID_ARG;
+    if (n_cand < 1 || n_cand > KVQ_SELECT_MAX_CANDIDATES || n_blocks < 1 || n_blocks > INT32_MAX)
+        return KVQ_ERR_INVALID_ARG;
+    const size_t need = kvq_select_signs_workspace_bytes(n_cand, n_blocks);
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < need) return KVQ_ERR_WORKSPACE;
+    SelectLaunch L;
+    L.a.x = reinterpret_cast<const __half*>(x);
+    L.a.signs = signs;
+    L.a.part = static_cast<double*>(ws);
+    L.a.n_blocks = (int)n_blocks;
+    L.a.rsqd = rsqd_of(cfg->head_dim);
+    L.a.sqd = sqd_of(cfg->head_dim);
+    L.n_cand = n_cand;
+    L.err = err;
+    L.best = best;
+    L.st = static_cast<cudaStream_t>(stream);
+    return dispatch(cfg->head_dim, cfg->bits, mi, L);
+}
+
 kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t tensor, int64_t t0, int64_t ntok,
                           float* out, void* stream) {
     ModeInfo mi;
@@ -547,6 +599,14 @@ kvq_status kvq_read_device_errors(uint32_t* host_out, int32_t clear) {
     }
     return KVQ_OK;
 }
+
+#ifdef KVQ_WAIT_TEST
+// Test build only (not declared in kvq.h): scale of the kernels' main-loop
+// wait limits; 0 makes every such wait give up at once.
+kvq_status kvq_test_set_wait_scale(uint32_t scale) {
+    return cudaMemcpyToSymbol(g_wait_scale, &scale, sizeof(scale)) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+#endif
 
 const char* kvq_status_string(kvq_status status) {
     switch (status) {

@@ -493,7 +493,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
     int waited = 0;
     bool ok = true;
     auto wait_unit = [&](int u) -> bool {
-        if (!mbar_wait(&my_bars[u % kRing], (u / kRing) & 1, 1u << 26)) return false;
+        if (!mbar_wait(&my_bars[u % kRing], (u / kRing) & 1, KVQ_WAIT_LIMIT(1u << 26))) return false;
         waited = u + 1;
         return true;
     };

@@ -23,6 +23,18 @@ constexpr uint32_t kErrTmaTimeout = 1u;
 constexpr uint32_t kErrBarrierTimeout = 2u;
 __device__ uint32_t g_error_word = 0;  // the library is a single translation unit
 
+// Poll limit of the bounded waits in the kernels' main loops.  A separate
+// test build of the library (KVQ_WAIT_TEST, never the product build) scales
+// it by a device variable that a test sets to 0: every such wait then gives
+// up at once, so the give-up paths run (error bit, bounded drain of the
+// copies in flight) without anything hanging.  The drains keep their limits.
+#ifdef KVQ_WAIT_TEST
+__device__ uint32_t g_wait_scale = 1;
+#define KVQ_WAIT_LIMIT(n) ((n) * g_wait_scale)
+#else
+#define KVQ_WAIT_LIMIT(n) (n)
+#endif
+
 // ---------------------------------------------------------------- PTX
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

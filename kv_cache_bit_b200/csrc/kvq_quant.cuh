@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(128, (quant_min_ctas<D, BITS, MODE, HAD>())) q
                 issue(w + stride, reg ^ 1);
             }
         }
-        const bool landed = mbar_wait(&bar[reg], (phases >> reg) & 1, 1u << 24);
+        const bool landed = mbar_wait(&bar[reg], (phases >> reg) & 1, KVQ_WAIT_LIMIT(1u << 24));
         if (__syncthreads_or(!landed)) {
             if (t == 0) report_error(kErrTmaTimeout);
             break;
@@ -285,10 +285,48 @@ struct DequantArgs {
     float rsqd, sqd;
 };
 
-// One CTA = one block of one (batch, head); thread t rebuilds token t:
+// Token row rebuilt in fp32 from its code words w32 and parameters (tp: its
+// per-token fp16 values; sig, off: the block's channel scales and means as
+// fp32; sgn: the rotation's signs as fp32 sign-bit masks), in the oracle's
+// operation order:
 //   w = q * sigma; nsep x = n * w, or s (.) (H w * (n rsqd)) under HADAMARD;
 //   naive x = w; NSN x = s1 * (b + o) with b = w * (s2 sqd), or
 //   s (.) (H w * s2) under HADAMARD.
+template <int D, int BITS, int MODE, bool HAD>
+__device__ __forceinline__ void dequant_row(const uint32_t (&w32)[RowLayout<D, BITS>::kWords], const __half* tp,
+                                            const float* sig, const float* off, const uint32_t* sgn, float rsqd,
+                                            float sqd, float (&w)[D]) {
+    using L = RowLayout<D, BITS>;
+    const float tsig = (MODE == kNaive) ? __half2float(tp[0]) : 0.0f;
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+        const float q = (float)((int)code_at<D, BITS>(w32, c) - L::kOff);
+        w[c] = __fmul_rn(q, (MODE == kNaive) ? tsig : sig[c]);
+    }
+    if constexpr (HAD) fwht_reg<D>(w);
+    if constexpr (MODE == kNsn) {
+        const float s1 = __half2float(tp[0]), s2 = __half2float(tp[1]);
+        const float kb = HAD ? s2 : __fmul_rn(s2, sqd);
+#pragma unroll
+        for (int c = 0; c < D; ++c) {
+            float b = __fmul_rn(w[c], kb);
+            if (HAD) b = __uint_as_float(__float_as_uint(b) ^ sgn[c]);
+            w[c] = __fmul_rn(s1, __fadd_rn(b, off[c]));
+        }
+    } else if constexpr (MODE == kNsep) {
+        const float n = __half2float(tp[0]);
+        if constexpr (HAD) {
+            const float kd = __fmul_rn(n, rsqd);
+#pragma unroll
+            for (int c = 0; c < D; ++c) w[c] = __uint_as_float(__float_as_uint(__fmul_rn(w[c], kd)) ^ sgn[c]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < D; ++c) w[c] = __fmul_rn(n, w[c]);
+        }
+    }
+}
+
+// One CTA = one block of one (batch, head); thread t rebuilds token t.
 template <int D, int BITS, int MODE, bool HAD>
 __global__ void __launch_bounds__(128) dequantize_kernel(DequantArgs a) {
     using L = RowLayout<D, BITS>;
@@ -324,39 +362,121 @@ __global__ void __launch_bounds__(128) dequantize_kernel(DequantArgs a) {
     } else {
         load_words<L::kWords>(a.codes + tok_idx * L::kBytes, w32);
     }
-    const __half* tp = a.tok + tok_idx * ntk;
     float w[D];
-    const float tsig = (MODE == kNaive) ? __half2float(tp[0]) : 0.0f;
-#pragma unroll
-    for (int c = 0; c < D; ++c) {
-        const float q = (float)((int)code_at<D, BITS>(w32, c) - L::kOff);
-        w[c] = __fmul_rn(q, (MODE == kNaive) ? tsig : s_sig[c]);
-    }
-    if constexpr (HAD) fwht_reg<D>(w);
+    dequant_row<D, BITS, MODE, HAD>(w32, a.tok + tok_idx * ntk, s_sig, s_off, s_sgn, a.rsqd, a.sqd, w);
     float* o = a.out + ((size_t)bh * a.ntok + (size_t)blockIdx.x * kT + t) * D;
-    if constexpr (MODE == kNsn) {
-        const float s1 = __half2float(tp[0]), s2 = __half2float(tp[1]);
-        const float kb = HAD ? s2 : __fmul_rn(s2, a.sqd);
-#pragma unroll
-        for (int c = 0; c < D; ++c) {
-            float b = __fmul_rn(w[c], kb);
-            if (HAD) b = __uint_as_float(__float_as_uint(b) ^ s_sgn[c]);
-            w[c] = __fmul_rn(s1, __fadd_rn(b, s_off[c]));
-        }
-    } else if constexpr (MODE == kNsep) {
-        const float n = __half2float(tp[0]);
-        if constexpr (HAD) {
-            const float kd = __fmul_rn(n, a.rsqd);
-#pragma unroll
-            for (int c = 0; c < D; ++c) w[c] = __uint_as_float(__float_as_uint(__fmul_rn(w[c], kd)) ^ s_sgn[c]);
-        } else {
-#pragma unroll
-            for (int c = 0; c < D; ++c) w[c] = __fmul_rn(n, w[c]);
-        }
-    }
 #pragma unroll
     for (int k = 0; k < D / 4; ++k)
         reinterpret_cast<float4*>(o)[k] = make_float4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+}
+
+// ---------------------------------------------------------------- sign selection
+
+struct SelectArgs {
+    const __half* x;      // [n_blocks][128][D] the sample
+    const int8_t* signs;  // [n_cand][D] candidate sign vectors
+    double* part;         // [n_cand][n_blocks] error of each (candidate, block)
+    int n_blocks;
+    float rsqd, sqd;
+};
+
+// Pairwise (recursive halving) fp64 sum of the squared differences between
+// the rebuilt row w and the input row x over channels [OFF, OFF + N).
+template <int OFF, int N, int D>
+__device__ __forceinline__ double row_sq_err(const float (&w)[D], const __half* x) {
+    if constexpr (N == 1) {
+        const double df = __dsub_rn((double)w[OFF], (double)__half2float(x[OFF]));
+        return __dmul_rn(df, df);
+    } else {
+        return __dadd_rn(row_sq_err<OFF, N / 2, D>(w, x), row_sq_err<OFF + N / 2, N / 2, D>(w, x));
+    }
+}
+
+template <int D, int BITS, int MODE>
+__host__ __device__ constexpr int select_smem_bytes() {
+    // the quantizer's scratch, then the block's outputs and the per-row errors
+    return (quant_smem_bytes<D, MODE>() + 127) / 128 * 128 + kT * RowLayout<D, BITS>::kBytes + kT * 2 * 2 +
+           D * 2 * 2 + D * 4 * 3 + kT * 8;
+}
+
+// CTA (block b, candidate k): the block quantized with candidate k's signs
+// exactly as the quantize kernel does, rebuilt as dequantize does, and the
+// block's reconstruction error: per row the pairwise sum over channels of
+// (x_hat - x)^2 in fp64, over the rows the pairwise sum over tokens.
+template <int D, int BITS, int MODE>
+__global__ void __launch_bounds__(128) select_signs_kernel(SelectArgs a) {
+    using L = RowLayout<D, BITS>;
+    constexpr int ntk = (MODE == kNsn) ? 2 : 1;
+    const int t = threadIdx.x, blk = blockIdx.x, cand = blockIdx.y;
+    extern __shared__ uint8_t smem_raw[];
+    uint64_t* bar;
+    uint8_t* regions;
+    QuantSmem<D> sm = carve_quant_smem<D, MODE>(smem_raw, bar, regions);
+    uint8_t* p = smem_raw + (quant_smem_bytes<D, MODE>() + 127) / 128 * 128;
+    uint8_t* s_codes = p;                                    p += kT * L::kBytes;
+    __half* s_tok = reinterpret_cast<__half*>(p);            p += kT * 2 * 2;
+    __half* s_chan = reinterpret_cast<__half*>(p);           p += D * 2;
+    __half* s_off16 = reinterpret_cast<__half*>(p);          p += D * 2;
+    float* s_sig = reinterpret_cast<float*>(p);              p += D * 4;
+    float* s_off = reinterpret_cast<float*>(p);              p += D * 4;
+    uint32_t* s_sgn = reinterpret_cast<uint32_t*>(p);        p += D * 4;
+    double* s_err = reinterpret_cast<double*>(p);
+    const int8_t* sg = a.signs + (size_t)cand * D;
+    if (t < D / 2) sm.sgn2[t] = (sg[2 * t] < 0 ? 0x8000u : 0u) | (sg[2 * t + 1] < 0 ? 0x80000000u : 0u);
+    if (t < D) s_sgn[t] = sg[t] < 0 ? 0x80000000u : 0u;
+    __syncthreads();
+    const __half* xr = a.x + ((size_t)blk * kT + t) * D;
+    uint4 raw[D / 8];
+#pragma unroll
+    for (int q = 0; q < D / 8; ++q) raw[q] = reinterpret_cast<const uint4*>(xr)[q];
+    QuantOut out;
+    out.codes = s_codes;
+    out.stage = nullptr;
+    out.tok = s_tok;
+    out.chan = s_chan;
+    out.off = s_off16;
+    out.pairv = false;
+    auto none = [] {};
+    quantize_rows<D, BITS, MODE, true, true>(raw, t, sm, out, a.rsqd, a.sqd, none, none);
+    __syncthreads();
+    if (t < D) {
+        s_sig[t] = __half2float(s_chan[t]);
+        s_off[t] = (MODE == kNsn) ? __half2float(s_off16[t]) : 0.0f;
+    }
+    __syncthreads();
+    uint32_t w32[L::kWords];
+    load_words<L::kWords>(s_codes + (size_t)t * L::kBytes, w32);
+    float w[D];
+    dequant_row<D, BITS, MODE, true>(w32, s_tok + t * ntk, s_sig, s_off, s_sgn, a.rsqd, a.sqd, w);
+    s_err[t] = row_sq_err<0, D, D>(w, xr);
+    __syncthreads();
+#pragma unroll
+    for (int h = 1; h < kT; h *= 2) {
+        if ((t & (2 * h - 1)) == 0) s_err[t] = __dadd_rn(s_err[t], s_err[t + h]);
+        __syncthreads();
+    }
+    if (t == 0) a.part[(size_t)cand * a.n_blocks + blk] = s_err[0];
+}
+
+// Errors of the candidates (their blocks added in order) and the index of
+// the smallest one (the lowest index among equal ones).
+__global__ void __launch_bounds__(256) select_reduce_kernel(const double* part, int n_blocks, int n_cand,
+                                                            double* err, int* best) {
+    __shared__ double s_e[256];
+    const int k = threadIdx.x;
+    if (k < n_cand) {
+        double e = 0.0;
+        for (int b = 0; b < n_blocks; ++b) e = __dadd_rn(e, part[(size_t)k * n_blocks + b]);
+        err[k] = e;
+        s_e[k] = e;
+    }
+    __syncthreads();
+    if (k == 0) {
+        int bi = 0;
+        for (int j = 1; j < n_cand; ++j)
+            if (s_e[j] < s_e[bi]) bi = j;
+        *best = bi;
+    }
 }
 
 }  // namespace kvq

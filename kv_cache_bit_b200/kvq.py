@@ -23,7 +23,7 @@ BLOCK_TOKENS = 128
 
 EXPORTS = ["kvq_row_bytes", "kvq_tok_params", "kvq_make_signs", "kvq_quantize_block", "kvq_append_token",
            "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_dequantize",
-           "kvq_read_device_errors",
+           "kvq_select_signs_workspace_bytes", "kvq_select_signs", "kvq_read_device_errors",
            "kvq_status_string"]
 
 
@@ -66,6 +66,11 @@ def _load():
     L.kvq_dequantize.restype = ctypes.c_int
     L.kvq_dequantize.argtypes = [ctypes.POINTER(kvq_config), ctypes.POINTER(kvq_cache), ctypes.c_int32,
                                  ctypes.c_int64, ctypes.c_int64, P, P]
+    L.kvq_select_signs_workspace_bytes.restype = ctypes.c_size_t
+    L.kvq_select_signs_workspace_bytes.argtypes = [ctypes.c_int32, ctypes.c_int64]
+    L.kvq_select_signs.restype = ctypes.c_int
+    L.kvq_select_signs.argtypes = [ctypes.POINTER(kvq_config), P, ctypes.c_int64, P, ctypes.c_int32, P, P, P,
+                                   ctypes.c_size_t, P]
     L.kvq_read_device_errors.restype = ctypes.c_int
     L.kvq_read_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
     L.kvq_status_string.restype = ctypes.c_char_p
@@ -154,6 +159,22 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 def kvq_dequantize(cfg: "Config", cache: "KVCache", tensor: int, t0: int, ntok: int, out, stream=None):
     _check(lib.kvq_dequantize(ctypes.byref(cfg.c), ctypes.byref(cache.c), tensor, t0, ntok, _ptr(out),
                               _stream(stream)), "kvq_dequantize")
+
+
+SELECT_MAX_CANDIDATES = 256
+
+
+def kvq_select_signs_workspace_bytes(n_cand: int, n_blocks: int) -> int:
+    return lib.kvq_select_signs_workspace_bytes(n_cand, n_blocks)
+
+
+def kvq_select_signs(cfg: "Config", x, n_blocks: int, signs, n_cand: int, err, best, ws, ws_bytes: int,
+                     stream=None):
+    """Sign-pattern selection (see include/kvq.h): x fp16 [n_blocks, 128,
+    head_dim], signs int8 [n_cand, head_dim], err float64 [n_cand] and best
+    int32 [1] outputs, all device tensors."""
+    _check(lib.kvq_select_signs(ctypes.byref(cfg.c), _ptr(x), n_blocks, _ptr(signs), n_cand, _ptr(err), _ptr(best),
+                                _ptr(ws), ws_bytes, _stream(stream)), "kvq_select_signs")
 
 
 def kvq_read_device_errors(clear: bool = True) -> int:

@@ -62,6 +62,8 @@ def lib():
         L.ko_dequantize_slice.argtypes = [_P, _P, _P, _P, _P, ctypes.c_long, ctypes.c_long, _P]
         L.ko_attention_f64.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_long, _P, _P, _P,
                                        ctypes.c_double, _P]
+        L.ko_select_signs.restype = ctypes.c_int
+        L.ko_select_signs.argtypes = [_P, _P, ctypes.c_long, _P, ctypes.c_int, _P]
         _lib = L
     return _lib
 
@@ -318,6 +320,21 @@ def cache_attention(cfg: Cfg, q16, cache_k, cache_v, resid_k16, resid_v16, lengt
     k = cache_tokens(cfg, cache_k, resid_k16, length, threads)
     v = cache_tokens(cfg, cache_v, resid_v16, length, threads)
     return attention(q16, k, v, scale, threads)
+
+
+def select_signs(cfg: Cfg, x16: np.ndarray, signs: np.ndarray):
+    """Sign-pattern selection for the randomized Hadamard rotation: x16 the
+    sample as whole blocks (fp16 bits [n_blocks, 128, d]), signs [n_cand, d]
+    of +-1.  Returns (index of the smallest reconstruction error, errors
+    float64 [n_cand]); cfg.signs is ignored."""
+    x16 = np.ascontiguousarray(x16, dtype=np.uint16)
+    signs = np.ascontiguousarray(signs, dtype=np.int8)
+    nb, t, d = x16.shape
+    assert t == T and d == cfg.d and signs.shape[1] == d
+    err = np.empty(signs.shape[0], np.float64)
+    c = Cfg(cfg.d, cfg.bits, cfg.flags, None).c()
+    best = lib().ko_select_signs(ctypes.byref(c), _ptr(x16), nb, _ptr(signs), signs.shape[0], _ptr(err))
+    return int(best), err
 
 
 def default_threads() -> int:

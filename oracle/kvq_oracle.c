@@ -418,6 +418,59 @@ int ko_dequantize_slice(const ko_cfg* cfg, const uint8_t* codes, const uint16_t*
 }
 
 /* ------------------------------------------------------------------ */
+/* Sign-pattern selection for the randomized Hadamard rotation [P4]:   */
+/* quantize a sample with each candidate sign vector and keep the one  */
+/* whose reconstruction error is smallest.                             */
+/*   x      [n_blocks][T][d] fp16 bits: the sample, whole blocks       */
+/*   signs  [n_cand][d] of +-1: the candidate sign vectors             */
+/*   err    [n_cand] out: sum over the sample of (x_hat - x)^2 in fp64  */
+/* The error of a block is the pairwise (recursive halving) sum over   */
+/* its tokens of the pairwise sum over channels of the squared         */
+/* differences; the blocks are added in order.  Returns the index of   */
+/* the smallest error (the lowest index among equal ones).             */
+/* ------------------------------------------------------------------ */
+static double ko_pairwise_sum_f64(const double* v, long n)
+{
+    if (n == 1) return v[0];
+    long h = n / 2;
+    return ko_pairwise_sum_f64(v, h) + ko_pairwise_sum_f64(v + h, h);
+}
+
+int ko_select_signs(const ko_cfg* cfg, const uint16_t* x, long n_blocks, const int8_t* signs, int n_cand,
+                    double* err)
+{
+    const int d = cfg->d, T = KO_T, rb = ko_row_bytes(d, cfg->bits), nt = ko_ntok(cfg->flags);
+    uint8_t* codes = (uint8_t*)malloc((size_t)T * rb);
+    uint16_t* tok = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)T * (nt > 0 ? nt : 1));
+    uint16_t chan[1024], off[1024];
+    float* xh = (float*)malloc(sizeof(float) * (size_t)T * d);
+    double sq[1024], rowe[KO_T];
+    int best = 0;
+    for (int k = 0; k < n_cand; k++) {
+        ko_cfg c = *cfg;
+        c.signs = signs + (size_t)k * d;
+        double e = 0.0;
+        for (long b = 0; b < n_blocks; b++) {
+            const uint16_t* xb = x + (size_t)b * T * d;
+            ko_quantize_block(&c, xb, codes, tok, chan, off);
+            ko_dequantize_block(&c, codes, tok, chan, off, xh);
+            for (int t = 0; t < T; t++) {
+                for (int ch = 0; ch < d; ch++) {
+                    double df = (double)xh[t * d + ch] - (double)ko_f16_to_f32(xb[t * d + ch]);
+                    sq[ch] = df * df;
+                }
+                rowe[t] = ko_pairwise_sum_f64(sq, d);
+            }
+            e = e + ko_pairwise_sum_f64(rowe, T);
+        }
+        err[k] = e;
+        if (e < err[best]) best = k;
+    }
+    free(codes); free(tok); free(xh);
+    return best;
+}
+
+/* ------------------------------------------------------------------ */
 /* Softmax attention of g query heads over L cached tokens, in fp64,   */
 /* brute force: out_j = sum_t softmax_t(scale * q_j . k_t) v_t.        */
 /*   q [g][d] fp16 bits; k, v [L][d] fp32; out [g][d] fp64.            */

@@ -135,3 +135,25 @@ def test_host_side_rejections(kvq):
     # failed checks leave len untouched
     assert held.len == 130 and full.len == 256
     assert kvq.lib.kvq_status_string(kvq.KVQ_ERR_CAPACITY) == b"cache capacity exceeded"
+
+
+def test_select_signs_host_checks(kvq):
+    a = 1 << 20  # placeholder, 16-byte aligned, never dereferenced: every call below fails a host check
+    L = kvq.lib
+    assert L.kvq_select_signs_workspace_bytes(8, 10) == 8 * 10 * 8
+    assert L.kvq_select_signs_workspace_bytes(0, 10) == 0
+    assert L.kvq_select_signs_workspace_bytes(kvq.SELECT_MAX_CANDIDATES + 1, 10) == 0
+    had = _cfg(kvq, flags=kvq.NORM_SEP | kvq.PER_CHANNEL | kvq.HADAMARD)
+    nsn = _cfg(kvq, flags=kvq.NSN | kvq.PER_CHANNEL | kvq.HADAMARD)
+    plain = _cfg(kvq, flags=kvq.NORM_SEP | kvq.PER_CHANNEL)
+    args = lambda cfg, x=a, nb=4, s=a, nc=2, ws=a, wsb=64: L.kvq_select_signs(
+        ctypes.byref(cfg), x, nb, s, nc, a, a, ws, wsb, None)
+    assert args(plain) == kvq.KVQ_ERR_UNSUPPORTED
+    assert args(_cfg(kvq, flags=0)) == kvq.KVQ_ERR_UNSUPPORTED
+    assert args(had, x=None) == kvq.KVQ_ERR_INVALID_ARG
+    assert args(had, x=a + 4) == kvq.KVQ_ERR_INVALID_ARG
+    assert args(nsn, s=None) == kvq.KVQ_ERR_INVALID_ARG
+    assert args(had, nc=0) == kvq.KVQ_ERR_INVALID_ARG
+    assert args(had, nb=0) == kvq.KVQ_ERR_INVALID_ARG
+    assert args(had, ws=None) == kvq.KVQ_ERR_WORKSPACE
+    assert args(had, wsb=63) == kvq.KVQ_ERR_WORKSPACE
