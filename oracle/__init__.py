@@ -26,7 +26,7 @@ import numpy as np
 
 from . import build as _build
 
-NORM_SEP, PER_CHANNEL, NSN, HADAMARD = 1, 2, 4, 8
+NORM_SEP, PER_CHANNEL, NSN, HADAMARD, DQ = 1, 2, 4, 8, 16
 T = 128
 
 _lib = None
@@ -62,6 +62,9 @@ def lib():
         L.ko_dequantize_slice.argtypes = [_P, _P, _P, _P, _P, ctypes.c_long, ctypes.c_long, _P]
         L.ko_attention_f64.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_long, _P, _P, _P,
                                        ctypes.c_double, _P]
+        L.ko_dq_record_bytes.argtypes = [ctypes.c_int]
+        L.ko_off_words.argtypes = [ctypes.c_uint, ctypes.c_int]
+        L.ko_dq_decode.argtypes = [_P, ctypes.c_int, _P, _P]
         L.ko_select_signs.restype = ctypes.c_int
         L.ko_select_signs.argtypes = [_P, _P, ctypes.c_long, _P, ctypes.c_int, _P]
         _lib = L
@@ -127,6 +130,25 @@ def ntok(flags: int) -> int:
     return lib().ko_ntok(flags)
 
 
+def off_words(flags: int, d: int) -> int:
+    """fp16 words per block of the NSN offsets array: d means, or under DQ
+    the block's side-parameter record (its bytes / 2)."""
+    return lib().ko_off_words(flags, d)
+
+
+def dq_record_bytes(d: int) -> int:
+    return lib().ko_dq_record_bytes(d)
+
+
+def dq_decode(rec: np.ndarray, d: int):
+    """(o_hat float32 [d], s1_hat float32 [128]) of one DQ record."""
+    rec = np.ascontiguousarray(rec).view(np.uint8)
+    o = np.empty(d, np.float32)
+    s1 = np.empty(T, np.float32)
+    lib().ko_dq_decode(_ptr(rec), d, _ptr(o), _ptr(s1))
+    return o, s1
+
+
 def splitmix64(seed: int, n: int) -> list:
     st = ctypes.c_uint64(seed)
     return [lib().ko_splitmix64_next(ctypes.byref(st)) for _ in range(n)]
@@ -185,7 +207,7 @@ def empty_cache(cfg: Cfg, B: int, H: int, S_max: int) -> dict:
         "codes": np.zeros((B, H, S_max, row_bytes(cfg.d, cfg.bits)), np.uint8),
         "tok": np.zeros((B, H, S_max, nt), np.uint16) if nt else None,
         "chan": np.zeros((B, H, nb, cfg.d), np.uint16) if cfg.flags & PER_CHANNEL else None,
-        "off": np.zeros((B, H, nb, cfg.d), np.uint16) if cfg.flags & NSN else None,
+        "off": np.zeros((B, H, nb, off_words(cfg.flags, cfg.d)), np.uint16) if cfg.flags & NSN else None,
     }
 
 

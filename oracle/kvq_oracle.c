@@ -47,7 +47,7 @@
 
 #define KO_T 128 /* tokens per scale block */
 
-enum { KO_NORM_SEP = 1, KO_PER_CHANNEL = 2, KO_NSN = 4, KO_HADAMARD = 8 };
+enum { KO_NORM_SEP = 1, KO_PER_CHANNEL = 2, KO_NSN = 4, KO_HADAMARD = 8, KO_DQ = 16 };
 
 typedef struct {
     int d;               /* head dim: power of two, 2..1024 */
@@ -158,7 +158,7 @@ int ko_row_bytes(int d, int bits) { return bits <= 4 ? d * bits / 8 : d; }
 int ko_ntok(unsigned flags)
 {
     int n;
-    if (flags & KO_NSN) n = 2;                      /* s1, s2 */
+    if (flags & KO_NSN) n = (flags & KO_DQ) ? 1 : 2; /* s1, s2 (under DQ s1 is in the block record) */
     else n = (flags & KO_NORM_SEP) ? 1 : 0;         /* norm */
     if (!(flags & KO_PER_CHANNEL)) n += 1;          /* token scale, last */
     return n;
@@ -195,6 +195,85 @@ int ko_unpack_row(const uint8_t* in, int d, int bits, int8_t* q)
         q[c] = (int8_t)((int)e - off);
     }
     return bad;
+}
+
+/* ------------------------------------------------------------------ */
+/* Double quantization of the NSN side parameters [P3 "Double          */
+/* Quantization (DQ)": the mean o and the scale s1 are themselves      */
+/* quantized to 4 bits].  Per block of T tokens, one byte record:      */
+/*   [0, d/2)            o codes: e = q + 8, channel 2j in the low      */
+/*                       nibble of byte j (the INT4 layout)             */
+/*   [d/2, d/2 + T/2)    s1 codes: q in 0..15, token 2j in the low      */
+/*                       nibble of byte j                               */
+/*   then fp16 sigma_o, lo, step; zero padding to a multiple of 16.     */
+/* o: symmetric, sigma_o = fp16(max|o| / 7), q = clamp(rne(o / sigma_o),*/
+/*    -7, 7), o_hat = q * sigma_o.                                      */
+/* s1 (positive): over [lo, lo + 15 step] with lo = fp16(min s1),       */
+/*    step = fp16(max(max s1 - lo, 0) / 15), q = clamp(rne((s1 - lo) /  */
+/*    step), 0, 15), s1_hat = lo + q * step.                            */
+/* ------------------------------------------------------------------ */
+int ko_dq_record_bytes(int d) { return (d / 2 + KO_T / 2 + 6 + 15) / 16 * 16; }
+
+/* fp16 words per block of the NSN offsets array: d means, or the record. */
+int ko_off_words(unsigned flags, int d) { return (flags & KO_DQ) ? ko_dq_record_bytes(d) / 2 : d; }
+
+static int ko_code_range(double y, int lo, int hi)
+{
+    double r = nearbyint(y);
+    if (r > hi) r = hi;
+    if (r < lo) r = lo;
+    return (int)r;
+}
+
+static void ko_dq_encode(const float* o, const float* s1, int d, uint8_t* rec, float* ohat)
+{
+    const int T = KO_T, rb = ko_dq_record_bytes(d);
+    memset(rec, 0, (size_t)rb);
+    float m = 0.0f;
+    for (int c = 0; c < d; c++) if (fabsf(o[c]) > m) m = fabsf(o[c]);
+    uint16_t so = ko_f32_to_f16(m / 7.0f);
+    float sof = ko_f16_to_f32(so);
+    float invo = sof > 0.0f ? 1.0f / sof : 0.0f;
+    for (int c = 0; c < d; c++) {
+        int q = ko_code_range((double)o[c] * (double)invo, -7, 7);
+        rec[c / 2] |= (uint8_t)((unsigned)(q + 8) << (4 * (c % 2)));
+        ohat[c] = (float)q * sof;
+    }
+    float mn = s1[0], mx = s1[0];
+    for (int t = 1; t < T; t++) { if (s1[t] < mn) mn = s1[t]; if (s1[t] > mx) mx = s1[t]; }
+    uint16_t lo16 = ko_f32_to_f16(mn);
+    float lo = ko_f16_to_f32(lo16);
+    float span = mx - lo;
+    if (span < 0.0f) span = 0.0f;
+    uint16_t st16 = ko_f32_to_f16(span / 15.0f);
+    float st = ko_f16_to_f32(st16);
+    float invs = st > 0.0f ? 1.0f / st : 0.0f;
+    for (int t = 0; t < T; t++) {
+        int q = ko_code_range((double)(s1[t] - lo) * (double)invs, 0, 15);
+        rec[d / 2 + t / 2] |= (uint8_t)((unsigned)q << (4 * (t % 2)));
+    }
+    memcpy(rec + d / 2 + T / 2, &so, 2);
+    memcpy(rec + d / 2 + T / 2 + 2, &lo16, 2);
+    memcpy(rec + d / 2 + T / 2 + 4, &st16, 2);
+}
+
+/* o_hat [d] and s1_hat [T] from a record. */
+void ko_dq_decode(const uint8_t* rec, int d, float* ohat, float* s1hat)
+{
+    const int T = KO_T;
+    uint16_t so, lo16, st16;
+    memcpy(&so, rec + d / 2 + T / 2, 2);
+    memcpy(&lo16, rec + d / 2 + T / 2 + 2, 2);
+    memcpy(&st16, rec + d / 2 + T / 2 + 4, 2);
+    float sof = ko_f16_to_f32(so), lo = ko_f16_to_f32(lo16), st = ko_f16_to_f32(st16);
+    for (int c = 0; c < d; c++) {
+        int q = (int)((rec[c / 2] >> (4 * (c % 2))) & 15u) - 8;
+        ohat[c] = (float)q * sof;
+    }
+    for (int t = 0; t < T; t++) {
+        int q = (int)((rec[d / 2 + t / 2] >> (4 * (t % 2))) & 15u);
+        s1hat[t] = lo + (float)q * st;
+    }
 }
 
 /* nearest integer to the exact product u * inv (both fp32, so the product is
@@ -237,25 +316,35 @@ static void ko_quantize_block_impl(const ko_cfg* cfg, const uint16_t* x, uint8_t
         for (int c = 0; c < d; c++) w[t * d + c] = ko_f16_to_f32(x[t * d + c]);
 
     if (fl & KO_NSN) {
+        const int dq = (fl & KO_DQ) != 0;
+        float s1v[KO_T], of[1024], oh[1024];
         /* [P3] Normalize: token norm -> sqrt(d); s1 = ||x|| / sqrt(d). */
         for (int t = 0; t < T; t++) {
             float* r = w + t * d;
             float n1 = ko_l2(r, d);
-            tok[t * ntok + 0] = ko_f32_to_f16(n1 * RSQD);
+            s1v[t] = n1 * RSQD;
+            if (!dq) tok[t * ntok + 0] = ko_f32_to_f16(s1v[t]);
             float r1 = n1 > 0.0f ? SQD / n1 : 0.0f;
             for (int c = 0; c < d; c++) r[c] = r[c] * r1;
         }
-        /* [P3] Shift: subtract the per-channel mean over the block. */
-        for (int c = 0; c < d; c++) {
-            float o = ko_pairwise_sum(w + c, T, d) * (1.0f / (float)T);
-            off[c] = ko_f32_to_f16(o);
+        /* [P3] Shift: subtract the per-channel mean over the block.  The
+           encoder subtracts the mean the decoder will add back: the stored
+           fp16 one, or under DQ its 4-bit reconstruction. */
+        for (int c = 0; c < d; c++) of[c] = ko_pairwise_sum(w + c, T, d) * (1.0f / (float)T);
+        if (dq) {
+            ko_dq_encode(of, s1v, d, (uint8_t*)off, oh);
+        } else {
+            for (int c = 0; c < d; c++) {
+                off[c] = ko_f32_to_f16(of[c]);
+                oh[c] = ko_f16_to_f32(off[c]);
+            }
         }
         /* [P3] Normalize again: s2 = ||b|| / sqrt(d). */
         for (int t = 0; t < T; t++) {
             float* r = w + t * d;
-            for (int c = 0; c < d; c++) r[c] = r[c] - ko_f16_to_f32(off[c]);
+            for (int c = 0; c < d; c++) r[c] = r[c] - oh[c];
             float n2 = ko_l2(r, d);
-            tok[t * ntok + 1] = ko_f32_to_f16(n2 * RSQD);
+            tok[t * ntok + (dq ? 0 : 1)] = ko_f32_to_f16(n2 * RSQD);
             ks[t] = n2 > 0.0f ? c0 / n2 : 0.0f;
         }
     } else if (fl & KO_NORM_SEP) {
@@ -333,8 +422,12 @@ int ko_dequantize_block(const ko_cfg* cfg, const uint8_t* codes, const uint16_t*
     const float RSQD = (float)(1.0 / sqrt((double)d));
     const float SQD = (float)sqrt((double)d);
     int8_t q[1024];
-    float w[1024];
+    float w[1024], ohat[1024], s1hat[KO_T];
     int bad = 0;
+    const int dq = (fl & KO_NSN) && (fl & KO_DQ);
+    if (dq) ko_dq_decode((const uint8_t*)off, d, ohat, s1hat);
+    else if (fl & KO_NSN)
+        for (int c = 0; c < d; c++) ohat[c] = ko_f16_to_f32(off[c]);
     for (int t = 0; t < T; t++) {
         bad += ko_unpack_row(codes + (size_t)t * rb, d, cfg->bits, q);
         for (int c = 0; c < d; c++) {
@@ -346,13 +439,13 @@ int ko_dequantize_block(const ko_cfg* cfg, const uint8_t* codes, const uint16_t*
         int had = (fl & KO_HADAMARD) != 0;
         if (had) ko_fwht(w, d);
         if (fl & KO_NSN) {
-            float s1 = ko_f16_to_f32(tok[t * ntok + 0]);
-            float s2 = ko_f16_to_f32(tok[t * ntok + 1]);
+            float s1 = dq ? s1hat[t] : ko_f16_to_f32(tok[t * ntok + 0]);
+            float s2 = ko_f16_to_f32(tok[t * ntok + (dq ? 0 : 1)]);
             float kb = had ? s2 : s2 * SQD;
             for (int c = 0; c < d; c++) {
                 float b = w[c] * kb;
                 if (had && cfg->signs && cfg->signs[c] < 0) b = -b;
-                o[c] = s1 * (b + ko_f16_to_f32(off[c]));
+                o[c] = s1 * (b + ohat[c]);
             }
         } else if (fl & KO_NORM_SEP) {
             float n = ko_f16_to_f32(tok[t * ntok + 0]);
@@ -391,7 +484,7 @@ void ko_quantize_slice_y(const ko_cfg* cfg, const uint16_t* x, long t0, long nto
         ko_quantize_block_impl(cfg, x + (size_t)t * d, codes + (size_t)tb * rb,
                                tok ? tok + (size_t)tb * nt : NULL,
                                chan ? chan + (size_t)blk * d : NULL,
-                               off ? off + (size_t)blk * d : NULL,
+                               off ? off + (size_t)blk * ko_off_words(cfg->flags, d) : NULL,
                                y ? y + (size_t)t * d : NULL);
     }
 }
@@ -412,7 +505,7 @@ int ko_dequantize_slice(const ko_cfg* cfg, const uint8_t* codes, const uint16_t*
         bad += ko_dequantize_block(cfg, codes + (size_t)tb * rb,
                                    tok ? tok + (size_t)tb * nt : NULL,
                                    chan ? chan + (size_t)blk * d : NULL,
-                                   off ? off + (size_t)blk * d : NULL, out + (size_t)t * d);
+                                   off ? off + (size_t)blk * ko_off_words(cfg->flags, d) : NULL, out + (size_t)t * d);
     }
     return bad;
 }
