@@ -81,7 +81,7 @@ def measured_peak_gbs():
 
 def flags_of(mode: str) -> int:
     names, _ = synth.MODES[mode]
-    m = {"NORM_SEP": 1, "PER_CHANNEL": 2, "NSN": 4, "HADAMARD": 8}
+    m = {"NORM_SEP": 1, "PER_CHANNEL": 2, "NSN": 4, "HADAMARD": 8, "DQ": 16}
     f = 0
     for n in names:
         f |= m[n]

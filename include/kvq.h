@@ -62,7 +62,8 @@ enum {
     KVQ_NORM_SEP = 1u,    /* split off the FP16 L2 norm; quantize the unit direction */
     KVQ_PER_CHANNEL = 2u, /* per-channel scale over each 128-token block (else per token) */
     KVQ_NSN = 4u,         /* Normalize-Shift-Normalize before quantization */
-    KVQ_HADAMARD = 8u     /* (randomized) Hadamard rotation of the direction */
+    KVQ_HADAMARD = 8u,    /* (randomized) Hadamard rotation of the direction */
+    KVQ_DQ = 16u          /* NSN only: double quantization of the side parameters o, s1 */
 };
 
 #define KVQ_BLOCK_TOKENS 128
@@ -73,7 +74,14 @@ enum {
  *   NORM_SEP | PER_CHANNEL | HADAMARD randomized Hadamard, then nsep+pchan
  *   0                                  naive per-token absmax
  *   NSN | PER_CHANNEL [| HADAMARD]     NSN (+ Hadamard), per-channel codes
+ *   NSN | PER_CHANNEL [| HADAMARD] | DQ   the same with double quantization
  * head_dim in {64, 128}; bits in {2, 3, 4}.
+ * DQ (NSNQuant explainer, "Double Quantization (DQ)": the NSN parameters o
+ * and s1 are themselves quantized to 4 bits): per 128-token block the means
+ * o get symmetric 4-bit codes with one fp16 scale sigma_o = fp16(max|o|/7),
+ * and the token scales s1 unsigned 4-bit codes over [lo, lo + 15 step] with
+ * lo = fp16(min s1), step = fp16((max s1 - lo) / 15); the encoder subtracts
+ * the rebuilt means.  Both go to a block record in off[] (layout below).
  */
 typedef struct {
     int32_t head_dim;
@@ -90,9 +98,16 @@ typedef struct {
  * Shapes (row-major, B = batch, H = kv_heads, S = capacity, nb = S / 128):
  *   codes[i] uint8  [B][H][S][row_bytes]   row_bytes = kvq_row_bytes(head_dim, bits)
  *   tok[i]   fp16   [B][H][S][ntok]        ntok = kvq_tok_params(flags):
- *                                          nsep: norm; naive: scale; NSN: s1, s2
+ *                                          nsep: norm; naive: scale; NSN: s1, s2;
+ *                                          NSN with DQ: s2
  *   chan[i]  fp16   [B][H][nb][head_dim]   per-channel block scale (PER_CHANNEL, else NULL)
- *   off[i]   fp16   [B][H][nb][head_dim]   NSN per-channel block mean (NSN, else NULL)
+ *   off[i]   fp16   [B][H][nb][kvq_off_words(flags, head_dim)]   (NSN, else NULL):
+ *            the per-channel block means, or under DQ the block record:
+ *            bytes [0, head_dim/2) the codes of o (e = q + 8, channel 2j in
+ *            the low nibble of byte j), [head_dim/2, head_dim/2 + 64) the
+ *            codes of s1 (q in 0..15, token 2j in the low nibble of byte j),
+ *            then fp16 sigma_o, lo, step, zeros up to a multiple of 16 bytes;
+ *            o_hat = (e - 8) sigma_o, s1_hat = lo + q step
  *   resid[i] fp16   [B][H][128][head_dim]  residual tokens not yet quantized
  * Code layout per token row: offset-binary e = q + 2^(bits-1) (never 0);
  *   INT4 byte j = e[2j] | e[2j+1] << 4; INT2 byte j = e[4j] | e[4j+1] << 2 |
@@ -127,6 +142,11 @@ int32_t kvq_row_bytes(int32_t head_dim, int32_t bits);
 /* fp16 per-token parameters stored for a flag set (ntok above); -1 if the
    flag set is not built for the GPU. */
 int32_t kvq_tok_params(uint32_t flags);
+
+/* fp16 words per block of the off[] arrays for a flag set and head_dim: the
+   head_dim means, or under DQ the record's bytes / 2; 0 without NSN; -1 if
+   the flag set or head_dim is not built for the GPU. */
+int32_t kvq_off_words(uint32_t flags, int32_t head_dim);
 
 /*
  * Random signs of the randomized Hadamard rotation ("random sign patterns",

@@ -3,7 +3,8 @@ through HBM at minimum), used for GB/s and roofline fractions.
 
 Per quantized token and tensor: row_bytes codes + 2 * ntok bytes of fp16
 per-token parameters + 2 * d / 128 bytes of per-block channel scales (and as
-much again for NSN channel means); residual tokens cost 2 * d bytes.
+much again for NSN channel means, or under DQ the block record's bytes /
+128); residual tokens cost 2 * d bytes.
 """
 from __future__ import annotations
 
@@ -14,13 +15,25 @@ def row_bytes(d: int, bits: int) -> int:
     return d * bits // 8
 
 
+NSN, DQ = 4, 16
+
+
 def ntok(flags: int) -> int:
-    return 2 if flags & 4 else 1
+    return (1 if flags & DQ else 2) if flags & NSN else 1
+
+
+def dq_record_bytes(d: int) -> int:
+    """Block record of the double-quantized NSN parameters: 4-bit codes of the
+    d means and of the 128 s1, three fp16 values, padding to 16 bytes."""
+    return (d // 2 + T // 2 + 6 + 15) // 16 * 16
 
 
 def token_bytes(d: int, bits: int, flags: int) -> float:
     """Bytes of one quantized token of one tensor, block parameters amortized."""
-    per_block = (2 * d if flags & 2 else 0) + (2 * d if flags & 4 else 0)
+    side = 0
+    if flags & NSN:
+        side = dq_record_bytes(d) if flags & DQ else 2 * d
+    per_block = (2 * d if flags & 2 else 0) + side
     return row_bytes(d, bits) + 2 * ntok(flags) + per_block / T
 
 

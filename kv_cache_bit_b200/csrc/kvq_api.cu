@@ -34,7 +34,14 @@ ModeInfo mode_of(uint32_t flags) {
     if (base == (KVQ_NORM_SEP | KVQ_PER_CHANNEL)) m.mode = kNsep;
     else if (flags == 0) m.mode = kNaive;
     else if (base == (KVQ_NSN | KVQ_PER_CHANNEL)) m.mode = kNsn;
+    else if (base == (KVQ_NSN | KVQ_PER_CHANNEL | KVQ_DQ)) m.mode = kNsnDq;
     return m;
+}
+
+int off_words_of(int mode, int d) {
+    if (!is_nsn(mode)) return 0;
+    if (mode == kNsn) return d;
+    return d == 64 ? off_words<64, kNsnDq>() : off_words<128, kNsnDq>();
 }
 
 int row_bytes(int d, int bits) {
@@ -63,7 +70,7 @@ kvq_status check_cache(const kvq_config* cfg, const ModeInfo& mi, const kvq_cach
     for (int i = 0; i < 2; ++i) {
         if (!ok_ptr(c->codes[i]) || !ok_ptr(c->tok[i]) || !ok_ptr(c->resid[i])) return KVQ_ERR_INVALID_ARG;
         if (mi.mode != kNaive && !ok_ptr(c->chan[i])) return KVQ_ERR_INVALID_ARG;
-        if (mi.mode == kNsn && !ok_ptr(c->off[i])) return KVQ_ERR_INVALID_ARG;
+        if (is_nsn(mi.mode) && !ok_ptr(c->off[i])) return KVQ_ERR_INVALID_ARG;
     }
     return KVQ_OK;
 }
@@ -81,6 +88,7 @@ template <int D, int BITS, typename Fn>
 kvq_status dispatch_mode(const ModeInfo& mi, Fn& fn) {
     if (mi.mode == kNsep) return mi.had ? fn.template run<D, BITS, kNsep, true>() : fn.template run<D, BITS, kNsep, false>();
     if (mi.mode == kNaive) return mi.had ? KVQ_ERR_UNSUPPORTED : fn.template run<D, BITS, kNaive, false>();
+    if (mi.mode == kNsnDq) return mi.had ? fn.template run<D, BITS, kNsnDq, true>() : fn.template run<D, BITS, kNsnDq, false>();
     return mi.had ? fn.template run<D, BITS, kNsn, true>() : fn.template run<D, BITS, kNsn, false>();
 }
 
@@ -357,7 +365,13 @@ int32_t kvq_row_bytes(int32_t head_dim, int32_t bits) { return row_bytes(head_di
 int32_t kvq_tok_params(uint32_t flags) {
     const ModeInfo mi = mode_of(flags);
     if (mi.mode < 0 || (mi.mode == kNaive && mi.had)) return -1;
-    return mi.mode == kNsn ? 2 : 1;
+    return tok_params(mi.mode);
+}
+
+int32_t kvq_off_words(uint32_t flags, int32_t head_dim) {
+    const ModeInfo mi = mode_of(flags);
+    if (mi.mode < 0 || (mi.mode == kNaive && mi.had) || (head_dim != 64 && head_dim != 128)) return -1;
+    return off_words_of(mi.mode, head_dim);
 }
 
 kvq_status kvq_make_signs(uint64_t seed, int32_t head_dim, int8_t* host_out) {

@@ -324,18 +324,42 @@ constexpr int kMaxCTAs = 4 * 148;  // cap of the persistent grid
 // A unit is one tensor's half block: packed codes and per-token parameters of
 // 64 tokens; the first half also carries the block's channel scales and NSN
 // channel means.
+//
+// Under DQ the block record (codes of o and s1, their fp16 parameters) sits
+// between the token parameters and the channel scales, and both halves
+// carry it (each half's tokens need their s1 codes).
 template <int D, int BITS, int MODE>
 struct SlotLayout {
+    static constexpr bool kDq = MODE == kNsnDq;
     static constexpr int kRB = D * BITS / 8;
-    static constexpr int kNtok = (MODE == kNsn) ? 2 : 1;
+    static constexpr int kNtok = tok_params(MODE);
     static constexpr int kCodes = 0;
     static constexpr int kTok = kUT * kRB;
-    static constexpr int kChan = kTok + kUT * kNtok * 2;
+    static constexpr int kRec = kTok + kUT * kNtok * 2;  // DQ record
+    static constexpr int kChan = kRec + (kDq ? dq_record_bytes<D>() : 0);
     static constexpr int kOff = kChan + ((MODE != kNaive) ? D * 2 : 0);
     static constexpr int kBytesLo = kOff + ((MODE == kNsn) ? D * 2 : 0);  // first half
     static constexpr int kBytesHi = kChan;                                 // second half
     static constexpr int kStride = (kBytesLo + 127) / 128 * 128;
+    static_assert(kRec % 16 == 0 && kChan % 16 == 0, "bulk copies start on 16-byte boundaries");
 };
+
+// The codes of o for 16 channels (8 bytes at p) as exact fp16 pairs q = e - 8
+// (channels 2k, 2k + 1 in pair k).
+__device__ __forceinline__ void dq_o_pairs(const uint8_t* p, __half2 (&o)[8]) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t b = ((k < 4 ? w.x : w.y) >> (8 * (k & 3))) & 0xFFu;
+        o[k] = __floats2half2_rn((float)((int)(b & 15u) - 8), (float)((int)(b >> 4) - 8));
+    }
+}
+
+// s1 of token tok (0..63) of unit half `half` from the record at rec (DQ).
+template <int D>
+__device__ __forceinline__ float dq_s1_unit(const uint8_t* rec, int half, int tok) {
+    return dq_s1<D>(rec, 64 * half + tok);
+}
 
 // Rotated-query table (fp32): channel c of head j at j * kQS + c + 4 (c / 32).
 // The B-fragment build reads 16-byte chunks of the 32-channel slice t of one
@@ -421,7 +445,7 @@ __device__ __forceinline__ uint32_t split_h2(float x) {
 // three resident CTAs per SM (168 registers), where the register allocator
 // otherwise spills or settles for fewer CTAs; the others are left to it.
 template <int D, int BITS, int MODE, bool HAD, int GP>
-__global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP == 4) ? 3 : 0)
+__global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP == 4) ? 3 : 0)
     decode_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "tensor-core decode is built for head dim 128");
     using SL = SlotLayout<D, BITS, MODE>;
@@ -473,6 +497,9 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
         mbar_expect_tx(bar, half ? SL::kBytesHi : SL::kBytesLo);
         bulk_load(slot + SL::kCodes, (ten ? a.codes[1] : a.codes[0]) + row0 * SL::kRB, kUT * SL::kRB, bar);
         bulk_load(slot + SL::kTok, (ten ? a.tok[1] : a.tok[0]) + row0 * SL::kNtok, kUT * SL::kNtok * 2, bar);
+        if (SL::kDq)
+            bulk_load(slot + SL::kRec, (ten ? a.off[1] : a.off[0]) + ((size_t)pair * nb_cap + blk) * off_words<D, MODE>(),
+                      dq_record_bytes<D>(), bar);
         if (!half) {
             if (PCH) bulk_load(slot + SL::kChan, (ten ? a.chan[1] : a.chan[0]) + bi, D * 2, bar);
             if (MODE == kNsn) bulk_load(slot + SL::kOff, (ten ? a.off[1] : a.off[0]) + bi, D * 2, bar);
@@ -575,7 +602,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
             l_run[n] = 0.0f;
             // 2^-qsc with the softmax scale (log2 units) and the fixed token
             // factor of the mode folded in
-            kcol[n] = alpha2 * ((MODE == kNsn && !HAD) ? a.sqd : (MODE == kNsep && HAD) ? a.rsqd : 1.0f) /
+            kcol[n] = alpha2 * ((is_nsn(MODE) && !HAD) ? a.sqd : (MODE == kNsep && HAD) ? a.rsqd : 1.0f) /
                       wqsc[4 * n + t];
 #pragma unroll
             for (int k = 0; k < 16; ++k) { acc[n][k] = 0.0f; acco[n][k] = 0.0f; }
@@ -584,6 +611,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
         float kb[NT][2];  // -1152 * sum of B over the biased pairs (hi, lo columns)
         float qoK[NT];
         __half2 sigv[8], offv[8];
+        float osv = 1.0f;  // DQ: sigma_o of the block's V means
 
         for (int it = pos; it < pos + seg; ++it) {
 #pragma unroll 1
@@ -650,22 +678,31 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
                             kb[n][1] = c0[1] + c1[1];
                         }
                     }
-                    if constexpr (MODE == kNsn) {
-                        // q . o^K for head 4n + t: lanes (g) split the channels
-                        const __half2* okp = reinterpret_cast<const __half2*>(sk + SL::kOff) + 8 * g;
+                    if constexpr (is_nsn(MODE)) {
+                        // q . o^K for head 4n + t: lanes (g) split the channels;
+                        // under DQ o = (e - 8) sigma_o, with sigma_o applied once
+                        __half2 okv[8];
+                        float osc = 1.0f;
+                        if constexpr (MODE == kNsn) {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) okv[k] = reinterpret_cast<const __half2*>(sk + SL::kOff)[8 * g + k];
+                        } else {
+                            dq_o_pairs(sk + SL::kRec + 8 * g, okv);
+                            osc = __half2float(reinterpret_cast<const __half*>(sk + SL::kRec + dq_params_at<D>())[0]);
+                        }
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
                             const uint32_t* qh = &wqw[qw_word(4 * n + t, 16 * g)];  // channels 16g .. 16g + 15
                             float s = 0.0f;
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
-                                const float2 o2 = __half22float2(okp[k]);
+                                const float2 o2 = __half22float2(okv[k]);
                                 const float2 q2 = __half22float2(*reinterpret_cast<const __half2*>(&qh[k]));
                                 s += q2.x * o2.x + q2.y * o2.y;
                             }
 #pragma unroll
                             for (int o = 4; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                            qoK[n] = s * alpha2;
+                            qoK[n] = s * (osc * alpha2);
                         }
                     }
                 }
@@ -679,6 +716,12 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
                         offv[k] = (MODE == kNsn) ? reinterpret_cast<const __half2*>(sv + SL::kOff)[8 * g + k]
                                                  : __floats2half2_rn(0.f, 0.f);
                     }
+                    // DQ: the codes q of o^V as exact fp16 pairs; sigma_o^V
+                    // multiplies the offset term once per unit
+                    if constexpr (MODE == kNsnDq) {
+                        dq_o_pairs(sv + SL::kRec + 8 * g, offv);
+                        osv = __half2float(reinterpret_cast<const __half*>(sv + SL::kRec + dq_params_at<D>())[0]);
+                    }
                 }
                 const __half* tk = reinterpret_cast<const __half*>(sk + SL::kTok);
                 const __half* tv = reinterpret_cast<const __half*>(sv + SL::kTok);
@@ -691,6 +734,8 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
                     if constexpr (MODE == kNsn) {
                         const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
                         v = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
+                    } else if constexpr (MODE == kNsnDq) {
+                        v = dq_s1_unit<D>(sv + SL::kRec, half, tok) * __half2float(tv[tok]) * (HAD ? 1.0f : a.sqd);
                     } else {
                         v = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
                     }
@@ -702,7 +747,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
                 const float pscale = pow2i(fexp), pinv = pow2i(-fexp);
                 // 2^f with the fixed token factor of the mode
                 const float pscale_m =
-                    pscale * ((MODE == kNsn && !HAD) ? a.sqd : (MODE == kNsep && HAD) ? a.rsqd : 1.0f);
+                    pscale * ((is_nsn(MODE) && !HAD) ? a.sqd : (MODE == kNsep && HAD) ? a.rsqd : 1.0f);
                 // ---- scores of the unit's 64 tokens (four independent 16-token tiles)
                 float l2[4][NT][2];
                 bool over = false;
@@ -734,6 +779,9 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
                             if constexpr (MODE == kNsn) {
                                 const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tk)[tok]);
                                 l2[m4][n][r] = s12.x * fmaf(sv_, s12.y * kcol[n], qoK[n]);
+                            } else if constexpr (MODE == kNsnDq) {
+                                const float s1 = dq_s1_unit<D>(sk + SL::kRec, half, tok);
+                                l2[m4][n][r] = s1 * fmaf(sv_, __half2float(tk[tok]) * kcol[n], qoK[n]);
                             } else {
                                 l2[m4][n][r] = sv_ * (__half2float(tk[tok]) * kcol[n]);
                             }
@@ -758,7 +806,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
 #pragma unroll
                         for (int k = 0; k < 16; ++k) {
                             acc[n][k] *= corr;
-                            if (MODE == kNsn) acco[n][k] *= corr;
+                            if (is_nsn(MODE)) acco[n][k] *= corr;
                         }
                     }
                 }
@@ -779,6 +827,9 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
                             const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
                             s1o = s12.x;
                             nu = s12.x * (s12.y * pscale_m);
+                        } else if constexpr (MODE == kNsnDq) {
+                            s1o = dq_s1_unit<D>(sv + SL::kRec, half, tok);
+                            nu = s1o * (__half2float(tv[tok]) * pscale_m);
                         } else {
                             nu = __half2float(tv[tok]) * pscale_m;
                         }
@@ -786,7 +837,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
                         for (int n = 0; n < NT; ++n) {
                             const float p = fast_exp2(l2[m4][n][r] - m_ref[n]);
                             lsum[n] += p;
-                            if constexpr (MODE == kNsn) bsum[n] += p * s1o;
+                            if constexpr (is_nsn(MODE)) bsum[n] += p * s1o;
                             const float x_ = p * nu;
                             if constexpr (VB) psum[n] += x_;
                             bpa[m4][n][r] = movmatrix_t(split_h2(x_));
@@ -843,11 +894,12 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
                             acc[n][2 * tc + 1] += (dv[n][tc][2] + dv[n][tc][3]) * s1_;
                     }
                 }
-                if constexpr (MODE == kNsn) {
+                if constexpr (is_nsn(MODE)) {
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
 #pragma unroll
                         for (int o = 4; o < 32; o <<= 1) bsum[n] += __shfl_xor_sync(0xffffffffu, bsum[n], o);
+                        if constexpr (MODE == kNsnDq) bsum[n] *= osv;
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
                             const float2 ov = __half22float2(offv[k]);
@@ -911,7 +963,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || MODE == kNsn) && GP =
 #pragma unroll
                 for (int k = 0; k < 16; k += 4) {
                     float4 v4 = make_float4(acc[n][k], acc[n][k + 1], acc[n][k + 2], acc[n][k + 3]);
-                    if constexpr (MODE == kNsn) {
+                    if constexpr (is_nsn(MODE)) {
                         v4.x += acco[n][k]; v4.y += acco[n][k + 1]; v4.z += acco[n][k + 2]; v4.w += acco[n][k + 3];
                     }
                     *reinterpret_cast<float4*>(pj + 4 + 16 * g + k) = v4;

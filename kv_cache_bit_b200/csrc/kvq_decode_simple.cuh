@@ -45,7 +45,8 @@ __global__ void __launch_bounds__(128) decode_split_kernel(DecodeArgs a) {
     const int split = blockIdx.x, bh = blockIdx.y;
     const int G = a.G;
     const int nb_cap = a.cap / kT;
-    const int ntk = (MODE == kNsn) ? 2 : 1;
+    const int ntk = tok_params(MODE);
+    constexpr int OW = off_words<D, MODE>();
 
     __shared__ float s_qo[kGMax][D];   // queries, original domain
     __shared__ float s_qt[kGMax][D];   // queries, rotated domain (HADAMARD)
@@ -85,6 +86,12 @@ __global__ void __launch_bounds__(128) decode_split_kernel(DecodeArgs a) {
     const int blk_end = min(a.nbq, blk_begin + a.bps);
     for (int blk = blk_begin; blk < blk_end; ++blk) {
         // 1. block parameters and q'
+        const uint8_t* reck = nullptr;
+        const uint8_t* recv = nullptr;
+        if constexpr (MODE == kNsnDq) {
+            reck = reinterpret_cast<const uint8_t*>(a.off[0] + ((size_t)bh * nb_cap + blk) * OW);
+            recv = reinterpret_cast<const uint8_t*>(a.off[1] + ((size_t)bh * nb_cap + blk) * OW);
+        }
         if (t < D) {
             const size_t bi = ((size_t)bh * nb_cap + blk) * D + t;
             const float sk = (MODE != kNaive) ? __half2float(a.chan[0][bi]) : 1.0f;
@@ -93,10 +100,14 @@ __global__ void __launch_bounds__(128) decode_split_kernel(DecodeArgs a) {
                 s_offk[t] = __half2float(a.off[0][bi]);
                 s_offv[t] = __half2float(a.off[1][bi]);
             }
+            if (MODE == kNsnDq) {
+                s_offk[t] = dq_o<D>(reck, t);
+                s_offv[t] = dq_o<D>(recv, t);
+            }
             for (int j = 0; j < G; ++j) s_qp[j][t] = s_qt[j][t] * sk;
         }
         __syncthreads();
-        if constexpr (MODE == kNsn) {
+        if constexpr (is_nsn(MODE)) {
             for (int j = warp; j < G; j += 4) {
                 float s = 0.0f;
                 for (int c = lane; c < D; c += 32) s += s_qo[j][c] * s_offk[c];
@@ -129,13 +140,18 @@ __global__ void __launch_bounds__(128) decode_split_kernel(DecodeArgs a) {
                 kap = s1k * __half2float(tp[1]) * (HAD ? 1.0f : a.sqd);
                 s1v = __half2float(tv[0]);
                 nu = s1v * __half2float(tv[1]) * (HAD ? 1.0f : a.sqd);
+            } else if constexpr (MODE == kNsnDq) {
+                s1k = dq_s1<D>(reck, t);
+                kap = s1k * __half2float(tp[0]) * (HAD ? 1.0f : a.sqd);
+                s1v = dq_s1<D>(recv, t);
+                nu = s1v * __half2float(tv[0]) * (HAD ? 1.0f : a.sqd);
             } else {
                 kap = __half2float(tp[0]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
                 nu = __half2float(tv[0]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
             }
             for (int j = 0; j < G; ++j) {
                 float lg = kap * sj[j];
-                if (MODE == kNsn) lg += s1k * s_qok[j];
+                if (is_nsn(MODE)) lg += s1k * s_qok[j];
                 s_lg[j][t] = a.scale * lg;
             }
             s_nu[t] = nu;
@@ -196,7 +212,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(DecodeArgs a) {
             for (int j = 0; j < kGMax; ++j) {
                 if (j < G) {
                     acc[j] = acc[j] * s_corr[j] + s_sigv[t] * aj[j];
-                    acco[j] = acco[j] * s_corr[j] + ((MODE == kNsn) ? s_beta[j] * s_offv[t] : 0.0f);
+                    acco[j] = acco[j] * s_corr[j] + (is_nsn(MODE) ? s_beta[j] * s_offv[t] : 0.0f);
                 }
             }
         }

@@ -16,7 +16,42 @@ namespace kvq {
 
 constexpr int kT = 128;  // tokens per scale block
 
-enum Mode : int { kNsep = 0, kNaive = 1, kNsn = 2 };
+// kNsnDq: NSN with its side parameters double quantized (the block mean o
+// and the token scale s1 kept as 4-bit codes in a per-block record).
+enum Mode : int { kNsep = 0, kNaive = 1, kNsn = 2, kNsnDq = 3 };
+
+__host__ __device__ constexpr bool is_nsn(int mode) { return mode == kNsn || mode == kNsnDq; }
+
+// fp16 per-token parameters stored: NSN (s1, s2); NSN with DQ (s2; s1 is in
+// the block record); nsep the norm; naive the token scale.
+__host__ __device__ constexpr int tok_params(int mode) { return mode == kNsn ? 2 : 1; }
+
+// Block record of the double-quantized NSN side parameters, bytes:
+//   [0, D/2)            codes of o: e = q + 8, channel 2j in the low nibble of byte j
+//   [D/2, D/2 + 64)     codes of s1: q in 0..15, token 2j in the low nibble of byte j
+//   D/2 + 64 + {0,2,4}  fp16 sigma_o, lo, step;  zeros up to a multiple of 16
+// o_hat_c = (e_c - 8) sigma_o;  s1_hat_t = lo + q_t step.
+template <int D>
+__host__ __device__ constexpr int dq_record_bytes() { return (D / 2 + 64 + 6 + 15) / 16 * 16; }
+template <int D>
+__host__ __device__ constexpr int dq_params_at() { return D / 2 + 64; }
+// o_hat of channel c and s1_hat of token t from a block record (as fp32, in
+// the oracle's operation order).
+template <int D>
+__device__ __forceinline__ float dq_o(const uint8_t* rec, int c) {
+    const int e = (rec[c >> 1] >> (4 * (c & 1))) & 15;
+    return __fmul_rn((float)(e - 8), __half2float(reinterpret_cast<const __half*>(rec + dq_params_at<D>())[0]));
+}
+template <int D>
+__device__ __forceinline__ float dq_s1(const uint8_t* rec, int t) {
+    const int q = (rec[D / 2 + (t >> 1)] >> (4 * (t & 1))) & 15;
+    const __half* pr = reinterpret_cast<const __half*>(rec + dq_params_at<D>());
+    return __fadd_rn(__half2float(pr[1]), __fmul_rn((float)q, __half2float(pr[2])));
+}
+
+// fp16 words per block of the NSN offsets array: D means, or the record.
+template <int D, int MODE>
+__host__ __device__ constexpr int off_words() { return MODE == kNsnDq ? dq_record_bytes<D>() / 2 : D; }
 
 // Sticky device error word, readable with kvq_read_device_errors().
 constexpr uint32_t kErrTmaTimeout = 1u;
@@ -575,6 +610,18 @@ __device__ __forceinline__ f2_t lds_f2(uint32_t addr) {
     return r;
 }
 
+// min / max over the warp's lanes of x (exact).
+__device__ __forceinline__ float warp_min(float x) {
+    float r;
+    asm volatile("redux.sync.min.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float warp_max(float x) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // max over the warp's lanes of |x| (exact: a comparison, no rounding).
 __device__ __forceinline__ float warp_max_abs(float x) {
     float r;
@@ -700,10 +747,22 @@ __device__ __forceinline__ void quantize_rows(uint4 (&raw)[D / 8], const int t, 
     float kscale = 1.0f;
     f2_t P[H2];
 
-    if constexpr (MODE == kNsn) {
+    if constexpr (is_nsn(MODE)) {
+        constexpr bool DQ = MODE == kNsnDq;
+        // DQ scratch past the group sums: [0, 4) warp minima of s1, [4, 8)
+        // warp maxima, [8, 8 + D/32) warp maxima of |o|, then the o codes
+        float* dqs = sm.gpart + 768;
+        uint8_t* dq_e = reinterpret_cast<uint8_t*>(dqs + 16);
         const float n1 = __fsqrt_rn(raw_row_sumsq<D>(raw));
         const float s1 = __fmul_rn(n1, rsqd);
         const float r1 = n1 > 0.0f ? __fdiv_rn(sqd, n1) : 0.0f;
+        if constexpr (DQ) {
+            const float mn = warp_min(s1), mx = warp_max(s1);
+            if ((t & 31) == 0) {
+                dqs[t >> 5] = mn;
+                dqs[4 + (t >> 5)] = mx;
+            }
+        }
         // a = x * r1, with the rotation's signs when SIGNS
         widen_row<D, SIGNS>(raw, sm, P);
         const f2_t R1 = f2_pack(r1, r1);
@@ -772,10 +831,64 @@ __device__ __forceinline__ void quantize_rows(uint4 (&raw)[D / 8], const int t, 
             }
             // the mean of the signed rows; the stored mean is of the unsigned
             // ones (a sign flip commutes exactly with the sum and the rounding)
-            const __half o16 = __float2half_rn(__fmul_rn(gs[0], 1.0f / 128.0f));
+            const float of = __fmul_rn(gs[0], 1.0f / 128.0f);
             const int c = (t >> 1) + (t & 1) * H2;
-            out.off[c] = (SIGNS && sign16(sm.sgn2, c)) ? __hneg(o16) : o16;
-            sm.vec[t] = __half2float(o16);
+            if constexpr (DQ) {
+                sm.vec[t] = of;
+                const float m = warp_max_abs(of);
+                if ((t & 31) == 0) dqs[8 + (t >> 5)] = m;
+            } else {
+                const __half o16 = __float2half_rn(of);
+                out.off[c] = (SIGNS && sign16(sm.sgn2, c)) ? __hneg(o16) : o16;
+                sm.vec[t] = __half2float(o16);
+            }
+        }
+        if constexpr (DQ) {
+            // 4-bit o and s1 (double quantization), into the block record
+            __syncthreads();
+            constexpr float kC = 12582912.0f;  // 1.5 * 2^23: fma(y, 1, kC) = kC + rne(y)
+            uint8_t* rec = reinterpret_cast<uint8_t*>(out.off);
+            float mo = dqs[8];
+#pragma unroll
+            for (int w = 1; w < D / 32; ++w) mo = fmaxf(mo, dqs[8 + w]);
+            const __half so16 = __float2half_rn(__fdiv_rn(mo, 7.0f));
+            const float so = __half2float(so16);
+            const float invo = so > 0.0f ? __fdiv_rn(1.0f, so) : 0.0f;
+            if (t < D) {
+                // e = q + 8, q = clamp(rne(o / sigma_o), -7, 7); the rows carry
+                // the signs: o_hat of the signed mean, the code of the unsigned
+                const float r = fminf(fmaxf(__fmaf_rn(sm.vec[t], invo, kC + 8.0f), kC + 1.0f), kC + 15.0f);
+                const int q = (int)(__float_as_uint(r) & 15u) - 8;
+                sm.vec[t] = __fmul_rn((float)q, so);
+                const int c = (t >> 1) + (t & 1) * H2;
+                dq_e[c] = (uint8_t)(((SIGNS && sign16(sm.sgn2, c)) ? -q : q) + 8);
+            }
+            float mn = dqs[0], mx = dqs[4];
+#pragma unroll
+            for (int w = 1; w < 4; ++w) {
+                mn = fminf(mn, dqs[w]);
+                mx = fmaxf(mx, dqs[4 + w]);
+            }
+            const __half lo16 = __float2half_rn(mn);
+            const float lo = __half2float(lo16);
+            const float span = fmaxf(__fsub_rn(mx, lo), 0.0f);
+            const __half st16 = __float2half_rn(__fdiv_rn(span, 15.0f));
+            const float st = __half2float(st16);
+            const float invs = st > 0.0f ? __fdiv_rn(1.0f, st) : 0.0f;
+            const float rq = fminf(fmaxf(__fmaf_rn(__fsub_rn(s1, lo), invs, kC), kC), kC + 15.0f);
+            const uint32_t qs = __float_as_uint(rq) & 15u;
+            const uint32_t qn = __shfl_xor_sync(0xffffffffu, qs, 1);
+            if ((t & 1) == 0) rec[D / 2 + t / 2] = (uint8_t)(qs | (qn << 4));
+            if (t == 0) {
+                __half* pr = reinterpret_cast<__half*>(rec + dq_params_at<D>());
+                pr[0] = so16;
+                pr[1] = lo16;
+                pr[2] = st16;
+#pragma unroll
+                for (int i = dq_params_at<D>() + 6; i < dq_record_bytes<D>(); ++i) rec[i] = 0;
+            }
+            __syncthreads();
+            if (t < D / 2) rec[t] = (uint8_t)(dq_e[2 * t] | (dq_e[2 * t + 1] << 4));
         }
         __syncthreads();
         after_means();  // the transposed buffer is free again
@@ -786,7 +899,8 @@ __device__ __forceinline__ void quantize_rows(uint4 (&raw)[D / 8], const int t, 
         const float n2 = __fsqrt_rn(row_sumsq<H2, false>(P));
         const float s2 = __fmul_rn(n2, rsqd);
         kscale = n2 > 0.0f ? __fdiv_rn(c0, n2) : 0.0f;
-        reinterpret_cast<__half2*>(out.tok)[t] = __halves2half2(__float2half_rn(s1), __float2half_rn(s2));
+        if constexpr (DQ) out.tok[t] = __float2half_rn(s2);
+        else reinterpret_cast<__half2*>(out.tok)[t] = __halves2half2(__float2half_rn(s1), __float2half_rn(s2));
     } else if constexpr (MODE == kNsep) {
         widen_row<D, SIGNS>(raw, sm, P);
         const float n = __fsqrt_rn(row_sumsq<H2, true>(P));

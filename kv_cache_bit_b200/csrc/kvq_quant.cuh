@@ -28,7 +28,7 @@ struct QuantArgs {
 // transposed buffer) while the third receives the next tile.
 template <int MODE>
 __host__ __device__ constexpr int quant_regions() {
-    return MODE == kNsn ? 3 : 2;
+    return is_nsn(MODE) ? 3 : 2;
 }
 
 template <int D>
@@ -49,7 +49,7 @@ __host__ __device__ constexpr int quant_smem_bytes() {
 // registers than three CTAs leave; those run two CTAs per SM.
 template <int D, int BITS, int MODE, bool HAD>
 __host__ __device__ constexpr int quant_min_ctas() {
-    return D == 128 ? ((MODE == kNsn || (HAD && BITS == 3)) ? 2 : 3) : 4;
+    return D == 128 ? ((is_nsn(MODE) || (HAD && BITS == 3)) ? 2 : 3) : 4;
 }
 
 template <int D, int MODE>
@@ -78,7 +78,7 @@ __device__ __forceinline__ QuantSmem<D> carve_quant_smem(uint8_t* base, uint64_t
 template <int D, int BITS, int MODE, bool HAD>
 __device__ __forceinline__ QuantOut quant_out(const QuantArgs& a, int tensor, int bh, int blk) {
     using L = RowLayout<D, BITS>;
-    const int ntk = (MODE == kNsn) ? 2 : 1;
+    const int ntk = tok_params(MODE);
     const int nb = a.cap / kT;
     QuantOut o;
     // select with ternaries: a runtime index into the parameter arrays would
@@ -87,7 +87,7 @@ __device__ __forceinline__ QuantOut quant_out(const QuantArgs& a, int tensor, in
     o.codes = (v ? a.codes[1] : a.codes[0]) + ((size_t)bh * a.cap + (size_t)blk * kT) * L::kBytes;
     o.tok = (v ? a.tok[1] : a.tok[0]) + ((size_t)bh * a.cap + (size_t)blk * kT) * ntk;
     o.chan = (MODE != kNaive) ? (v ? a.chan[1] : a.chan[0]) + ((size_t)bh * nb + blk) * D : nullptr;
-    o.off = (MODE == kNsn) ? (v ? a.off[1] : a.off[0]) + ((size_t)bh * nb + blk) * D : nullptr;
+    o.off = is_nsn(MODE) ? (v ? a.off[1] : a.off[0]) + ((size_t)bh * nb + blk) * off_words<D, MODE>() : nullptr;
     o.stage = nullptr;
     o.pairv = pairv_layout<D>() && v;
     return o;
@@ -286,16 +286,16 @@ struct DequantArgs {
 };
 
 // Token row rebuilt in fp32 from its code words w32 and parameters (tp: its
-// per-token fp16 values; sig, off: the block's channel scales and means as
-// fp32; sgn: the rotation's signs as fp32 sign-bit masks), in the oracle's
-// operation order:
+// per-token fp16 values; s1dq: its s1 rebuilt from the block record under
+// DQ; sig, off: the block's channel scales and means as fp32; sgn: the
+// rotation's signs as fp32 sign-bit masks), in the oracle's operation order:
 //   w = q * sigma; nsep x = n * w, or s (.) (H w * (n rsqd)) under HADAMARD;
 //   naive x = w; NSN x = s1 * (b + o) with b = w * (s2 sqd), or
 //   s (.) (H w * s2) under HADAMARD.
 template <int D, int BITS, int MODE, bool HAD>
 __device__ __forceinline__ void dequant_row(const uint32_t (&w32)[RowLayout<D, BITS>::kWords], const __half* tp,
-                                            const float* sig, const float* off, const uint32_t* sgn, float rsqd,
-                                            float sqd, float (&w)[D]) {
+                                            float s1dq, const float* sig, const float* off, const uint32_t* sgn,
+                                            float rsqd, float sqd, float (&w)[D]) {
     using L = RowLayout<D, BITS>;
     const float tsig = (MODE == kNaive) ? __half2float(tp[0]) : 0.0f;
 #pragma unroll
@@ -304,8 +304,10 @@ __device__ __forceinline__ void dequant_row(const uint32_t (&w32)[RowLayout<D, B
         w[c] = __fmul_rn(q, (MODE == kNaive) ? tsig : sig[c]);
     }
     if constexpr (HAD) fwht_reg<D>(w);
-    if constexpr (MODE == kNsn) {
-        const float s1 = __half2float(tp[0]), s2 = __half2float(tp[1]);
+    if constexpr (is_nsn(MODE)) {
+        // under DQ s1 comes from the block record (s1dq) and tp holds s2 only
+        const float s1 = (MODE == kNsnDq) ? s1dq : __half2float(tp[0]);
+        const float s2 = __half2float(tp[MODE == kNsnDq ? 0 : 1]);
         const float kb = HAD ? s2 : __fmul_rn(s2, sqd);
 #pragma unroll
         for (int c = 0; c < D; ++c) {
@@ -333,12 +335,16 @@ __global__ void __launch_bounds__(128) dequantize_kernel(DequantArgs a) {
     const int t = threadIdx.x;
     const int blk = a.blk0 + blockIdx.x, bh = blockIdx.y;
     const int nb = a.cap / kT;
-    const int ntk = (MODE == kNsn) ? 2 : 1;
+    const int ntk = tok_params(MODE);
     __shared__ float s_sig[D], s_off[D];
     __shared__ uint32_t s_sgn[D];
+    const __half* offb = is_nsn(MODE) ? a.off + ((size_t)bh * nb + blk) * off_words<D, MODE>() : nullptr;
+    float s1dq = 0.0f;
+    if constexpr (MODE == kNsnDq) s1dq = dq_s1<D>(reinterpret_cast<const uint8_t*>(offb), t);
     if (t < D) {
         if (MODE != kNaive) s_sig[t] = __half2float(a.chan[((size_t)bh * nb + blk) * D + t]);
-        if (MODE == kNsn) s_off[t] = __half2float(a.off[((size_t)bh * nb + blk) * D + t]);
+        if (MODE == kNsn) s_off[t] = __half2float(offb[t]);
+        if (MODE == kNsnDq) s_off[t] = dq_o<D>(reinterpret_cast<const uint8_t*>(offb), t);
         s_sgn[t] = (HAD && a.signs != nullptr && a.signs[t] < 0) ? 0x80000000u : 0u;
     }
     __syncthreads();
@@ -363,7 +369,7 @@ __global__ void __launch_bounds__(128) dequantize_kernel(DequantArgs a) {
         load_words<L::kWords>(a.codes + tok_idx * L::kBytes, w32);
     }
     float w[D];
-    dequant_row<D, BITS, MODE, HAD>(w32, a.tok + tok_idx * ntk, s_sig, s_off, s_sgn, a.rsqd, a.sqd, w);
+    dequant_row<D, BITS, MODE, HAD>(w32, a.tok + tok_idx * ntk, s1dq, s_sig, s_off, s_sgn, a.rsqd, a.sqd, w);
     float* o = a.out + ((size_t)bh * a.ntok + (size_t)blockIdx.x * kT + t) * D;
 #pragma unroll
     for (int k = 0; k < D / 4; ++k)
@@ -392,6 +398,9 @@ __device__ __forceinline__ double row_sq_err(const float (&w)[D], const __half* 
     }
 }
 
+static_assert(dq_record_bytes<64>() <= 64 * 2 && dq_record_bytes<128>() <= 128 * 2,
+              "a block record fits the means buffer of the selection kernel");
+
 template <int D, int BITS, int MODE>
 __host__ __device__ constexpr int select_smem_bytes() {
     // the quantizer's scratch, then the block's outputs and the per-row errors
@@ -406,7 +415,7 @@ __host__ __device__ constexpr int select_smem_bytes() {
 template <int D, int BITS, int MODE>
 __global__ void __launch_bounds__(128) select_signs_kernel(SelectArgs a) {
     using L = RowLayout<D, BITS>;
-    constexpr int ntk = (MODE == kNsn) ? 2 : 1;
+    constexpr int ntk = tok_params(MODE);
     const int t = threadIdx.x, blk = blockIdx.x, cand = blockIdx.y;
     extern __shared__ uint8_t smem_raw[];
     uint64_t* bar;
@@ -441,13 +450,15 @@ __global__ void __launch_bounds__(128) select_signs_kernel(SelectArgs a) {
     __syncthreads();
     if (t < D) {
         s_sig[t] = __half2float(s_chan[t]);
-        s_off[t] = (MODE == kNsn) ? __half2float(s_off16[t]) : 0.0f;
+        s_off[t] = (MODE == kNsn) ? __half2float(s_off16[t])
+                 : (MODE == kNsnDq) ? dq_o<D>(reinterpret_cast<const uint8_t*>(s_off16), t) : 0.0f;
     }
     __syncthreads();
     uint32_t w32[L::kWords];
     load_words<L::kWords>(s_codes + (size_t)t * L::kBytes, w32);
     float w[D];
-    dequant_row<D, BITS, MODE, true>(w32, s_tok + t * ntk, s_sig, s_off, s_sgn, a.rsqd, a.sqd, w);
+    const float s1dq = (MODE == kNsnDq) ? dq_s1<D>(reinterpret_cast<const uint8_t*>(s_off16), t) : 0.0f;
+    dequant_row<D, BITS, MODE, true>(w32, s_tok + t * ntk, s1dq, s_sig, s_off, s_sgn, a.rsqd, a.sqd, w);
     s_err[t] = row_sq_err<0, D, D>(w, xr);
     __syncthreads();
 #pragma unroll

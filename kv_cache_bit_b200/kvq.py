@@ -17,11 +17,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "_lib", "libkvq.so")
 
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = range(6)
-KVQ_NORM_SEP, KVQ_PER_CHANNEL, KVQ_NSN, KVQ_HADAMARD = 1, 2, 4, 8
-NORM_SEP, PER_CHANNEL, NSN, HADAMARD = KVQ_NORM_SEP, KVQ_PER_CHANNEL, KVQ_NSN, KVQ_HADAMARD
+KVQ_NORM_SEP, KVQ_PER_CHANNEL, KVQ_NSN, KVQ_HADAMARD, KVQ_DQ = 1, 2, 4, 8, 16
+NORM_SEP, PER_CHANNEL, NSN, HADAMARD, DQ = KVQ_NORM_SEP, KVQ_PER_CHANNEL, KVQ_NSN, KVQ_HADAMARD, KVQ_DQ
 BLOCK_TOKENS = 128
 
-EXPORTS = ["kvq_row_bytes", "kvq_tok_params", "kvq_make_signs", "kvq_quantize_block", "kvq_append_token",
+EXPORTS = ["kvq_row_bytes", "kvq_tok_params", "kvq_off_words", "kvq_make_signs", "kvq_quantize_block", "kvq_append_token",
            "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_dequantize",
            "kvq_select_signs_workspace_bytes", "kvq_select_signs", "kvq_read_device_errors",
            "kvq_status_string"]
@@ -48,6 +48,8 @@ def _load():
     L.kvq_row_bytes.argtypes = [ctypes.c_int32, ctypes.c_int32]
     L.kvq_tok_params.restype = ctypes.c_int32
     L.kvq_tok_params.argtypes = [ctypes.c_uint32]
+    L.kvq_off_words.restype = ctypes.c_int32
+    L.kvq_off_words.argtypes = [ctypes.c_uint32, ctypes.c_int32]
     L.kvq_make_signs.restype = ctypes.c_int
     L.kvq_make_signs.argtypes = [ctypes.c_uint64, ctypes.c_int32, P]
     L.kvq_quantize_block.restype = ctypes.c_int
@@ -115,6 +117,10 @@ def kvq_row_bytes(head_dim: int, bits: int) -> int:
 
 def kvq_tok_params(flags: int) -> int:
     return lib.kvq_tok_params(flags)
+
+
+def kvq_off_words(flags: int, head_dim: int) -> int:
+    return lib.kvq_off_words(flags, head_dim)
 
 
 def kvq_make_signs(seed: int, head_dim: int):
@@ -222,7 +228,8 @@ class KVCache:
         tok = [mk((batch, kv_heads, capacity, nt), torch.int16) for _ in range(2)]
         pchan = bool(cfg.flags & PER_CHANNEL)
         chan = [mk((batch, kv_heads, nb, d), torch.int16) if pchan else None for _ in range(2)]
-        off = [mk((batch, kv_heads, nb, d), torch.int16) if cfg.flags & NSN else None for _ in range(2)]
+        ow = kvq_off_words(cfg.flags, d)
+        off = [mk((batch, kv_heads, nb, ow), torch.int16) if cfg.flags & NSN else None for _ in range(2)]
         resid = [mk((batch, kv_heads, BLOCK_TOKENS, d), torch.int16) for _ in range(2)]
         c = kvq_cache(batch, kv_heads, d, capacity, 0,
                       (ctypes.c_void_p * 2)(*[_ptr(x) for x in codes]),

@@ -156,6 +156,8 @@ MODES = {
     "rht+nsep+pchan": (("NORM_SEP", "PER_CHANNEL", "HADAMARD"), True),
     "nsn+hadamard": (("NSN", "PER_CHANNEL", "HADAMARD"), False),
     "nsn": (("NSN", "PER_CHANNEL"), False),
+    "nsn+hadamard+dq": (("NSN", "PER_CHANNEL", "HADAMARD", "DQ"), False),
+    "nsn+dq": (("NSN", "PER_CHANNEL", "DQ"), False),
     "nsep-only": (("NORM_SEP",), False),
     "pchan-only": (("PER_CHANNEL",), False),
 }

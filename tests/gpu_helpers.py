@@ -120,8 +120,13 @@ def compare_cache(gcache, ck, cv, d, bits, nq, bh_slice=slice(None), t0=0):
             res["chan_ulp"] = max(res["chan_ulp"], fp16_ulp_diff(host16(gcache.chan[i][bh_slice][:, :, b0:nb]),
                                                                  oc["chan"][:, :, b0:nb]))
         if oc["off"] is not None:
-            res["off_ulp"] = max(res["off_ulp"], fp16_ulp_diff(host16(gcache.off[i][bh_slice][:, :, b0:nb]),
-                                                               oc["off"][:, :, b0:nb]))
+            g_off = host16(gcache.off[i][bh_slice][:, :, b0:nb])
+            if oc["off"].shape[-1] == d:
+                res["off_ulp"] = max(res["off_ulp"], fp16_ulp_diff(g_off, oc["off"][:, :, b0:nb]))
+            else:
+                # DQ block records (4-bit codes of o and s1, fp16 parameters):
+                # byte for byte
+                assert np.array_equal(g_off, oc["off"][:, :, b0:nb]), "DQ block records differ"
     HALF_POINT_LOG.append((res["half_points"], res["codes"]))
     return res
 

@@ -157,3 +157,16 @@ def test_select_signs_host_checks(kvq):
     assert args(had, nb=0) == kvq.KVQ_ERR_INVALID_ARG
     assert args(had, ws=None) == kvq.KVQ_ERR_WORKSPACE
     assert args(had, wsb=63) == kvq.KVQ_ERR_WORKSPACE
+
+
+def test_dq_flag_sizes(kvq):
+    nsn_dq = kvq.NSN | kvq.PER_CHANNEL | kvq.DQ
+    assert kvq.kvq_tok_params(nsn_dq) == 1 and kvq.kvq_tok_params(nsn_dq | kvq.HADAMARD) == 1
+    assert kvq.kvq_tok_params(kvq.NORM_SEP | kvq.PER_CHANNEL | kvq.DQ) == -1    # DQ only with NSN
+    for d in (64, 128):
+        assert kvq.kvq_off_words(nsn_dq, d) == oracle.off_words(oracle.NSN | oracle.PER_CHANNEL | oracle.DQ, d)
+        assert kvq.kvq_off_words(nsn_dq, d) * 2 == oracle.dq_record_bytes(d)
+        assert kvq.kvq_off_words(kvq.NSN | kvq.PER_CHANNEL, d) == d
+        assert kvq.kvq_off_words(kvq.NORM_SEP | kvq.PER_CHANNEL, d) == 0
+    assert kvq.kvq_off_words(nsn_dq, 96) == -1
+    assert oracle.ntok(oracle.NSN | oracle.PER_CHANNEL | oracle.DQ) == 1

@@ -19,7 +19,7 @@ from tests.modes import f16bits
 pytestmark = pytest.mark.gpu
 
 ATOL = 2e-3
-MODES = ["nsep+pchan", "naive", "rht+nsep+pchan", "nsn+hadamard", "nsn"]
+MODES = ["nsep+pchan", "naive", "rht+nsep+pchan", "nsn+hadamard", "nsn", "nsn+hadamard+dq"]
 
 
 @pytest.mark.parametrize("mode", MODES)

@@ -35,6 +35,7 @@ CASES = [
     ("llama-long-ctx", "rht+nsep+pchan", 4, 5),
     ("throughput", "nsn+hadamard", 4, 256),
     ("throughput", "nsn+hadamard", 2, 256),
+    ("throughput", "nsn+hadamard+dq", 4, 256),
 ]
 
 

@@ -19,7 +19,7 @@ from tests.modes import f16bits
 pytestmark = pytest.mark.gpu
 
 ATOL = 2e-3
-MODES = ["nsep+pchan", "naive", "rht+nsep+pchan", "nsn+hadamard", "nsn"]
+MODES = ["nsep+pchan", "naive", "rht+nsep+pchan", "nsn+hadamard", "nsn", "nsn+hadamard+dq", "nsn+dq"]
 
 
 def small_workload(mode, d, B=2, H=2, Hq=None, S=384, seed=3):
@@ -100,6 +100,12 @@ DECODE_CASES = [
     # one long pair spread over every CTA of the persistent grid: more than
     # 128 candidate partials per pair in the combine
     ("nsn+hadamard", 128, 4, 1, 1, 4, 200 * 128, 17),
+    # double-quantized NSN side parameters (both decode paths, flushes)
+    ("nsn+hadamard+dq", 128, 4, 2, 2, 8, 512, 140),
+    ("nsn+hadamard+dq", 128, 2, 1, 2, 16, 384, 5),
+    ("nsn+dq", 128, 3, 2, 2, 4, 256, 0),
+    ("nsn+dq", 64, 4, 1, 4, 8, 384, 130),
+    ("nsn+hadamard+dq", 64, 2, 1, 2, 2, 256, 1),
 ]
 
 
