@@ -433,8 +433,9 @@ def run_ours(args, rank: int, world: int):
     q_gbs = q_bytes / q_avg_s / 1e9
     value = world * step_bytes / (ms / 1e3) / 1e9
 
-    int2 = None if (args.no_int2 or world > 1 or BITS != 4 or WORKLOAD != "throughput") else run_int2(w, flags, Kd, Vd, ksd, vsd, qsd, stream,
-                                                                          dev, peak)
+    extra = not (args.no_int2 or world > 1 or BITS != 4 or WORKLOAD != "throughput")
+    int2 = run_variant(w, 2, flags, Kd, Vd, ksd, vsd, qsd, stream, peak) if extra else None
+    dq = run_variant(w, 4, flags | 16, Kd, Vd, ksd, vsd, qsd, stream, peak) if extra and flags & 4 else None
 
     # end to end through the public calls, host buffers, copies inside the region
     ref_last = out.clone()  # the last decode output of the device-resident run
@@ -464,6 +465,7 @@ def run_ours(args, rank: int, world: int):
                      "traffic_source": "profiles/decode_traffic_throughput.md (ncu dram bytes, one call)"},
         "e2e": e2e,
         "int2": int2,
+        "int4_dq": dq,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -480,13 +482,13 @@ def run_ours(args, rank: int, world: int):
     return 0
 
 
-def run_int2(w, flags, Kd, Vd, ksd, vsd, qsd, stream, dev, peak):
-    """The same workload quantized to INT2 codes: quantize of the prefill,
-    the streamed appends, then decode calls at the final length (CUDA events
-    on the launching stream)."""
+def run_variant(w, bits, flags, Kd, Vd, ksd, vsd, qsd, stream, peak):
+    """The same workload with other codes (INT2) or side parameters (DQ):
+    quantize of the prefill, the streamed appends, then decode calls at the
+    final length (CUDA events on the launching stream)."""
     import torch
     from kv_cache_bit_b200 import kvq
-    bits = 2
+    dev = Kd.device
     cap = ((w.S + w.stream + 127) // 128) * 128
     cfg = kvq.Config(w.d, bits, flags, None, device=dev)
     cache = kvq.KVCache.allocate(cfg, w.B, w.Hkv, cap, device=dev)

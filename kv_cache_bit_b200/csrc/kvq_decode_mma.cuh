@@ -340,7 +340,10 @@ struct SlotLayout {
     static constexpr int kOff = kChan + ((MODE != kNaive) ? D * 2 : 0);
     static constexpr int kBytesLo = kOff + ((MODE == kNsn) ? D * 2 : 0);  // first half
     static constexpr int kBytesHi = kChan;                                 // second half
-    static constexpr int kStride = (kBytesLo + 127) / 128 * 128;
+    // DQ: s1 of the unit's 64 tokens as fp32, rebuilt from the record by the
+    // warp once the unit has landed (not a copy target)
+    static constexpr int kS1 = (kBytesLo + 15) / 16 * 16;
+    static constexpr int kStride = (kS1 + (kDq ? kUT * 4 : 0) + 127) / 128 * 128;
     static_assert(kRec % 16 == 0 && kChan % 16 == 0, "bulk copies start on 16-byte boundaries");
 };
 
@@ -355,10 +358,14 @@ __device__ __forceinline__ void dq_o_pairs(const uint8_t* p, __half2 (&o)[8]) {
     }
 }
 
-// s1 of token tok (0..63) of unit half `half` from the record at rec (DQ).
-template <int D>
-__device__ __forceinline__ float dq_s1_unit(const uint8_t* rec, int half, int tok) {
-    return dq_s1<D>(rec, 64 * half + tok);
+// DQ: s1 of the unit's 64 tokens (half `half` of the block) rebuilt from the
+// slot's record into the slot's fp32 s1 area, two tokens per lane.
+template <int D, typename SL>
+__device__ __forceinline__ void dq_fill_s1(uint8_t* slot, int half, int lane) {
+    float* s1 = reinterpret_cast<float*>(slot + SL::kS1);
+    s1[2 * lane] = dq_s1<D>(slot + SL::kRec, 64 * half + 2 * lane);
+    s1[2 * lane + 1] = dq_s1<D>(slot + SL::kRec, 64 * half + 2 * lane + 1);
+    __syncwarp();
 }
 
 // Rotated-query table (fp32): channel c of head j at j * kQS + c + 4 (c / 32).
@@ -619,6 +626,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                 const int uk = 4 * it + 2 * half, uv = uk + 1;
                 if (!wait_unit(uk)) { ok = false; break; }
                 uint8_t* sk = my_ring + (uk % kRing) * SL::kStride;
+                if constexpr (SL::kDq) dq_fill_s1<D, SL>(sk, half, lane);
                 if (half == 0) {
                     // B fragments: q' = qs * sigma^K as (hi, lo) fp16 parts; a
                     // group of PG pairs takes 2 PG channels of the slice
@@ -708,6 +716,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                 }
                 if (!wait_unit(uv)) { ok = false; break; }
                 uint8_t* sv = my_ring + (uv % kRing) * SL::kStride;
+                if constexpr (SL::kDq) dq_fill_s1<D, SL>(sv, half, lane);
                 if (half == 0) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -735,7 +744,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                         const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tv)[tok]);
                         v = s12.x * s12.y * (HAD ? 1.0f : a.sqd);
                     } else if constexpr (MODE == kNsnDq) {
-                        v = dq_s1_unit<D>(sv + SL::kRec, half, tok) * __half2float(tv[tok]) * (HAD ? 1.0f : a.sqd);
+                        v = reinterpret_cast<const float*>(sv + SL::kS1)[tok] * __half2float(tv[tok]) * (HAD ? 1.0f : a.sqd);
                     } else {
                         v = __half2float(tv[tok]) * ((MODE == kNsep && HAD) ? a.rsqd : 1.0f);
                     }
@@ -780,7 +789,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                                 const float2 s12 = __half22float2(reinterpret_cast<const __half2*>(tk)[tok]);
                                 l2[m4][n][r] = s12.x * fmaf(sv_, s12.y * kcol[n], qoK[n]);
                             } else if constexpr (MODE == kNsnDq) {
-                                const float s1 = dq_s1_unit<D>(sk + SL::kRec, half, tok);
+                                const float s1 = reinterpret_cast<const float*>(sk + SL::kS1)[tok];
                                 l2[m4][n][r] = s1 * fmaf(sv_, __half2float(tk[tok]) * kcol[n], qoK[n]);
                             } else {
                                 l2[m4][n][r] = sv_ * (__half2float(tk[tok]) * kcol[n]);
@@ -828,7 +837,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                             s1o = s12.x;
                             nu = s12.x * (s12.y * pscale_m);
                         } else if constexpr (MODE == kNsnDq) {
-                            s1o = dq_s1_unit<D>(sv + SL::kRec, half, tok);
+                            s1o = reinterpret_cast<const float*>(sv + SL::kS1)[tok];
                             nu = s1o * (__half2float(tv[tok]) * pscale_m);
                         } else {
                             nu = __half2float(tv[tok]) * pscale_m;

@@ -308,17 +308,21 @@ __device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
     return r;
 }
 
-// Lane-wise product rounded to fp32 on its own, as two scalar mul.rn.f32:
-// the assembler keeps an explicitly rounded scalar multiply separate, while
-// it may fuse a packed mul.rn.f32x2 with the add or subtract that consumes
-// it into one fused multiply-add (one rounding instead of two).  Every
-// product that feeds an add whose operands are not exact products uses this.
-__device__ __forceinline__ f2_t f2_mul_sep(f2_t a, f2_t b) {
+// Lane-wise product rounded to fp32 on its own.  The assembler may fuse a
+// packed mul.rn.f32x2 with the add or subtract that consumes it into one
+// fused multiply-add (one rounding instead of two), and it also did so for
+// an FMA whose addend was the literal -0.  So the product is an FMA whose
+// addend nz is the pair (-0, -0) loaded from constant memory, a value the
+// assembler cannot assume: a * b + (-0) rounds the exact product once (zero
+// signs included), and an FMA is not fused again.  Every product that feeds
+// an add whose operands are not exact products uses this.
+__constant__ float g_neg_zero[2] = {-0.0f, -0.0f};
+
+__device__ __forceinline__ f2_t neg_zero2() { return *reinterpret_cast<const f2_t*>(g_neg_zero); }
+
+__device__ __forceinline__ f2_t f2_mul_sep(f2_t a, f2_t b, f2_t nz) {
     f2_t r;
-    asm("{\n .reg .f32 a0, a1, b0, b1, r0, r1;\n mov.b64 {a0, a1}, %1;\n mov.b64 {b0, b1}, %2;\n"
-        " mul.rn.f32 r0, a0, b0;\n mul.rn.f32 r1, a1, b1;\n mov.b64 %0, {r0, r1};\n}"
-        : "=l"(r)
-        : "l"(a), "l"(b));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(nz));
     return r;
 }
 
@@ -340,17 +344,18 @@ __device__ __forceinline__ f2_t f2_add_ordered(f2_t a, f2_t b) {
 // fused square-and-add rounds like the separate operations and the packed
 // multiply may be used; otherwise the squares are rounded on their own.
 template <int OFF, int N, int H2, bool EXACT>
-__device__ __forceinline__ f2_t pw_sumsq2(const f2_t (&P)[H2]) {
-    if constexpr (N == 1) return EXACT ? f2_mul_ordered(P[OFF], P[OFF]) : f2_mul_sep(P[OFF], P[OFF]);
-    else return f2_add_ordered(pw_sumsq2<OFF, N / 2, H2, EXACT>(P), pw_sumsq2<OFF + N / 2, N / 2, H2, EXACT>(P));
+__device__ __forceinline__ f2_t pw_sumsq2(const f2_t (&P)[H2], f2_t nz) {
+    if constexpr (N == 1) return EXACT ? f2_mul_ordered(P[OFF], P[OFF]) : f2_mul_sep(P[OFF], P[OFF], nz);
+    else
+        return f2_add_ordered(pw_sumsq2<OFF, N / 2, H2, EXACT>(P, nz), pw_sumsq2<OFF + N / 2, N / 2, H2, EXACT>(P, nz));
 }
 
 // Pairwise sum of squares of the whole row: the top split of the halving
-// tree adds the two lanes.
+// tree adds the two lanes.  nz: see f2_mul_sep (unused when EXACT).
 template <int H2, bool EXACT>
-__device__ __forceinline__ float row_sumsq(const f2_t (&P)[H2]) {
+__device__ __forceinline__ float row_sumsq(const f2_t (&P)[H2], f2_t nz) {
     float lo, hi;
-    f2_unpack(pw_sumsq2<0, H2, H2, EXACT>(P), lo, hi);
+    f2_unpack(pw_sumsq2<0, H2, H2, EXACT>(P, nz), lo, hi);
     return __fadd_rn(lo, hi);
 }
 
@@ -462,9 +467,29 @@ __device__ __forceinline__ void pack_codes(const uint32_t (&cw)[D], uint32_t (&w
 
 // ---------------------------------------------------------------- the quantizer
 
+// NSN block means: from the fp16 tile with the row still in its fp16 form
+// (two tile regions, three CTAs per SM), or from the fp32 rows through a
+// transposed buffer (three regions, two CTAs per SM).
+#ifndef KVQ_NSN_TILE_MEANS
+#define KVQ_NSN_TILE_MEANS 1
+#endif
+constexpr bool kNsnTileMeans = KVQ_NSN_TILE_MEANS != 0;
+
 // Bytes of the per-token-group partials: the NSN column sums are
 // (128 / (D / 8)) groups x D floats, the per-channel maxima half of that.
-constexpr int kGpartBytes = 4096;
+constexpr int kGpartBytes = 4096 + 512;  // group sums / warp maxima, then the DQ scratch
+
+// Output pointers of one (tensor, batch, head, block).
+struct QuantOut {
+    uint8_t* codes;  // [128][row_bytes] rows of this block
+    uint8_t* stage;  // if set, codes go here instead, for a TMA store: row t at t * row_bytes,
+                     // 16-byte chunk c at chunk c ^ ((t >> 1) & 3) (INT4, 64-byte swizzle) or
+                     // c ^ ((t >> 2) & 1) (INT2, 32-byte swizzle)
+    __half* tok;     // [128][ntok]
+    __half* chan;    // [D] (PER_CHANNEL)
+    __half* off;     // [D] (NSN)
+    bool pairv;      // V codes of head dim 128: pair-interleaved rows
+};
 
 // Shared-memory scratch of one quantizer CTA.
 template <int D>
@@ -481,6 +506,7 @@ struct QuantSmem {
     float* gpart;    // [4 KB] per-token-group partial sums (NSN means), then per-warp maxima
     float* tokv;     // [128] a per-token scalar (NSN 1/||x|| * sqrt(d))
     uint32_t* sgn2;  // [D/2] fp16x2 sign masks of channels (2i, 2i+1)
+    QuantOut* out;   // the current block's output pointers
 };
 
 // Widen 8 fp16 channels of the low half (lo) and the matching 8 of the high
@@ -525,17 +551,6 @@ __host__ __device__ constexpr bool pairv_layout() { return D == 128; }
 template <int BITS>
 __host__ __device__ constexpr int pairv_chunk_xor(int k) { return BITS == 4 ? 2 * (k & 1) : 0; }
 
-// Output pointers of one (tensor, batch, head, block).
-struct QuantOut {
-    uint8_t* codes;  // [128][row_bytes] rows of this block
-    uint8_t* stage;  // if set, codes go here instead, for a TMA store: row t at t * row_bytes,
-                     // 16-byte chunk c at chunk c ^ ((t >> 1) & 3) (INT4, 64-byte swizzle) or
-                     // c ^ ((t >> 2) & 1) (INT2, 32-byte swizzle)
-    __half* tok;     // [128][ntok]
-    __half* chan;    // [D] (PER_CHANNEL)
-    __half* off;     // [D] (NSN)
-    bool pairv;      // V codes of head dim 128: pair-interleaved rows
-};
 
 // Row t of packed codes: straight to global memory, or into the swizzled
 // staging tile of a TMA store (then visible to the async proxy).
@@ -602,12 +617,11 @@ __device__ __forceinline__ uint16_t sign16(const uint32_t* sgn2, int c) {
     return (uint16_t)((sgn2[c >> 1] >> ((c & 1) * 16)) & 0x8000u);
 }
 
-// 8-byte shared-memory load kept in program order (volatile), so that a loop
-// of them does not have all its loads hoisted ahead of their uses.
-__device__ __forceinline__ f2_t lds_f2(uint32_t addr) {
-    f2_t r;
-    asm volatile("ld.shared.b64 %0, [%1];" : "=l"(r) : "r"(addr));
-    return r;
+// 16-byte shared-memory load of two pairs kept in program order (volatile),
+// so that a loop of them does not have all its loads hoisted ahead of their
+// uses.
+__device__ __forceinline__ void lds_f2x2(uint32_t addr, f2_t& a, f2_t& b) {
+    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr));
 }
 
 // min / max over the warp's lanes of x (exact).
@@ -749,13 +763,15 @@ __device__ __forceinline__ void quantize_rows(uint4 (&raw)[D / 8], const int t, 
 
     if constexpr (is_nsn(MODE)) {
         constexpr bool DQ = MODE == kNsnDq;
-        // DQ scratch past the group sums: [0, 4) warp minima of s1, [4, 8)
-        // warp maxima, [8, 8 + D/32) warp maxima of |o|, then the o codes
-        float* dqs = sm.gpart + 768;
+        const f2_t NZ = neg_zero2();
+        // DQ scratch past the group sums (4 KB): [0, 4) warp minima of s1,
+        // [4, 8) warp maxima, [8, 8 + D/32) warp maxima of |o|, then the o codes
+        float* dqs = sm.gpart + 1024;
         uint8_t* dq_e = reinterpret_cast<uint8_t*>(dqs + 16);
         const float n1 = __fsqrt_rn(raw_row_sumsq<D>(raw));
         const float s1 = __fmul_rn(n1, rsqd);
         const float r1 = n1 > 0.0f ? __fdiv_rn(sqd, n1) : 0.0f;
+        const f2_t R1 = f2_pack(r1, r1);
         if constexpr (DQ) {
             const float mn = warp_min(s1), mx = warp_max(s1);
             if ((t & 31) == 0) {
@@ -763,64 +779,116 @@ __device__ __forceinline__ void quantize_rows(uint4 (&raw)[D / 8], const int t, 
                 dqs[4 + (t >> 5)] = mx;
             }
         }
-        // a = x * r1, with the rotation's signs when SIGNS
-        widen_row<D, SIGNS>(raw, sm, P);
-        const f2_t R1 = f2_pack(r1, r1);
+        if constexpr (kNsnTileMeans) {
+            // block means of a = x * r1 from the fp16 tile (unsigned values,
+            // the same separately rounded products as the rows'), while the
+            // row waits in its fp16 form: thread t sums the 8 channels of
+            // chunk column kc8 over the TGC tokens of group gc in the
+            // pairwise (binary-counter) order
+            sm.tokv[t] = r1;
+            __syncthreads();
+            constexpr int NKC = D / 8, NGC = kT / NKC, TGC = kT / NGC;
+            static_assert(NGC * D * 4 <= 4096, "group sums fit below the DQ scratch");
+            constexpr int LV = (TGC == 16) ? 4 : 3;  // log2 TGC
+            const int kc8 = t % NKC, gc = t / NKC;
+            const uint8_t* colp = sm.tile + (kc8 / 8) * (kT * 128);
+            const int ck = kc8 % 8;
+            f2_t acc[4][LV];
+            f2_t cur[4];
 #pragma unroll
-        for (int j = 0; j < H2; ++j) P[j] = f2_mul_sep(P[j], R1);
-        before_spill();
-        __syncthreads();  // every row has been read from the tile region
-        {
-            // the rows of a into the transposed buffer
-            constexpr int NCH2 = D / 8;  // 16-byte chunks (two pairs) per half row
-            char* lo = reinterpret_cast<char*>(sm.red_lo) + (size_t)t * (D / 2) * 4;
-            char* hi = reinterpret_cast<char*>(sm.red_hi) + (size_t)t * (D / 2) * 4;
+            for (int i = 0; i < TGC; ++i) {
+                const int tt = gc * TGC + i;
+                const uint4 xr = *reinterpret_cast<const uint4*>(colp + tt * 128 + ((ck ^ (tt & 7)) << 4));
+                const float rt = sm.tokv[tt];
+                const f2_t RT = f2_pack(rt, rt);
+                const __half2* hp = reinterpret_cast<const __half2*>(&xr);
 #pragma unroll
-            for (int k = 0; k < 2 * NCH2; ++k) {
-                const int pk = (k % NCH2) ^ (t & (NCH2 - 1));
-                *reinterpret_cast<ulonglong2*>((k < NCH2 ? lo : hi) + pk * 16) = make_ulonglong2(P[2 * k], P[2 * k + 1]);
-            }
-        }
-        __syncthreads();
-        {
-            // block means: thread t sums chunk column kc (pairs 2 kc, 2 kc + 1)
-            // over the TG tokens of group g in the pairwise (binary-counter)
-            // order; the NG group sums meet in the top levels of the tree
-            constexpr int NCH2 = D / 8, NCH = 2 * NCH2, TG = NCH, NG = kT / TG;
-            static_assert(NG * D * 4 <= kGpartBytes, "group sums fit the partials buffer");
-            constexpr int LV = (TG == 32) ? 5 : 4;  // log2 TG
-            const int kc = t % NCH, g = t / NCH;
-            const char* base = reinterpret_cast<const char*>(kc < NCH2 ? sm.red_lo : sm.red_hi) +
-                               (size_t)g * TG * (D / 2) * 4;
-            const int kh = kc % NCH2;
-            f2_t acc[2][LV];
-            f2_t cur[2];
-#pragma unroll
-            for (int i = 0; i < TG; ++i) {
-                const int tt = g * TG + i;
-                const ulonglong2 x =
-                    *reinterpret_cast<const ulonglong2*>(base + (size_t)i * (D / 2) * 4 + ((kh ^ (tt & (NCH2 - 1))) << 4));
-                cur[0] = x.x;
-                cur[1] = x.y;
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = __half22float2(hp[e]);
+                    cur[e] = f2_mul_sep(f2_pack(x.x, x.y), RT, NZ);
+                }
 #pragma unroll
                 for (int l = 0; l < LV; ++l) {
                     if ((i >> l) & 1) {
-                        cur[0] = f2_add(acc[0][l], cur[0]);
-                        cur[1] = f2_add(acc[1][l], cur[1]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) cur[e] = f2_add(acc[e][l], cur[e]);
                     } else {
-                        acc[0][l] = cur[0];
-                        acc[1][l] = cur[1];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[e][l] = cur[e];
                         break;
                     }
                 }
             }
-            // cur: the sum over the group (pair order index 4 kc .. 4 kc + 3)
-            *reinterpret_cast<ulonglong2*>(sm.gpart + g * D + 4 * kc) = make_ulonglong2(cur[0], cur[1]);
+            // cur: channels 8 kc8 .. 8 kc8 + 7 of the group; into pair order
+            // (index 2 (c mod D/2) + c / (D/2)) for the combine below
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float lo, hi;
+                f2_unpack(cur[e], lo, hi);
+                const int c = 8 * kc8 + 2 * e;
+                sm.gpart[gc * D + 2 * (c % (D / 2)) + c / (D / 2)] = lo;
+                sm.gpart[gc * D + 2 * ((c + 1) % (D / 2)) + (c + 1) / (D / 2)] = hi;
+            }
+        } else {
+            // a = x * r1, with the rotation's signs when SIGNS
+            widen_row<D, SIGNS>(raw, sm, P);
+#pragma unroll
+            for (int j = 0; j < H2; ++j) P[j] = f2_mul_sep(P[j], R1, NZ);
+            before_spill();
+            __syncthreads();  // every row has been read from the tile region
+            {
+                // the rows of a into the transposed buffer
+                constexpr int NCH2 = D / 8;  // 16-byte chunks (two pairs) per half row
+                char* lo = reinterpret_cast<char*>(sm.red_lo) + (size_t)t * (D / 2) * 4;
+                char* hi = reinterpret_cast<char*>(sm.red_hi) + (size_t)t * (D / 2) * 4;
+#pragma unroll
+                for (int k = 0; k < 2 * NCH2; ++k) {
+                    const int pk = (k % NCH2) ^ (t & (NCH2 - 1));
+                    *reinterpret_cast<ulonglong2*>((k < NCH2 ? lo : hi) + pk * 16) =
+                        make_ulonglong2(P[2 * k], P[2 * k + 1]);
+                }
+            }
+            __syncthreads();
+            {
+                // block means: thread t sums chunk column kc (pairs 2 kc, 2 kc + 1)
+                // over the TG tokens of group g in the pairwise (binary-counter)
+                // order; the NG group sums meet in the top levels of the tree
+                constexpr int NCH2 = D / 8, NCH = 2 * NCH2, TG = NCH, NG = kT / TG;
+                static_assert(NG * D * 4 <= 4096, "group sums fit below the DQ scratch");
+                constexpr int LV = (TG == 32) ? 5 : 4;  // log2 TG
+                const int kc = t % NCH, g = t / NCH;
+                const char* base = reinterpret_cast<const char*>(kc < NCH2 ? sm.red_lo : sm.red_hi) +
+                                   (size_t)g * TG * (D / 2) * 4;
+                const int kh = kc % NCH2;
+                f2_t acc[2][LV];
+                f2_t cur[2];
+#pragma unroll
+                for (int i = 0; i < TG; ++i) {
+                    const int tt = g * TG + i;
+                    const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(base + (size_t)i * (D / 2) * 4 +
+                                                                               ((kh ^ (tt & (NCH2 - 1))) << 4));
+                    cur[0] = x.x;
+                    cur[1] = x.y;
+#pragma unroll
+                    for (int l = 0; l < LV; ++l) {
+                        if ((i >> l) & 1) {
+                            cur[0] = f2_add(acc[0][l], cur[0]);
+                            cur[1] = f2_add(acc[1][l], cur[1]);
+                        } else {
+                            acc[0][l] = cur[0];
+                            acc[1][l] = cur[1];
+                            break;
+                        }
+                    }
+                }
+                // cur: the sum over the group (pair order index 4 kc .. 4 kc + 3)
+                *reinterpret_cast<ulonglong2*>(sm.gpart + g * D + 4 * kc) = make_ulonglong2(cur[0], cur[1]);
+            }
         }
         __syncthreads();
         if (t < D) {
             // pair-order index t: channel c = pair t >> 1 of half t & 1
-            constexpr int NG = kT / (D / 4);
+            constexpr int NG = kNsnTileMeans ? kT / (D / 8) : kT / (D / 4);
             float gs[NG];
 #pragma unroll
             for (int k = 0; k < NG; ++k) gs[k] = sm.gpart[k * D + t];
@@ -830,9 +898,11 @@ __device__ __forceinline__ void quantize_rows(uint4 (&raw)[D / 8], const int t, 
                 for (int k = 0; k < NG; k += 2 * w) gs[k] = __fadd_rn(gs[k], gs[k + w]);
             }
             // the mean of the signed rows; the stored mean is of the unsigned
-            // ones (a sign flip commutes exactly with the sum and the rounding)
-            const float of = __fmul_rn(gs[0], 1.0f / 128.0f);
+            // ones (a sign flip commutes exactly with the sum and the rounding);
+            // the tile holds the unsigned values
             const int c = (t >> 1) + (t & 1) * H2;
+            float of = __fmul_rn(gs[0], 1.0f / 128.0f);
+            if (kNsnTileMeans && SIGNS && sign16(sm.sgn2, c)) of = -of;
             if constexpr (DQ) {
                 sm.vec[t] = of;
                 const float m = warp_max_abs(of);
@@ -892,18 +962,29 @@ __device__ __forceinline__ void quantize_rows(uint4 (&raw)[D / 8], const int t, 
         }
         __syncthreads();
         after_means();  // the transposed buffer is free again
+        if constexpr (kNsnTileMeans) {
+            // a = x * r1 (the row leaves its fp16 form only now)
+            widen_row<D, SIGNS>(raw, sm, P);
+#pragma unroll
+            for (int j = 0; j < H2; ++j) P[j] = f2_mul_sep(P[j], R1, NZ);
+        }
         // b = a - s (.) o
         const uint32_t mv = smem_u32(sm.vec);
 #pragma unroll
-        for (int j = 0; j < H2; ++j) P[j] = f2_sub(P[j], lds_f2(mv + 8 * j));
-        const float n2 = __fsqrt_rn(row_sumsq<H2, false>(P));
+        for (int j = 0; j < H2; j += 2) {
+            f2_t m0, m1;
+            lds_f2x2(mv + 8 * j, m0, m1);
+            P[j] = f2_sub(P[j], m0);
+            P[j + 1] = f2_sub(P[j + 1], m1);
+        }
+        const float n2 = __fsqrt_rn(row_sumsq<H2, false>(P, NZ));
         const float s2 = __fmul_rn(n2, rsqd);
         kscale = n2 > 0.0f ? __fdiv_rn(c0, n2) : 0.0f;
         if constexpr (DQ) out.tok[t] = __float2half_rn(s2);
         else reinterpret_cast<__half2*>(out.tok)[t] = __halves2half2(__float2half_rn(s1), __float2half_rn(s2));
     } else if constexpr (MODE == kNsep) {
         widen_row<D, SIGNS>(raw, sm, P);
-        const float n = __fsqrt_rn(row_sumsq<H2, true>(P));
+        const float n = __fsqrt_rn(row_sumsq<H2, true>(P, f2_t(0)));
         out.tok[t] = __float2half_rn(n);
         kscale = n > 0.0f ? __fdiv_rn(c0, n) : 0.0f;
     } else {

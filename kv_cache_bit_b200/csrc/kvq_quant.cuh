@@ -28,7 +28,7 @@ struct QuantArgs {
 // transposed buffer) while the third receives the next tile.
 template <int MODE>
 __host__ __device__ constexpr int quant_regions() {
-    return is_nsn(MODE) ? 3 : 2;
+    return (is_nsn(MODE) && !kNsnTileMeans) ? 3 : 2;
 }
 
 template <int D>
@@ -40,7 +40,7 @@ template <int D, int MODE>
 __host__ __device__ constexpr int quant_smem_bytes() {
     // 1024 B alignment slack + regions + vec + group partials + token vector + sign masks + mbarriers
     return 1024 + quant_regions<MODE>() * quant_region_bytes<D>() + D * 4 + kGpartBytes + kT * 4 + D * 4 +
-           quant_regions<MODE>() * 8;
+           quant_regions<MODE>() * 8 + 64;
 }
 
 // Resident quantizer CTAs per SM the register budget is set for: a thread
@@ -49,7 +49,7 @@ __host__ __device__ constexpr int quant_smem_bytes() {
 // registers than three CTAs leave; those run two CTAs per SM.
 template <int D, int BITS, int MODE, bool HAD>
 __host__ __device__ constexpr int quant_min_ctas() {
-    return D == 128 ? ((is_nsn(MODE) || (HAD && BITS == 3)) ? 2 : 3) : 4;
+    return D == 128 ? (((is_nsn(MODE) && !kNsnTileMeans) || (HAD && BITS == 3)) ? 2 : 3) : 4;
 }
 
 template <int D, int MODE>
@@ -72,6 +72,8 @@ __device__ __forceinline__ QuantSmem<D> carve_quant_smem(uint8_t* base, uint64_t
     sm.sgn2 = reinterpret_cast<uint32_t*>(p);
     p += D * 4;
     bar = reinterpret_cast<uint64_t*>(p);
+    p += quant_regions<MODE>() * 8;
+    sm.out = reinterpret_cast<QuantOut*>(p);
     return sm;
 }
 
@@ -182,6 +184,15 @@ __global__ void __launch_bounds__(128, (quant_min_ctas<D, BITS, MODE, HAD>())) q
                 issue(w + stride, reg ^ 1);
             }
         }
+        if (t == 0) {
+            // the item's output pointers, published by the barrier below (the
+            // threads read them from shared memory where they are used)
+            const int r = w >> 1;
+            const int bh = r / nblk, blk = r - bh * nblk;
+            QuantOut o = quant_out<D, BITS, MODE, HAD>(a, w & 1, bh, a.blk0 + blk);
+            if constexpr (kTmaStore) o.stage = regions + reg * kTileBytes;
+            *sm.out = o;
+        }
         const bool landed = mbar_wait(&bar[reg], (phases >> reg) & 1, KVQ_WAIT_LIMIT(1u << 24));
         if (__syncthreads_or(!landed)) {
             if (t == 0) report_error(kErrTmaTimeout);
@@ -198,8 +209,7 @@ __global__ void __launch_bounds__(128, (quant_min_ctas<D, BITS, MODE, HAD>())) q
         const int bh = r / nblk, blk = r - bh * nblk;
         uint4 raw[D / 8];
         load_tile_raw<D>(tile, t, raw);
-        QuantOut out = quant_out<D, BITS, MODE, HAD>(a, tensor, bh, a.blk0 + blk);
-        if constexpr (kTmaStore) out.stage = tile;
+        const QuantOut& out = *sm.out;
         // NSN: the spare region is written once the previous item's code store
         // has read it, and takes item w + 2 stride after the means
         auto before_spill = [&] {
@@ -264,8 +274,18 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
     const __half* src = (t == kT - 1) ? xn : res + (size_t)t * D;
     uint4 raw[D / 8];
 #pragma unroll
-    for (int q = 0; q < D / 8; ++q) raw[q] = reinterpret_cast<const uint4*>(src)[q];
-    const QuantOut out = quant_out<D, BITS, MODE, HAD>(a.q, tensor, bh, a.blk);
+    for (int q = 0; q < D / 8; ++q) {
+        raw[q] = reinterpret_cast<const uint4*>(src)[q];
+        if constexpr (is_nsn(MODE) && kNsnTileMeans) {
+            // the fp16 tile in the quantize kernel's layout, for the block means
+            const int c = 8 * q;
+            *reinterpret_cast<uint4*>(regions + (c / 64) * (kT * 128) + t * 128 + ((((c % 64) / 8) ^ (t & 7)) << 4)) =
+                raw[q];
+        }
+    }
+    if (t == 0) *sm.out = quant_out<D, BITS, MODE, HAD>(a.q, tensor, bh, a.blk);
+    __syncthreads();
+    const QuantOut& out = *sm.out;
     auto none = [] {};
     if (HAD && a.q.signs != nullptr)
         quantize_rows<D, BITS, MODE, HAD, true>(raw, t, sm, out, a.q.rsqd, a.q.sqd, none, none);
@@ -437,14 +457,27 @@ __global__ void __launch_bounds__(128) select_signs_kernel(SelectArgs a) {
     const __half* xr = a.x + ((size_t)blk * kT + t) * D;
     uint4 raw[D / 8];
 #pragma unroll
-    for (int q = 0; q < D / 8; ++q) raw[q] = reinterpret_cast<const uint4*>(xr)[q];
-    QuantOut out;
-    out.codes = s_codes;
-    out.stage = nullptr;
-    out.tok = s_tok;
-    out.chan = s_chan;
-    out.off = s_off16;
-    out.pairv = false;
+    for (int q = 0; q < D / 8; ++q) {
+        raw[q] = reinterpret_cast<const uint4*>(xr)[q];
+        if constexpr (is_nsn(MODE) && kNsnTileMeans) {
+            // the fp16 tile in the quantize kernel's layout, for the block means
+            const int c = 8 * q;
+            *reinterpret_cast<uint4*>(regions + (c / 64) * (kT * 128) + t * 128 + ((((c % 64) / 8) ^ (t & 7)) << 4)) =
+                raw[q];
+        }
+    }
+    if (t == 0) {
+        QuantOut o;
+        o.codes = s_codes;
+        o.stage = nullptr;
+        o.tok = s_tok;
+        o.chan = s_chan;
+        o.off = s_off16;
+        o.pairv = false;
+        *sm.out = o;
+    }
+    __syncthreads();
+    const QuantOut& out = *sm.out;
     auto none = [] {};
     quantize_rows<D, BITS, MODE, true, true>(raw, t, sm, out, a.rsqd, a.sqd, none, none);
     __syncthreads();
