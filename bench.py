@@ -47,7 +47,9 @@ WORKLOAD_MODES = {"tiny": "nsep+pchan", "qwen2-7b-gqa": "nsep+pchan", "pythia-6.
 METRIC = "INT4-KV decode attention GB/s (% of HBM peak) & tokens/s; quantize GB/s"
 
 
-KERNEL_SOURCES = ["kvq_api.cu", "kvq_decode_mma.cuh", "kvq_decode_simple.cuh", "kvq_device.cuh", "kvq_quant.cuh"]
+# The sources the decode kernels are built from (the host file holds their
+# launch configuration); the quantizer's own files are not among them.
+KERNEL_SOURCES = ["kvq_api.cu", "kvq_decode_mma.cuh", "kvq_decode_simple.cuh", "kvq_device.cuh"]
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "decode_traffic_throughput.md")
 
 

@@ -2,7 +2,7 @@
 // kernels (sm_100a).  Included once, by kvq_api.cu.
 #pragma once
 
-#include "kvq_device.cuh"
+#include "kvq_quant_rows.cuh"
 
 namespace kvq {
 
