@@ -94,6 +94,15 @@ __device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
+// D = A * B + C with C = (c0, c1) on row g and (c2, c3) on row g + 8.
+__device__ __forceinline__ void mma16816_c4(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1, float c0, float c1, float c2, float c3) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2), "f"(c3));
+}
+
 // D = A * B + C with the same C pair (c0, c1) on rows g and g + 8.
 __device__ __forceinline__ void mma16816_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                            uint32_t b0, uint32_t b1, float c0, float c1) {
@@ -148,14 +157,22 @@ __device__ __forceinline__ uint32_t h2c(float v) { return pack_h2(v, v); }
 template <int BITS>
 struct KUnpack;
 
-// INT4: a low nibble OR-ed into fp16 1024 reads 1024 + e, and one
-// subtraction gives q = e - 8.  A high nibble (bits 4..7 of its byte) OR-ed
-// into 1024 reads 1024 + 16 e = 16 (q + 72) and is used in that biased form,
-// one LOP3 per pair with no fp16 arithmetic (kBiased): the kernel scales the
-// other operand of those channels by 1/16 and removes the bias 1152 = 16 * 72
-// times the sum of that operand: for the scores with one MMA against a
-// constant A of -1152 per block, for the values from the unit's sum of P'.
-constexpr float kBiasA = -1152.0f;
+// INT4: the offset-binary code e = q + 8 of a nibble is used in place, as an
+// fp16 subnormal: a low nibble masked out of its 16-bit half reads
+// e * 2^-24, a high nibble (bits 4..7 of its byte) 16 e * 2^-24, one LOP3 per
+// pair and no fp16 arithmetic (kBiased).  The kernel scales the other
+// operand of the high-nibble channels by 1/16, folds 2^24 into the scales it
+// applies to the fp32 results, and removes the bias 8 times the sum of the
+// other operand: for the scores with one MMA chain per block against a
+// constant A of -8 * 2^-24 (low) and -128 * 2^-24 (high nibbles), for the
+// values from the unit's sum of P'.  Subnormal fp16 inputs are exact values;
+// the tensor core's sum of such products measured within 2^-19 of the sum
+// of their magnitudes (against 2^-23 for normal inputs), which the bias
+// (|e| <= 15 against |q| <= 7) costs about one bit of.
+constexpr uint32_t kBiasLoH2 = 0x80088008u;  // fp16x2 -8 * 2^-24
+constexpr uint32_t kBiasHiH2 = 0x80808080u;  // fp16x2 -128 * 2^-24
+constexpr float kTwo24 = 16777216.0f;        // 2^24
+constexpr float kBiasV = -8.0f / 16777216.0f;  // -8 * 2^-24
 
 template <>
 struct KUnpack<4> {
@@ -163,19 +180,18 @@ struct KUnpack<4> {
     static constexpr bool kBiased = true;
     __device__ static int ca(int p) { return 8 * (p >> 2) + (p & 3); }
     __device__ static int cb(int p) { return ca(p) + 4; }
-    // row points at the row's first byte; even pairs p hold q = e - 8, odd
-    // pairs (high nibbles) 16 (q + 72)
+    // row points at the row's first byte; even pairs p hold e * 2^-24, odd
+    // pairs (high nibbles) 16 e * 2^-24
     __device__ static void run(const uint8_t* row, int t, uint32_t (&pr)[16]) {
         const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * t);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        const uint32_t sub = h2c(1032.0f);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t W = w[i], W8 = w[i] >> 8;
-            pr[4 * i + 0] = h2_sub(lop_and_or(W, 0x000F000Fu, kMagic), sub);
-            pr[4 * i + 1] = lop_and_or(W, 0x00F000F0u, kMagic);
-            pr[4 * i + 2] = h2_sub(lop_and_or(W8, 0x000F000Fu, kMagic), sub);
-            pr[4 * i + 3] = lop_and_or(W8, 0x00F000F0u, kMagic);
+            pr[4 * i + 0] = W & 0x000F000Fu;
+            pr[4 * i + 1] = W & 0x00F000F0u;
+            pr[4 * i + 2] = W8 & 0x000F000Fu;
+            pr[4 * i + 3] = W8 & 0x00F000F0u;
         }
     }
 };
@@ -261,20 +277,19 @@ struct VUnpack;
 
 template <>
 struct VUnpack<4> {
-    static constexpr bool kBiased = true;  // odd channels (high nibbles) as 16 (q + 72)
+    static constexpr bool kBiased = true;  // e * 2^-24; odd channels (high nibbles) 16 e * 2^-24
     // units 4g .. 4g + 3: the 16-byte chunk g, at g ^ (2 (k & 1))
     __device__ static void run(const uint8_t* pb, int k, int g, uint32_t (&pr)[16]) {
         const uint4 v = *reinterpret_cast<const uint4*>(pb + 16 * (g ^ pairv_chunk_xor<4>(k)));
         const uint32_t x4[4] = {v.x, v.y, v.z, v.w};
-        const uint32_t sub = h2c(1032.0f);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             // unit 4g + i of both rows: channels 16g + 4i .. + 3
             const uint32_t x = x4[i], x8 = x >> 8;
-            pr[4 * i + 0] = h2_sub(lop_and_or(x, 0x000F000Fu, kMagic), sub);
-            pr[4 * i + 1] = lop_and_or(x, 0x00F000F0u, kMagic);
-            pr[4 * i + 2] = h2_sub(lop_and_or(x8, 0x000F000Fu, kMagic), sub);
-            pr[4 * i + 3] = lop_and_or(x8, 0x00F000F0u, kMagic);
+            pr[4 * i + 0] = x & 0x000F000Fu;
+            pr[4 * i + 1] = x & 0x00F000F0u;
+            pr[4 * i + 2] = x8 & 0x000F000Fu;
+            pr[4 * i + 3] = x8 & 0x00F000F0u;
         }
     }
 };
@@ -463,7 +478,6 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
     constexpr int QMAX = (1 << (BITS - 1)) - 1;
     constexpr float kTau = 8.0f;  // reference-max slack (log2 units): p <= 2^kTau
     constexpr bool KB = KUnpack<BITS>::kBiased, VB = VUnpack<BITS>::kBiased;
-    const uint32_t kBiasH2 = h2c(kBiasA);
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     grid_dep_launch();
@@ -610,7 +624,7 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
             // 2^-qsc with the softmax scale (log2 units) and the fixed token
             // factor of the mode folded in
             kcol[n] = alpha2 * ((is_nsn(MODE) && !HAD) ? a.sqd : (MODE == kNsep && HAD) ? a.rsqd : 1.0f) /
-                      wqsc[4 * n + t];
+                      wqsc[4 * n + t] * (KB ? kTwo24 : 1.0f);
 #pragma unroll
             for (int k = 0; k < 16; ++k) { acc[n][k] = 0.0f; acco[n][k] = 0.0f; }
         }
@@ -670,17 +684,18 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                         }
                     }
                     if constexpr (KB) {
-                        // bias of the score chains: A = 0 on the even pairs of
-                        // a k-step (a0, a1), -1152 on the odd ones (a2, a3)
+                        // bias of the score chains: A = -8 * 2^-24 on the even
+                        // pairs of a k-step (a0, a1), -128 * 2^-24 on the odd
+                        // ones (a2, a3), whose B carries 1/16
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
                             float c0[4], c1[4];
-                            mma16816_z(c0, 0u, 0u, kBiasH2, kBiasH2, bq[n][0], bq[n][1]);
-                            mma16816_z(c1, 0u, 0u, kBiasH2, kBiasH2, bq[n][2], bq[n][3]);
+                            mma16816_z(c0, kBiasLoH2, kBiasLoH2, kBiasHiH2, kBiasHiH2, bq[n][0], bq[n][1]);
+                            mma16816_z(c1, kBiasLoH2, kBiasLoH2, kBiasHiH2, kBiasHiH2, bq[n][2], bq[n][3]);
 #pragma unroll
                             for (int s = 2; s < 8; s += 2) {
-                                mma16816(c0, 0u, 0u, kBiasH2, kBiasH2, bq[n][2 * s], bq[n][2 * s + 1]);
-                                mma16816(c1, 0u, 0u, kBiasH2, kBiasH2, bq[n][2 * s + 2], bq[n][2 * s + 3]);
+                                mma16816(c0, kBiasLoH2, kBiasLoH2, kBiasHiH2, kBiasHiH2, bq[n][2 * s], bq[n][2 * s + 1]);
+                                mma16816(c1, kBiasLoH2, kBiasLoH2, kBiasHiH2, kBiasHiH2, bq[n][2 * s + 2], bq[n][2 * s + 3]);
                             }
                             kb[n][0] = c0[0] + c1[0];
                             kb[n][1] = c0[1] + c1[1];
@@ -853,6 +868,19 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                         }
                     }
                 }
+                // biased INT4 codes: the bias (8 e-units per code, scaled like
+                // the codes) enters the value chains as their starting C, from
+                // the unit's sum of P' (rows g: low nibbles, g + 8: high)
+                float vlo[NT], vhi[NT];
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    if constexpr (VB) {
+#pragma unroll
+                        for (int o = 4; o < 32; o <<= 1) psum[n] += __shfl_xor_sync(0xffffffffu, psum[n], o);
+                    }
+                    vlo[n] = VB ? kBiasV * psum[n] : 0.0f;
+                    vhi[n] = VB ? (16.0f * kBiasV) * psum[n] : 0.0f;
+                }
 #pragma unroll
                 for (int m4 = 0; m4 < 4; ++m4) {
                     const uint32_t (&bp)[NT][2] = bpa[m4];
@@ -866,7 +894,10 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                     for (int tc = 0; tc < 8; ++tc) {
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
-                            if (m4 == 0)
+                            if (m4 == 0 && VB)
+                                mma16816_c4(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1],
+                                            bp[n][0], bp[n][1], vlo[n], 0.0f, vhi[n], 0.0f);
+                            else if (m4 == 0)
                                 mma16816_z(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1],
                                            bp[n][0], bp[n][1]);
                             else
@@ -877,30 +908,19 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                 }
 #pragma unroll
                 for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
-                // unit epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f
-                // odd channels (rows g + 8) hold biased codes: the bias is
-                // removed and 1/16 goes into their scale
-                float vbs[NT];
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    if constexpr (VB) {
-#pragma unroll
-                        for (int o = 4; o < 32; o <<= 1) psum[n] += __shfl_xor_sync(0xffffffffu, psum[n], o);
-                    }
-                    vbs[n] = VB ? kBiasA * psum[n] : 0.0f;
-                }
-                const float pinv_v = VB ? pinv * 0.0625f : pinv;
+                // unit epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f, with
+                // 2^24 of the subnormal INT4 codes and 1/16 of their high
+                // nibbles (odd channels, rows g + 8) in the scales
+                const float pinv_e = VB ? pinv * kTwo24 : pinv;
+                const float pinv_v = VB ? pinv * (kTwo24 / 16.0f) : pinv;
 #pragma unroll
                 for (int tc = 0; tc < 8; ++tc) {
                     const float2 sg = __half22float2(sigv[tc]);
-                    const float s0 = sg.x * pinv, s1_ = sg.y * pinv_v;
+                    const float s0 = sg.x * pinv_e, s1_ = sg.y * pinv_v;
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
                         acc[n][2 * tc] += (dv[n][tc][0] + dv[n][tc][1]) * s0;
-                        if constexpr (VB)
-                            acc[n][2 * tc + 1] += ((dv[n][tc][2] + dv[n][tc][3]) + vbs[n]) * s1_;
-                        else
-                            acc[n][2 * tc + 1] += (dv[n][tc][2] + dv[n][tc][3]) * s1_;
+                        acc[n][2 * tc + 1] += (dv[n][tc][2] + dv[n][tc][3]) * s1_;
                     }
                 }
                 if constexpr (is_nsn(MODE)) {

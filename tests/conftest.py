@@ -28,11 +28,17 @@ def pytest_collection_modifyitems(config, items):
 
 
 def pytest_terminal_summary(terminalreporter, exitstatus, config):
-    """Report the rounding half-point cases met by the GPU parity tests."""
+    """Report the rounding half-point cases met by the GPU parity tests and
+    the largest decode-attention difference from the oracle."""
     try:
-        from tests.gpu_helpers import HALF_POINT_LOG
+        from tests.gpu_helpers import ATTN_ERR_LOG, HALF_POINT_LOG
     except Exception:
         return
+    if ATTN_ERR_LOG:
+        name, worst = max(ATTN_ERR_LOG, key=lambda x: x[1])
+        terminalreporter.write_line(
+            f"GPU decode: {len(ATTN_ERR_LOG)} attention comparisons with the oracle; largest max-abs "
+            f"difference {worst:.3g} ({name}); tolerance 2e-3")
     if not HALF_POINT_LOG:
         return
     n = sum(h for h, _ in HALF_POINT_LOG)

@@ -82,6 +82,19 @@ HALF_POINT_TOL = 1e-6
 # Half-point cases met by the GPU parity tests of this session, reported in
 # the pytest terminal summary (tests/conftest.py).
 HALF_POINT_LOG = []
+# (test, max |GPU - oracle|) of every decode-attention comparison, for the
+# run summary: the margin left under the tolerance
+ATTN_ERR_LOG = []
+
+
+def check_attention(name, got, ref, atol):
+    """Max-abs difference of GPU attention outputs from the oracle's,
+    recorded for the run summary and checked against atol."""
+    import numpy as np
+    err = float(np.max(np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64)))) if np.size(got) else 0.0
+    ATTN_ERR_LOG.append((name, err))
+    assert err <= atol, (name, err)
+    return err
 
 
 def compare_cache(gcache, ck, cv, d, bits, nq, bh_slice=slice(None), t0=0):

@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 from tests.edges import T, edge_kv
-from tests.gpu_helpers import (assert_cache_parity, compare_cache, gpu_decode, gpu_prefill, host16,
+from tests.gpu_helpers import (assert_cache_parity, check_attention, compare_cache, gpu_decode, gpu_prefill, host16,
                                oracle_prefill, to_dev)
 from tests.modes import f16bits
 
@@ -64,4 +64,4 @@ def test_degenerate_inputs_match_oracle(d, bits, mode):
     ref = oracle.cache_attention(ocfg, f16bits(q), ck, cv, f16bits(K[:, :, nq:S]), f16bits(V[:, :, nq:S]), S,
                                  threads=2)
     assert np.all(np.isfinite(out))
-    assert float(np.max(np.abs(out - ref))) <= ATOL
+    check_attention(f"edges {mode} d{d} int{bits}", out, ref, ATOL)

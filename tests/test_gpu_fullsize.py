@@ -15,7 +15,7 @@ import pytest
 
 import oracle
 from kv_cache_bit_b200 import synth
-from tests.gpu_helpers import assert_cache_parity, compare_cache, gpu_decode, gpu_prefill, host16, to_dev
+from tests.gpu_helpers import assert_cache_parity, check_attention, compare_cache, gpu_decode, gpu_prefill, host16, to_dev
 from tests.layout import pairv_applies, pairv_to_rows
 from tests.modes import f16bits, oracle_cfg
 
@@ -135,7 +135,6 @@ def test_full_size_sampled_parity(name, mode, bits, n_app):
         ref = oracle.cache_attention(ocfg, f16bits(q[b:b + 1, h * G:(h + 1) * G]), ck, cv,
                                      f16bits(kk[:, :, nq:length]), f16bits(vv[:, :, nq:length]), length,
                                      threads=1)
-        err = float(np.max(np.abs(out[b, h * G:(h + 1) * G] - ref[0])))
-        assert err <= ATOL, (name, mode, bits, (b, h), err)
+        check_attention(f"full size {name} {mode} int{bits} ({b}, {h})", out[b, h * G:(h + 1) * G], ref[0], ATOL)
     del cache
     torch.cuda.empty_cache()

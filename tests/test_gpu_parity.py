@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 from kv_cache_bit_b200 import synth
-from tests.gpu_helpers import (assert_cache_parity, compare_cache, gpu_decode, gpu_prefill, host16,
+from tests.gpu_helpers import (assert_cache_parity, check_attention, compare_cache, gpu_decode, gpu_prefill, host16,
                                oracle_prefill, to_dev)
 from tests.modes import f16bits
 
@@ -132,8 +132,7 @@ def test_decode_matches_oracle(mode, d, bits, B, Hkv, Hq, S, n_app):
         assert np.array_equal(host16(cache.resid[1])[:, :, :r], f16bits(V[:, :, nq:length]))
     out = gpu_decode(cfg, cache, q)
     ref = _oracle_attention(ocfg, ck, cv, K, V, q, length)
-    err = float(np.max(np.abs(out - ref)))
-    assert err <= ATOL, err
+    check_attention(f"decode {mode} d{d} int{bits} B{B} S{S}+{n_app}", out, ref, ATOL)
 
 
 def test_decode_custom_scale_and_empty_cache():
@@ -147,7 +146,7 @@ def test_decode_custom_scale_and_empty_cache():
     ocfg, ck, cv = oracle_prefill(mode, d, bits, K, V)
     out = gpu_decode(cfg, cache, q, scale=0.02)
     ref = _oracle_attention(ocfg, ck, cv, K, V, q, 256, scale=0.02)
-    assert np.max(np.abs(out - ref)) <= ATOL
+    check_attention("decode custom scale", out, ref, ATOL)
 
 
 def test_residual_only_cache():
@@ -162,7 +161,7 @@ def test_residual_only_cache():
                              to_dev(f16bits(V[:, :, t]).view(np.int16)))
     out = gpu_decode(cfg, cache, q)
     ref = oracle.attention(f16bits(q), K.astype(np.float32), V.astype(np.float32))
-    assert np.max(np.abs(out - ref)) <= ATOL
+    check_attention("decode residual only", out, ref, ATOL)
 
 
 def test_streaming_flush_equals_bulk_quantize():

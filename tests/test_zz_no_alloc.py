@@ -18,7 +18,7 @@ import pytest
 
 import oracle
 from kv_cache_bit_b200 import synth
-from tests.gpu_helpers import gpu_decode, gpu_prefill, oracle_prefill, to_dev
+from tests.gpu_helpers import check_attention, gpu_decode, gpu_prefill, oracle_prefill, to_dev
 from tests.modes import f16bits
 
 ATOL = 2e-3
@@ -59,7 +59,7 @@ def test_noalloc_decode_matches_workspace_decode_and_oracle_twice(d, mode):
         rk = extra[0][:, :, :step] if step else np.zeros((w.B, w.Hkv, 0, w.d), np.uint16)
         rv = extra[1][:, :, :step] if step else np.zeros((w.B, w.Hkv, 0, w.d), np.uint16)
         oref = oracle.cache_attention(ocfg, f16bits(q), ck, cv, rk, rv, length, threads=4)
-        assert np.max(np.abs(got - oref)) <= ATOL
+        check_attention(f"no-alloc decode {mode} d{d} call {step}", got, oref, ATOL)
         # a token more between the calls changes the cache the second call sees
         kvq.kvq_append_token(cfg, cache, to_dev(f16bits(K[:, :, 0]).view(np.int16)),
                              to_dev(f16bits(V[:, :, 0]).view(np.int16)))
