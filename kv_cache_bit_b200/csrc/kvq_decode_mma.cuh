@@ -157,27 +157,32 @@ __device__ __forceinline__ uint32_t h2c(float v) { return pack_h2(v, v); }
 template <int BITS>
 struct KUnpack;
 
-// INT4: the offset-binary code e = q + 8 of a nibble is used in place, as an
-// fp16 subnormal: a low nibble masked out of its 16-bit half reads
-// e * 2^-24, a high nibble (bits 4..7 of its byte) 16 e * 2^-24, one LOP3 per
-// pair and no fp16 arithmetic (kBiased).  The kernel scales the other
-// operand of the high-nibble channels by 1/16, folds 2^24 into the scales it
-// applies to the fp32 results, and removes the bias 8 times the sum of the
-// other operand: for the scores with one MMA chain per block against a
-// constant A of -8 * 2^-24 (low) and -128 * 2^-24 (high nibbles), for the
-// values from the unit's sum of P'.  Subnormal fp16 inputs are exact values;
-// the tensor core's sum of such products measured within 2^-19 of the sum
-// of their magnitudes (against 2^-23 for normal inputs), which the bias
-// (|e| <= 15 against |q| <= 7) costs about one bit of.
-constexpr uint32_t kBiasLoH2 = 0x80088008u;  // fp16x2 -8 * 2^-24
-constexpr uint32_t kBiasHiH2 = 0x80808080u;  // fp16x2 -128 * 2^-24
-constexpr float kTwo24 = 16777216.0f;        // 2^24
-constexpr float kBiasV = -8.0f / 16777216.0f;  // -8 * 2^-24
+// INT4 (kSubnormal): the offset-binary code e = q + kOff of a nibble is
+// used in place, as an fp16 subnormal: a nibble at bits 4j .. of a byte,
+// masked out of its 16-bit half, reads e * f * 2^-24 with the field scale
+// f = 16^j (cscale), one mask per pair of codes and no fp16 arithmetic.  The kernel scales the other operand
+// of a channel by 1/f, folds 2^24 into the scales it applies to the fp32
+// results, and removes the bias kOff times the sum of the other operand: for
+// the scores with one MMA chain per block against a constant A of
+// -kOff f 2^-24 per channel, for the values from the unit's sum of P' as
+// the value chains' starting C.  Subnormal fp16 inputs are exact values; the
+// tensor core's sum of such products measured within 2^-19 of the sum of
+// their magnitudes (against 2^-23 for normal inputs), which the bias
+// (|e| <= 2 qmax + 1 against |q| <= qmax) costs about one bit of.
+constexpr float kTwo24 = 16777216.0f;  // 2^24
+
+// fp16x2 bits of -kOff * f * 2^-24 (both halves); kOff * f < 1024 keeps it subnormal
+__host__ __device__ constexpr uint32_t sub_bias_h2(int off_times_f) {
+    return (0x8000u | (uint32_t)off_times_f) * 0x00010001u;
+}
 
 template <>
 struct KUnpack<4> {
     static constexpr int kPairGroup = 4;  // pairs 4i + j: channels 8i + j and 8i + 4 + j
-    static constexpr bool kBiased = true;
+    static constexpr bool kSubnormal = true;
+    static constexpr int kOff = 8;
+    // field scale of channel c (low nibble 1, high nibble 16)
+    __host__ __device__ static constexpr int cscale(int c) { return (c & 1) ? 16 : 1; }
     __device__ static int ca(int p) { return 8 * (p >> 2) + (p & 3); }
     __device__ static int cb(int p) { return ca(p) + 4; }
     // row points at the row's first byte; even pairs p hold e * 2^-24, odd
@@ -197,6 +202,9 @@ struct KUnpack<4> {
 };
 
 // 2-bit fields j = 0..3 of a byte pair: value 1024 + e * 4^j, q = e - off.
+// (INT2 codes are converted to exact q: as subnormals with field scales up
+// to 64 the score and value sums measured about four times the error of
+// this form.)
 template <int OFF>
 __device__ __forceinline__ uint32_t dec2(uint32_t x, int j) {
     const float m = float(1 << (2 * j));
@@ -205,7 +213,9 @@ __device__ __forceinline__ uint32_t dec2(uint32_t x, int j) {
 
 template <>
 struct KUnpack<2> {
-    static constexpr bool kBiased = false;
+    static constexpr bool kSubnormal = false;
+    static constexpr int kOff = 0;
+    __host__ __device__ static constexpr int cscale(int) { return 1; }
     static constexpr int kPairGroup = 8;  // pairs 8i + j: channels 16i + j and 16i + 8 + j
     __device__ static int ca(int p) { return 16 * (p >> 3) + (p & 7); }
     __device__ static int cb(int p) { return ca(p) + 8; }
@@ -248,7 +258,9 @@ __device__ __forceinline__ uint32_t hi_to(uint32_t h, int j) {
 
 template <>
 struct KUnpack<3> {
-    static constexpr bool kBiased = false;
+    static constexpr bool kSubnormal = false;
+    static constexpr int kOff = 0;
+    __host__ __device__ static constexpr int cscale(int) { return 1; }
     static constexpr int kPairGroup = 8;  // pairs 8i + j: channels 16i + j and 16i + 8 + j
     __device__ static int ca(int p) { return 16 * (p >> 3) + (p & 7); }
     __device__ static int cb(int p) { return ca(p) + 8; }
@@ -277,7 +289,10 @@ struct VUnpack;
 
 template <>
 struct VUnpack<4> {
-    static constexpr bool kBiased = true;  // e * 2^-24; odd channels (high nibbles) 16 e * 2^-24
+    static constexpr bool kSubnormal = true;  // e * 2^-24; odd channels (high nibbles) 16 e * 2^-24
+    static constexpr int kOff = 8;
+    // field scale of register i of run() (the MMA's row g for even i, g + 8 for odd)
+    __host__ __device__ static constexpr int vscale(int i) { return (i & 1) ? 16 : 1; }
     // units 4g .. 4g + 3: the 16-byte chunk g, at g ^ (2 (k & 1))
     __device__ static void run(const uint8_t* pb, int k, int g, uint32_t (&pr)[16]) {
         const uint4 v = *reinterpret_cast<const uint4*>(pb + 16 * (g ^ pairv_chunk_xor<4>(k)));
@@ -296,7 +311,9 @@ struct VUnpack<4> {
 
 template <>
 struct VUnpack<2> {
-    static constexpr bool kBiased = false;
+    static constexpr bool kSubnormal = false;
+    static constexpr int kOff = 0;
+    __host__ __device__ static constexpr int vscale(int) { return 1; }
     // units 2g, 2g + 1: words 2g, 2g + 1 of the pair block
     __device__ static void run(const uint8_t* pb, int, int g, uint32_t (&pr)[16]) {
         const uint2 v = *reinterpret_cast<const uint2*>(pb + 8 * g);
@@ -314,7 +331,9 @@ struct VUnpack<2> {
 
 template <>
 struct VUnpack<3> {
-    static constexpr bool kBiased = false;
+    static constexpr bool kSubnormal = false;
+    static constexpr int kOff = 0;
+    __host__ __device__ static constexpr int vscale(int) { return 1; }
     // 2-bit plane: units 2g, 2g + 1 (words 2g, 2g + 1); bit plane: unit 16 + g
     __device__ static void run(const uint8_t* pb, int, int g, uint32_t (&pr)[16]) {
         const uint2 v = *reinterpret_cast<const uint2*>(pb + 8 * g);
@@ -477,7 +496,9 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
     constexpr float kLog2e = 1.4426950408889634f;
     constexpr int QMAX = (1 << (BITS - 1)) - 1;
     constexpr float kTau = 8.0f;  // reference-max slack (log2 units): p <= 2^kTau
-    constexpr bool KB = KUnpack<BITS>::kBiased, VB = VUnpack<BITS>::kBiased;
+    using KU = KUnpack<BITS>;
+    using VU = VUnpack<BITS>;
+    constexpr bool KB = KU::kSubnormal, VB = VU::kSubnormal;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     grid_dep_launch();
@@ -606,8 +627,8 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
             const float qsc = bound > 0.0f ? pow2i(13 - ceil_log2(bound)) : 1.0f;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                // odd channels meet biased INT4 codes 16 (q + 72): 1/16
-                const float bs = (KB && (k & 1)) ? 0.0625f : 1.0f;
+                // channels of field scale f meet codes e f 2^-24: 1/f
+                const float bs = KB ? 1.0f / (float)KU::cscale(k) : 1.0f;
                 wqs[qs_index(j, 4 * lane + k)] = v[k] * qsc * bs;
             }
             if (lane == 0) wqsc[j] = qsc;
@@ -684,18 +705,23 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                         }
                     }
                     if constexpr (KB) {
-                        // bias of the score chains: A = -8 * 2^-24 on the even
-                        // pairs of a k-step (a0, a1), -128 * 2^-24 on the odd
-                        // ones (a2, a3), whose B carries 1/16
+                        // bias of the score chains: A = -kOff f 2^-24 for the
+                        // field scale f of each pair's channels (a0, a1: pair
+                        // 2s of k-step s; a2, a3: pair 2s + 1), whose B carries
+                        // 1/f; pairs p and p + 4 have the scale of channel p & 3
+                        constexpr uint32_t z0 = sub_bias_h2(KU::kOff * KU::cscale(0));
+                        constexpr uint32_t z1 = sub_bias_h2(KU::kOff * KU::cscale(1));
+                        constexpr uint32_t z2 = sub_bias_h2(KU::kOff * KU::cscale(2));
+                        constexpr uint32_t z3 = sub_bias_h2(KU::kOff * KU::cscale(3));
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
                             float c0[4], c1[4];
-                            mma16816_z(c0, kBiasLoH2, kBiasLoH2, kBiasHiH2, kBiasHiH2, bq[n][0], bq[n][1]);
-                            mma16816_z(c1, kBiasLoH2, kBiasLoH2, kBiasHiH2, kBiasHiH2, bq[n][2], bq[n][3]);
+                            mma16816_z(c0, z0, z0, z1, z1, bq[n][0], bq[n][1]);
+                            mma16816_z(c1, z2, z2, z3, z3, bq[n][2], bq[n][3]);
 #pragma unroll
                             for (int s = 2; s < 8; s += 2) {
-                                mma16816(c0, kBiasLoH2, kBiasLoH2, kBiasHiH2, kBiasHiH2, bq[n][2 * s], bq[n][2 * s + 1]);
-                                mma16816(c1, kBiasLoH2, kBiasLoH2, kBiasHiH2, kBiasHiH2, bq[n][2 * s + 2], bq[n][2 * s + 3]);
+                                mma16816(c0, z0, z0, z1, z1, bq[n][2 * s], bq[n][2 * s + 1]);
+                                mma16816(c1, z2, z2, z3, z3, bq[n][2 * s + 2], bq[n][2 * s + 3]);
                             }
                             kb[n][0] = c0[0] + c1[0];
                             kb[n][1] = c0[1] + c1[1];
@@ -868,18 +894,17 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                         }
                     }
                 }
-                // biased INT4 codes: the bias (8 e-units per code, scaled like
-                // the codes) enters the value chains as their starting C, from
-                // the unit's sum of P' (rows g: low nibbles, g + 8: high)
-                float vlo[NT], vhi[NT];
+                // subnormal codes: the bias (kOff per code, times the field
+                // scale of the row) enters the value chains as their starting
+                // C, from the unit's sum of P'
+                float vlo[NT];
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     if constexpr (VB) {
 #pragma unroll
                         for (int o = 4; o < 32; o <<= 1) psum[n] += __shfl_xor_sync(0xffffffffu, psum[n], o);
                     }
-                    vlo[n] = VB ? kBiasV * psum[n] : 0.0f;
-                    vhi[n] = VB ? (16.0f * kBiasV) * psum[n] : 0.0f;
+                    vlo[n] = VB ? (-(float)VU::kOff / kTwo24) * psum[n] : 0.0f;  // times the field scale
                 }
 #pragma unroll
                 for (int m4 = 0; m4 < 4; ++m4) {
@@ -896,7 +921,8 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
                         for (int n = 0; n < NT; ++n) {
                             if (m4 == 0 && VB)
                                 mma16816_c4(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1],
-                                            bp[n][0], bp[n][1], vlo[n], 0.0f, vhi[n], 0.0f);
+                                            bp[n][0], bp[n][1], (float)VU::vscale(2 * tc) * vlo[n], 0.0f,
+                                            (float)VU::vscale(2 * tc + 1) * vlo[n], 0.0f);
                             else if (m4 == 0)
                                 mma16816_z(dv[n][tc], va[2 * tc], va[2 * tc + 1], vb[2 * tc], vb[2 * tc + 1],
                                            bp[n][0], bp[n][1]);
@@ -909,14 +935,14 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
 #pragma unroll
                 for (int n = 0; n < NT; ++n) l_run[n] += lsum[n];
                 // unit epilogue: acc[c] += (hi + lo) * sigma^V_c * 2^-f, with
-                // 2^24 of the subnormal INT4 codes and 1/16 of their high
-                // nibbles (odd channels, rows g + 8) in the scales
+                // 2^24 of the subnormal codes and 1 / field scale of the row
+                // in the scales
                 const float pinv_e = VB ? pinv * kTwo24 : pinv;
-                const float pinv_v = VB ? pinv * (kTwo24 / 16.0f) : pinv;
 #pragma unroll
                 for (int tc = 0; tc < 8; ++tc) {
                     const float2 sg = __half22float2(sigv[tc]);
-                    const float s0 = sg.x * pinv_e, s1_ = sg.y * pinv_v;
+                    const float s0 = sg.x * (pinv_e / (float)VU::vscale(2 * tc));
+                    const float s1_ = sg.y * (pinv_e / (float)VU::vscale(2 * tc + 1));
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
                         acc[n][2 * tc] += (dv[n][tc][0] + dv[n][tc][1]) * s0;

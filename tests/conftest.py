@@ -35,10 +35,10 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     except Exception:
         return
     if ATTN_ERR_LOG:
-        name, worst = max(ATTN_ERR_LOG, key=lambda x: x[1])
+        ranked = sorted(ATTN_ERR_LOG, key=lambda x: -x[1])
         terminalreporter.write_line(
             f"GPU decode: {len(ATTN_ERR_LOG)} attention comparisons with the oracle; largest max-abs "
-            f"difference {worst:.3g} ({name}); tolerance 2e-3")
+            f"differences (tolerance 2e-3): " + "; ".join(f"{e:.3g} {n}" for n, e in ranked[:6]))
     if not HALF_POINT_LOG:
         return
     n = sum(h for h, _ in HALF_POINT_LOG)
