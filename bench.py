@@ -410,28 +410,56 @@ def run_ours(args, rank: int, world: int):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    # the timed steps: events only at the two ends (an event between two
+    # calls holds back the launch of the second)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for _ in range(args.steps):
-        step(True)
+        step(False)
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop()
     ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, dev)
 
+    # the decode kernels' duration: consecutive calls at the stream's mean
+    # cache shape (the last length with 64 residual tokens: 65 blocks + 64
+    # tokens for the throughput workload), events around the loop
+    final = cache.len
+    t_len = next((L for L in range(final, w.S, -1) if L % 128 == 64), final)
+    cache.c.len = t_len
+    for _ in range(3):
+        kvq.kvq_decode_attention(cfg, cache, qsd[n_stream - 1 if n_stream else 0], w.Hq, 0.0, out, ws, ws_bytes,
+                                 stream)
+    n_dec = 32
+    k0 = torch.cuda.Event(enable_timing=True)
+    k1 = torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    for _ in range(n_dec):
+        kvq.kvq_decode_attention(cfg, cache, qsd[n_stream - 1 if n_stream else 0], w.Hq, 0.0, out, ws, ws_bytes,
+                                 stream)
+    k1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    k_s = max_over_ranks(k0.elapsed_time(k1) / n_dec, world, dev) / 1e3
+    k_bytes = accounting.decode_bytes(w.d, BITS, flags, w.B, w.Hkv, w.Hq, t_len)
+    cache.c.len = final
+
+    # one more step with events around every call: where the step's time goes
+    # (each event delays the launch behind it, so these spans run long)
+    step(True)
+    torch.cuda.synchronize()
     q_ms = [a.elapsed_time(b) for k, a, b in ev if k == "quantize"]
     d_ms = [a.elapsed_time(b) for k, a, b in ev if k == "decode"]
     a_ms = [a.elapsed_time(b) for k, a, b in ev if k == "append"]
     f_ms = [a.elapsed_time(b) for k, a, b in ev if k == "flush"]
     dec_avg_bytes = sum(dec_bytes) / len(dec_bytes)
-    dec_avg_s = (sum(d_ms) / len(d_ms)) / 1e3
+    dec_span_s = (sum(d_ms) / len(d_ms)) / 1e3
     q_avg_s = (sum(q_ms) / len(q_ms)) / 1e3
     q_bytes = accounting.quantize_bytes(w.d, BITS, flags, w.B, w.Hkv, w.S)
     peak, peak_kind = measured_peak_gbs()
-    dec_gbs = dec_avg_bytes / dec_avg_s / 1e9
+    dec_gbs = k_bytes / k_s / 1e9
     q_gbs = q_bytes / q_avg_s / 1e9
     value = world * step_bytes / (ms / 1e3) / 1e9
 
@@ -451,9 +479,13 @@ def run_ours(args, rank: int, world: int):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": bench_config(w, BITS, world),
-        "decode": {"gbs": dec_gbs, "frac_of_hbm": dec_gbs / peak, "us_per_call": dec_avg_s * 1e6,
-                   "tokens_per_s": world * w.B / dec_avg_s, "bytes_per_call": dec_avg_bytes,
-                   "cache_tokens_per_s": world * w.B * w.Hkv * (w.S + (n_stream + 1) / 2) / dec_avg_s},
+        "decode": {"gbs": dec_gbs, "frac_of_hbm": dec_gbs / peak, "us_per_call": k_s * 1e6,
+                   "bytes_per_call": k_bytes, "length": t_len,
+                   "timing": f"{n_dec} consecutive calls at {t_len} tokens, CUDA events around the loop",
+                   "tokens_per_s": world * w.B / k_s,
+                   "cache_tokens_per_s": world * w.B * w.Hkv * t_len / k_s,
+                   "in_step_us_per_call": dec_span_s * 1e6, "in_step_bytes_per_call": dec_avg_bytes,
+                   "in_step_gbs": dec_avg_bytes / dec_span_s / 1e9},
         "append": {"us_per_call": 1e3 * sum(a_ms) / max(1, len(a_ms)),
                    "flush_us_per_call": 1e3 * sum(f_ms) / max(1, len(f_ms)) if f_ms else None,
                    "flushes_per_step": len(f_ms) // max(1, args.steps)},
@@ -462,7 +494,7 @@ def run_ours(args, rank: int, world: int):
         "tokens_per_s": world * w.B * n_stream / (ms / 1e3),
         "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peak, "unit": "GB/s", "frac": dec_gbs / peak,
                      "traffic": decode_traffic(),
-                     "kernel": "kvq_decode_attention (decode + combine launches), per call",
+                     "kernel": "kvq_decode_attention (decode + combine launches), per call, consecutive calls",
                      "peak_kind": f"{peak_kind} copy bandwidth (burst)",
                      "traffic_source": "profiles/decode_traffic_throughput.md (ncu dram bytes, one call)"},
         "e2e": e2e,
@@ -486,8 +518,9 @@ def run_ours(args, rank: int, world: int):
 
 def run_variant(w, bits, flags, Kd, Vd, ksd, vsd, qsd, stream, peak):
     """The same workload with other codes (INT2) or side parameters (DQ):
-    quantize of the prefill, the streamed appends, then decode calls at the
-    final length (CUDA events on the launching stream)."""
+    quantize of the prefill, the streamed appends, then consecutive decode
+    calls at the stream's mean cache shape (the last length with 64 residual
+    tokens), CUDA events on the launching stream."""
     import torch
     from kv_cache_bit_b200 import kvq
     dev = Kd.device
@@ -510,6 +543,8 @@ def run_variant(w, bits, flags, Kd, Vd, ksd, vsd, qsd, stream, peak):
     q1.record(stream)
     for i in range(w.stream):
         kvq.kvq_append_token(cfg, cache, ksd[i], vsd[i], stream)
+    t_len = next((L for L in range(cache.len, w.S, -1) if L % 128 == 64), cache.len)
+    cache.c.len = t_len
     qlast = qsd[w.stream - 1] if w.stream else qsd[0]
     for _ in range(3):
         kvq.kvq_decode_attention(cfg, cache, qlast, w.Hq, 0.0, out, ws, ws_bytes, stream)
@@ -523,11 +558,11 @@ def run_variant(w, bits, flags, Kd, Vd, ksd, vsd, qsd, stream, peak):
     q_s = q0.elapsed_time(q1) / reps / 1e3
     d_s = d0.elapsed_time(d1) / n / 1e3
     qb = accounting.quantize_bytes(w.d, bits, flags, w.B, w.Hkv, w.S)
-    db = accounting.decode_bytes(w.d, bits, flags, w.B, w.Hkv, w.Hq, w.S + w.stream)
+    db = accounting.decode_bytes(w.d, bits, flags, w.B, w.Hkv, w.Hq, t_len)
     return {"quantize": {"gbs": qb / q_s / 1e9, "frac_of_hbm": qb / q_s / 1e9 / peak, "us_per_call": q_s * 1e6,
                          "bytes_per_call": qb},
             "decode": {"gbs": db / d_s / 1e9, "frac_of_hbm": db / d_s / 1e9 / peak, "us_per_call": d_s * 1e6,
-                       "bytes_per_call": db, "length": w.S + w.stream}}
+                       "bytes_per_call": db, "length": t_len}}
 
 
 def run_e2e(args, w, cfg, cache, out, ws, ws_bytes, K, V, ks, vs, qs, stream, dev, step_bytes, world, ref_last):

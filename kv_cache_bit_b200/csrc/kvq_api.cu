@@ -239,9 +239,15 @@ struct AppendLaunch {
     cudaStream_t st;
     template <int D, int BITS, int MODE, bool HAD>
     kvq_status run() {
+        if (a.slot < kT - 1) {
+            // a plain copy into the residual slot
+            const int n = 2 * bh * (D / 8);
+            append_copy_kernel<D><<<(n + 255) / 256, 256, 0, st>>>(a, bh);
+            return launch_status();
+        }
         constexpr int smem = quant_smem_bytes<D, MODE>();
         if (!ensure_smem<append_kernel<D, BITS, MODE, HAD>>(smem)) return KVQ_ERR_CUDA;
-        append_kernel<D, BITS, MODE, HAD><<<dim3(bh, 2), kT, a.slot == kT - 1 ? smem : 0, st>>>(a);
+        append_kernel<D, BITS, MODE, HAD><<<dim3(bh, 2), kT, smem, st>>>(a);
         return launch_status();
     }
 };
@@ -295,7 +301,20 @@ kvq_status launch_decode_mma(DecodeArgs a, int bh, cudaStream_t st) {
     a.work = (long long)bh * a.nbq;
     if (a.work >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
     if (a.work > 0) {
-        kern<<<grid, kNW * 32, smem, st>>>(a);
+        // a programmatic dependent of the kernel ahead of it in the stream:
+        // its launch overlaps that kernel's tail (the kernel waits for it
+        // before touching memory)
+        cudaLaunchConfig_t dc = {};
+        dc.gridDim = dim3(grid);
+        dc.blockDim = dim3(kNW * 32);
+        dc.dynamicSmemBytes = smem;
+        dc.stream = st;
+        cudaLaunchAttribute da[1];
+        da[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        da[0].val.programmaticStreamSerializationAllowed = 1;
+        dc.attrs = da;
+        dc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&dc, kern, a) != cudaSuccess) return KVQ_ERR_CUDA;
         kvq_status s = launch_status();
         if (s != KVQ_OK) return s;
     }

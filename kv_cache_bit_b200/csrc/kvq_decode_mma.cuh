@@ -137,13 +137,6 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Programmatic dependent launch: the decode kernel lets the combine kernel
-// be scheduled early; the combine kernel does its residual work and then
-// waits here until the decode kernel has finished and its partials are
-// visible.  Without the launch attribute the wait returns at once.
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 constexpr uint32_t kMagic = 0x64006400u;  // fp16x2 1024.0, 1024.0
 
@@ -501,7 +494,6 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
     constexpr bool KB = KU::kSubnormal, VB = VU::kSubnormal;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    grid_dep_launch();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int G = a.G;
@@ -554,6 +546,12 @@ __global__ void __launch_bounds__(kNW * 32, ((BITS == 3 || is_nsn(MODE)) && GP =
             while (iss_blk >= nbq) { iss_blk -= nbq; ++iss_pair; }
         }
     };
+    // the kernel is a programmatic dependent of the one ahead of it (an
+    // append, or the previous call's combine): nothing of the cache, the
+    // queries or the workspace is touched before that one has finished; the
+    // combine kernel behind this one may be scheduled from here on
+    grid_dep_wait();
+    grid_dep_launch();
     int issued = min(kRing, nunits);
     for (int u = 0; u < issued; ++u) {
         if (lane == 0) issue(u);

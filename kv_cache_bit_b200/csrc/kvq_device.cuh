@@ -144,6 +144,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 __device__ __forceinline__ void report_error(uint32_t bit) { atomicOr(&g_error_word, bit); }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start before the kernel ahead of it in the stream has
+// finished; grid_dep_wait() returns once that kernel has completed and its
+// memory is visible (at once when the launch attribute is absent), and
+// grid_dep_launch() lets the kernel behind this one be scheduled early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- packing
 
 template <int D, int BITS>

@@ -250,21 +250,30 @@ struct AppendArgs {
     int blk;                 // destination block when the slot is the last one
 };
 
-// One CTA per (batch*head, tensor).  The new token goes to its residual slot;
-// when that slot is the block's last, the CTA instead quantizes the 127 held
-// tokens plus the new one into block `blk` (same arithmetic as
-// quantize_kernel).
+// The new token of every (batch*head, tensor) into its residual slot, when
+// that slot is not the block's last: one 16-byte chunk per thread.  The
+// decode kernel behind it may be scheduled at once.
+template <int D>
+__global__ void __launch_bounds__(256) append_copy_kernel(AppendArgs a, int bh) {
+    grid_dep_launch();
+    constexpr int NC = D / 8;  // 16-byte chunks per row
+    const int i = blockIdx.x * 256 + threadIdx.x;
+    if (i >= 2 * bh * NC) return;
+    const int tensor = i / (bh * NC), r = i - tensor * bh * NC, row = r / NC, c = r - row * NC;
+    const uint4* src = reinterpret_cast<const uint4*>((tensor ? a.x_new[1] : a.x_new[0]) + (size_t)row * D) + c;
+    uint4* dst = reinterpret_cast<uint4*>((tensor ? a.resid[1] : a.resid[0]) + ((size_t)row * kT + a.slot) * D) + c;
+    *dst = *src;
+}
+
+// One CTA per (batch*head, tensor), launched when the new token's slot is
+// the block's last: the CTA quantizes the 127 held tokens plus the new one
+// into block `blk` (same arithmetic as quantize_kernel).
 template <int D, int BITS, int MODE, bool HAD>
 __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
     const int t = threadIdx.x;
     const int bh = blockIdx.x, tensor = blockIdx.y;
     const __half* xn = (tensor ? a.x_new[1] : a.x_new[0]) + (size_t)bh * D;
     __half* res = (tensor ? a.resid[1] : a.resid[0]) + (size_t)bh * kT * D;
-    if (a.slot < kT - 1) {
-        if (t < D / 8)
-            reinterpret_cast<uint4*>(res + (size_t)a.slot * D)[t] = reinterpret_cast<const uint4*>(xn)[t];
-        return;
-    }
     extern __shared__ uint8_t smem_raw[];
     uint64_t* bar;
     uint8_t* regions;
