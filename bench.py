@@ -269,6 +269,26 @@ def rank_workload(rank: int, batch=None, stream=None):
     return w
 
 
+def batch_shard(B: int, rank: int, world: int):
+    """Batch rows [lo, hi) of rank `rank` when one workload's batch is split
+    over `world` ranks: contiguous, sizes differ by at most one row.  Every
+    (batch row, kv head) pair is an independent problem, so the shards need
+    no collective on the data path."""
+    q, r = divmod(B, world)
+    lo = rank * q + min(rank, r)
+    return lo, lo + q + (1 if rank < r else 0)
+
+
+def sum_over_ranks(x: float, world: int, device) -> float:
+    """The job's total of a per-rank figure (bytes moved by all ranks)."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
 def max_over_ranks(ms: float, world: int, device) -> float:
     """The slowest rank's time: the job's step time under weak scaling."""
     if world == 1:
@@ -289,11 +309,12 @@ def l2_note(w, bits):
             f"126 MB L2 stays there between calls (no flush)")
 
 
-def bench_config(w, bits, world):
+def bench_config(w, bits, world, split=False):
     return {"workload": WORKLOAD, "mode": MODE, "bits": bits, "batch": w.B, "q_heads": w.Hq,
             "kv_heads": w.Hkv, "head_dim": w.d, "seq_len": w.S, "streamed": w.stream,
             "l2": l2_note(w, bits),
-            "parallelism": f"weak x{world} (independent batches, no collective)"}
+            "parallelism": (f"batch split over {world} ranks (strong; batch above is per rank, no collective)"
+                            if split else f"weak x{world} (independent batches, no collective)")}
 
 
 def host_cores() -> int:
@@ -340,7 +361,10 @@ def run_ours(args, rank: int, world: int):
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    w = rank_workload(rank, args.batch, args.stream)
+    split = args.split_batch and world > 1
+    # weak scaling: every rank its own draw of the workload; --split-batch:
+    # one workload (rank 0's draw) whose batch is split over the ranks
+    w = rank_workload(0 if split else rank, args.batch, args.stream)
     BITS = args.bits
     flags = flags_of(MODE)
     G = w.Hq // w.Hkv
@@ -351,6 +375,11 @@ def run_ours(args, rank: int, world: int):
     K, V = synth.kv(w)
     ks, vs = synth.stream_tokens(w)
     qs = synth.queries(w, steps=n_stream)
+    if split:
+        lo, hi = batch_shard(w.B, rank, world)
+        K, V = K[lo:hi], V[lo:hi]
+        ks, vs, qs = ks[:, lo:hi], vs[:, lo:hi], qs[:, lo:hi]
+        w = w.scaled(B=hi - lo)
     tod = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
     Kd, Vd, ksd, vsd, qsd = tod(K), tod(V), tod(ks), tod(vs), tod(qs)
     signs = kvq.kvq_make_signs(synth.SIGN_SEED, w.d) if synth.MODES[MODE][1] else None
@@ -461,7 +490,7 @@ def run_ours(args, rank: int, world: int):
     peak, peak_kind = measured_peak_gbs()
     dec_gbs = k_bytes / k_s / 1e9
     q_gbs = q_bytes / q_avg_s / 1e9
-    value = world * step_bytes / (ms / 1e3) / 1e9
+    value = sum_over_ranks(step_bytes, world, dev) / (ms / 1e3) / 1e9
 
     extra = not (args.no_int2 or world > 1 or BITS != 4 or WORKLOAD != "throughput")
     int2 = run_variant(w, 2, flags, Kd, Vd, ksd, vsd, qsd, stream, peak) if extra else None
@@ -476,9 +505,10 @@ def run_ours(args, rank: int, world: int):
         return 0
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": bench_config(w, BITS, world),
+        "config": bench_config(w, BITS, world, split),
         "decode": {"gbs": dec_gbs, "frac_of_hbm": dec_gbs / peak, "us_per_call": k_s * 1e6,
                    "bytes_per_call": k_bytes, "length": t_len,
                    "timing": f"{n_dec} consecutive calls at {t_len} tokens, CUDA events around the loop",
@@ -681,6 +711,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-int2", action="store_true", help="skip the INT2 measurement of the same workload")
+    ap.add_argument("--split-batch", action="store_true",
+                    help="under torchrun: split one workload's batch over the ranks (strong scaling) instead of "
+                         "one workload per rank (weak scaling)")
     ap.add_argument("--batch", type=int, default=None, help="override the batch size (smaller profiling cases)")
     ap.add_argument("--stream", type=int, default=None, help="override the number of streamed decode steps")
     ap.add_argument("--bits", type=int, default=BITS, choices=[2, 3, 4])

@@ -185,7 +185,7 @@ kvq_status kvq_quantize_block(const kvq_config* cfg, kvq_cache* cache,
  * Append one token per (b, h) to the residual (NSNQuant "Implementation
  * details": full-precision residual flushed into the quantized part when
  * full).  k_new, v_new fp16 [B][H][head_dim].  The token goes to residual
- * slot len % 128; when that slot is 127 the same launch quantizes the 128
+ * slot len % 128; when that slot is 127 the call instead quantizes the 128
  * residual tokens into block floor(len/128) exactly as kvq_quantize_block
  * would, which empties the residual.  On success len += 1.
  * Errors: INVALID_ARG; CAPACITY (len + 1 > capacity); UNSUPPORTED; CUDA.
@@ -195,8 +195,10 @@ kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache,
 
 /* Workspace bytes kvq_decode_attention needs for this cache and q_heads
    (partial softmax states of the sequence splits); 0 on invalid arguments.
-   Each call writes every partial state it reads, so the workspace needs no
-   initialization. */
+   At head dim 128 the size depends on the current device's SM count (the
+   persistent grid is at most 4 CTAs per SM): size it on the device the
+   decode runs on.  Each call writes every partial state it reads, so the
+   workspace needs no initialization. */
 size_t kvq_decode_workspace_bytes(const kvq_config* cfg, const kvq_cache* cache, int32_t q_heads);
 
 /*

@@ -296,7 +296,7 @@ kvq_status launch_decode_mma(DecodeArgs a, int bh, cudaStream_t st) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kNW * 32, smem) != cudaSuccess)
         return KVQ_ERR_CUDA;
     int grid = sms * (occ > 0 ? occ : 1);
-    if (grid > kMaxCTAs) grid = kMaxCTAs;
+    if (grid > kMaxCtasPerSM * sms) grid = kMaxCtasPerSM * sms;
     a.nwarps = (long long)grid * kNW;
     a.work = (long long)bh * a.nbq;
     if (a.work >= (1ll << 31)) return KVQ_ERR_UNSUPPORTED;
@@ -465,9 +465,19 @@ size_t kvq_decode_workspace_bytes(const kvq_config* cfg, const kvq_cache* cache,
     if (G > kGMax) return 0;
     const size_t bh = (size_t)cache->batch * cache->kv_heads;
     // tensor-core path: one partial per (warp, pair) segment, kNW slots per
-    // (CTA, pair) meeting; those are bounded by (largest persistent grid) + (pairs)
-    if (cfg->head_dim == 128)
-        return (size_t)kNW * ((size_t)kMaxCTAs + bh) * (size_t)G * part_stride<128>() * sizeof(float);
+    // (CTA, pair) meeting; those are bounded by (largest persistent grid on
+    // the current device) + (pairs)
+    if (cfg->head_dim == 128) {
+        // without a usable device (host-side checks), the bound of a 256-SM part
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+            cudaGetLastError();
+            sms = 256;
+        }
+        const size_t max_ctas = (size_t)kMaxCtasPerSM * (size_t)sms;
+        return (size_t)kNW * (max_ctas + bh) * (size_t)G * part_stride<128>() * sizeof(float);
+    }
     return bh * (size_t)decode_splits(cache) * (size_t)G * (2 + 2 * (size_t)cfg->head_dim) * sizeof(float);
 }
 

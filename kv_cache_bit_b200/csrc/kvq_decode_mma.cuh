@@ -346,7 +346,7 @@ struct VUnpack<3> {
 // ---------------------------------------------------------------- slot layout
 
 constexpr int kUT = 64;  // tokens per staging unit (half a block)
-constexpr int kMaxCTAs = 4 * 148;  // cap of the persistent grid
+constexpr int kMaxCtasPerSM = 4;  // cap of the persistent grid: this many CTAs per SM
 
 // A unit is one tensor's half block: packed codes and per-token parameters of
 // 64 tokens; the first half also carries the block's channel scales and NSN
