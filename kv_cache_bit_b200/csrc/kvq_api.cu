@@ -11,6 +11,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kvq.h"
 #include "kvq_decode_mma.cuh"
 #include "kvq_decode_simple.cuh"
@@ -20,6 +22,15 @@ namespace kvq {
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range around each entry point (no cost beyond a few loads unless
+// a profiler has attached its NVTX hooks).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 
 struct ModeInfo {
@@ -410,6 +421,7 @@ kvq_status kvq_make_signs(uint64_t seed, int32_t head_dim, int8_t* host_out) {
 
 kvq_status kvq_quantize_block(const kvq_config* cfg, kvq_cache* cache, const uint16_t* k, const uint16_t* v,
                               int64_t t0, int64_t ntok, void* stream) {
+    NvtxRange nvtx_range("kvq_quantize_block");
     ModeInfo mi;
     kvq_status s = check_cfg(cfg, &mi);
     if (s != KVQ_OK) return s;
@@ -437,6 +449,7 @@ kvq_status kvq_quantize_block(const kvq_config* cfg, kvq_cache* cache, const uin
 
 kvq_status kvq_append_token(const kvq_config* cfg, kvq_cache* cache, const uint16_t* k_new, const uint16_t* v_new,
                             void* stream) {
+    NvtxRange nvtx_range("kvq_append_token");
     ModeInfo mi;
     kvq_status s = check_cfg(cfg, &mi);
     if (s != KVQ_OK) return s;
@@ -483,6 +496,7 @@ size_t kvq_decode_workspace_bytes(const kvq_config* cfg, const kvq_cache* cache,
 
 kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache, const uint16_t* q, int32_t q_heads,
                                 float scale, float* out, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("kvq_decode_attention");
     ModeInfo mi;
     kvq_status s = check_cfg(cfg, &mi);
     if (s != KVQ_OK) return s;
@@ -528,6 +542,7 @@ size_t kvq_select_signs_workspace_bytes(int32_t n_cand, int64_t n_blocks) {
 
 kvq_status kvq_select_signs(const kvq_config* cfg, const uint16_t* x, int64_t n_blocks, const int8_t* signs,
                             int32_t n_cand, double* err, int32_t* best, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("kvq_select_signs");
     ModeInfo mi;
     kvq_status s = check_cfg(cfg, &mi);
     if (s != KVQ_OK) return s;
@@ -553,6 +568,7 @@ kvq_status kvq_select_signs(const kvq_config* cfg, const uint16_t* x, int64_t n_
 
 kvq_status kvq_dequantize(const kvq_config* cfg, const kvq_cache* cache, int32_t tensor, int64_t t0, int64_t ntok,
                           float* out, void* stream) {
+    NvtxRange nvtx_range("kvq_dequantize");
     ModeInfo mi;
     kvq_status s = check_cfg(cfg, &mi);
     if (s != KVQ_OK) return s;
@@ -616,6 +632,7 @@ extern "C" {
 
 kvq_status kvq_decode_attention_noalloc(const kvq_config* cfg, const kvq_cache* cache, const uint16_t* q,
                                         int32_t q_heads, float scale, float* out, void* stream) {
+    NvtxRange nvtx_range("kvq_decode_attention_noalloc");
     ModeInfo mi;
     kvq_status s = check_cfg(cfg, &mi);
     if (s != KVQ_OK) return s;

@@ -256,6 +256,25 @@ class KVCache:
     def len(self) -> int:
         return self.c.len
 
+    def snapshot(self) -> dict:
+        """A host copy of the cache (checkpoint): every buffer and the
+        token count.  The cache is plain caller-owned memory, so this is the
+        whole state."""
+        cp = lambda ts: [t.cpu() if t is not None else None for t in ts]
+        return {"len": self.c.len, "codes": cp(self.codes), "tok": cp(self.tok), "chan": cp(self.chan),
+                "off": cp(self.off), "resid": cp(self.resid)}
+
+    def restore(self, snap: dict) -> None:
+        """Load a snapshot taken from a cache of the same configuration and
+        shape (resume)."""
+        for name in ("codes", "tok", "chan", "off", "resid"):
+            for dst, src in zip(getattr(self, name), snap[name]):
+                if (dst is None) != (src is None) or (dst is not None and dst.shape != src.shape):
+                    raise KvqError(KVQ_ERR_INVALID_ARG, "KVCache.restore: snapshot of another cache shape")
+                if dst is not None:
+                    dst.copy_(src)
+        self.c.len = snap["len"]
+
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for group in (self.codes, self.tok, self.chan, self.off, self.resid)
                    for t in group if t is not None)

@@ -170,3 +170,26 @@ def test_dq_flag_sizes(kvq):
         assert kvq.kvq_off_words(kvq.NORM_SEP | kvq.PER_CHANNEL, d) == 0
     assert kvq.kvq_off_words(nsn_dq, 96) == -1
     assert oracle.ntok(oracle.NSN | oracle.PER_CHANNEL | oracle.DQ) == 1
+
+
+def test_cache_snapshot_and_restore_on_host_tensors(kvq):
+    """Checkpoint / resume of the binding's cache object: a snapshot holds
+    every buffer and the token count; restore refuses another shape."""
+    import torch
+    cfg = kvq.Config(128, 4, kvq.NSN | kvq.PER_CHANNEL | kvq.HADAMARD, None, device="cpu")
+    c = kvq.KVCache.allocate(cfg, 2, 2, 256, device="cpu")
+    g = torch.Generator().manual_seed(0)
+    for grp in (c.codes, c.tok, c.chan, c.off, c.resid):
+        for t in grp:
+            t.copy_(torch.randint(-100, 100, t.shape, generator=g).to(t.dtype))
+    c.c.len = 200
+    snap = c.snapshot()
+    d = kvq.KVCache.allocate(cfg, 2, 2, 256, device="cpu")
+    d.restore(snap)
+    assert d.len == 200
+    for name in ("codes", "tok", "chan", "off", "resid"):
+        for a, b in zip(getattr(c, name), getattr(d, name)):
+            assert torch.equal(a, b), name
+    small = kvq.KVCache.allocate(cfg, 2, 2, 128, device="cpu")
+    with pytest.raises(kvq.KvqError):
+        small.restore(snap)
