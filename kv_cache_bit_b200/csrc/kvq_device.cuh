@@ -163,48 +163,13 @@ struct RowLayout {
     static constexpr int kQmax = (1 << (BITS - 1)) - 1;
 };
 
-// Pack offset-binary codes e[c] (1 .. 2^BITS - 1) of one token row into
-// 32-bit words, little-endian byte order:
+// A packed token row holds the offset-binary codes e[c] (1 .. 2^BITS - 1)
+// in 32-bit words, little-endian byte order:
 //   INT4 byte j = e[2j] | e[2j+1] << 4
 //   INT2 byte j = e[4j] | e[4j+1] << 2 | e[4j+2] << 4 | e[4j+3] << 6
 //   INT3 plane of (e & 3) in the INT2 layout (D/4 bytes), then a plane whose
 //        bit i of byte j is bit 2 of e[8j+i] (D/8 bytes)
-template <int D, int BITS>
-__device__ __forceinline__ void pack_row(const uint32_t (&e)[D], uint32_t (&w)[RowLayout<D, BITS>::kWords]) {
-    if constexpr (BITS == 4) {
-#pragma unroll
-        for (int k = 0; k < D / 8; ++k) {
-            uint32_t v = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v |= (e[8 * k + i] & 15u) << (4 * i);
-            w[k] = v;
-        }
-    } else if constexpr (BITS == 2) {
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-            uint32_t v = 0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v |= (e[16 * k + i] & 3u) << (2 * i);
-            w[k] = v;
-        }
-    } else {
-        static_assert(BITS == 3, "bits");
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-            uint32_t v = 0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v |= (e[16 * k + i] & 3u) << (2 * i);
-            w[k] = v;
-        }
-#pragma unroll
-        for (int k = 0; k < D / 32; ++k) {
-            uint32_t v = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v |= ((e[32 * k + i] >> 2) & 1u) << i;
-            w[D / 16 + k] = v;
-        }
-    }
-}
+// (V rows of head dim 128 are further pair-interleaved, see pairv_layout).
 
 // Offset-binary code of channel c from a packed row held as 32-bit words.
 template <int D, int BITS>

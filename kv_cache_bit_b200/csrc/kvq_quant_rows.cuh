@@ -169,42 +169,6 @@ __device__ __forceinline__ uint32_t prmt32(uint32_t a, uint32_t b, uint32_t sel)
     return r;
 }
 
-// Codes from the words of r = fma(u, inv, 1.5 * 2^23 + 2^(BITS-1)): for any
-// |rne(u * inv)| <= qmax the float lies in [2^23, 2^24), where its ulp is 1,
-// so the single rounding of the fused product is round-half-even of u * inv
-// (the added constant is even) and the low mantissa bits hold the
-// offset-binary code e.  cw[c] holds that word for channel c; the bits above
-// the code (bit 22 upward) never reach the low 16 bits of the sums below.
-template <int D, int BITS>
-__device__ __forceinline__ void pack_codes(const uint32_t (&cw)[D], uint32_t (&w)[RowLayout<D, BITS>::kWords]) {
-    if constexpr (BITS == 4) {
-#pragma unroll
-        for (int k = 0; k < D / 8; ++k) {
-            const uint32_t* e = cw + 8 * k;
-            const uint32_t h0 = e[0] + 16u * e[1] + 256u * e[2] + 4096u * e[3];
-            const uint32_t h1 = e[4] + 16u * e[5] + 256u * e[6] + 4096u * e[7];
-            w[k] = prmt32(h0, h1, 0x5410u);
-        }
-    } else if constexpr (BITS == 2) {
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-            const uint32_t* e = cw + 16 * k;
-            uint32_t h0 = 0, h1 = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                h0 += e[i] << (2 * i);
-                h1 += e[8 + i] << (2 * i);
-            }
-            w[k] = prmt32(h0, h1, 0x5410u);
-        }
-    } else {
-        uint32_t e[D];
-#pragma unroll
-        for (int c = 0; c < D; ++c) e[c] = cw[c] & 7u;
-        pack_row<D, BITS>(e, w);
-    }
-}
-
 // ---------------------------------------------------------------- the quantizer
 
 // NSN block means: from the fp16 tile with the row still in its fp16 form
@@ -371,8 +335,13 @@ __device__ __forceinline__ float warp_max_abs(float x) {
     return r;
 }
 
-// Offset-binary code words of one pair: lanes of fma(x, inv, kC) (see
-// pack_codes), clamped to [-qmax, qmax] when CLAMP.
+// Offset-binary code words of one pair: lanes of r = fma(x, inv, kC) with
+// kC = 1.5 * 2^23 + 2^(BITS-1).  For any |rne(x * inv)| <= qmax the float
+// lies in [2^23, 2^24), where its ulp is 1, so the single rounding of the
+// fused product is round-half-even of x * inv (the added constant is even)
+// and the low mantissa bits hold the offset-binary code e; the bits above
+// the code (bit 22 upward) never reach the low 16 bits of the packing sums.
+// Clamped to [-qmax, qmax] when CLAMP.
 template <bool CLAMP>
 __device__ __forceinline__ void code_pair(f2_t x, f2_t inv, float kQ, float kC, uint32_t& clo, uint32_t& chi) {
     float lo, hi;
@@ -386,7 +355,7 @@ __device__ __forceinline__ void code_pair(f2_t x, f2_t inv, float kQ, float kC, 
 }
 
 // Low 16 bits of sum_i e[i] << (NB * i) for N codes of NB bits (the bits of
-// each word above bit 21 stay out of the low half, see pack_codes).
+// each word above bit 21 stay out of the low half, see code_pair).
 template <int N, int NB>
 __device__ __forceinline__ uint32_t pack_half(const uint32_t* e) {
     uint32_t h = e[0];
@@ -396,14 +365,15 @@ __device__ __forceinline__ uint32_t pack_half(const uint32_t* e) {
 }
 
 // Codes of the row held in registers (reciprocal scales in pair order in
-// vec), packed as they are produced: a group of GP pairs gives GP codes of
-// the low half (channels j ..) and GP of the high half (channels j + D/2 ..),
+// vec, or, when UNIFORM, one reciprocal scale inv for the whole row),
+// packed as they are produced: a group of GP pairs gives GP codes of the
+// low half (channels j ..) and GP of the high half (channels j + D/2 ..),
 // folded at once into half-words (INT4 / INT2, and the 2-bit plane of INT3)
 // or bytes (the bit plane of INT3), so that few code words are live while
 // most of the row still is.
-template <int D, int BITS, bool CLAMP>
+template <int D, int BITS, bool CLAMP, bool UNIFORM = false>
 __device__ __forceinline__ void codes_from_regs(const f2_t (&P)[D / 2], const float* vec,
-                                                uint32_t (&w)[RowLayout<D, BITS>::kWords]) {
+                                                uint32_t (&w)[RowLayout<D, BITS>::kWords], float inv = 0.0f) {
     using L = RowLayout<D, BITS>;
     constexpr int H2 = D / 2;
     constexpr float kQ = (float)L::kQmax;
@@ -416,7 +386,9 @@ __device__ __forceinline__ void codes_from_regs(const f2_t (&P)[D / 2], const fl
         uint32_t lo[GP], hi[GP];
 #pragma unroll
         for (int i = 0; i < GP; i += 2) {
-            const ulonglong2 r = *reinterpret_cast<const ulonglong2*>(iv + q * GP + i);
+            ulonglong2 r;
+            if constexpr (UNIFORM) r = make_ulonglong2(f2_pack(inv, inv), f2_pack(inv, inv));
+            else r = *reinterpret_cast<const ulonglong2*>(iv + q * GP + i);
             code_pair<CLAMP>(P[q * GP + i], r.x, kQ, kC, lo[i], hi[i]);
             code_pair<CLAMP>(P[q * GP + i + 1], r.y, kQ, kC, lo[i + 1], hi[i + 1]);
         }
@@ -731,30 +703,27 @@ __device__ __forceinline__ void quantize_rows(uint4 (&raw)[D / 8], const int t, 
     constexpr float kC = 12582912.0f + (float)L::kOff;  // 1.5 * 2^23 + offset
     if constexpr (MODE == kNaive) {
         __syncthreads();  // every row has been read from the tile the codes are staged over
-        uint32_t cw[D];
-        float m = 0.0f;
+        // max |x| over the row (exact in any order): eight independent chains
+        float mp[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int j = 0; j < H2; ++j) {
             float lo, hi;
             f2_unpack(P[j], lo, hi);
-            m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
+            mp[j & 7] = fmaxf(mp[j & 7], fmaxf(fabsf(lo), fabsf(hi)));
         }
+        const float m = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                              fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
         const __half s16 = __float2half_rn(__fdiv_rn(m, kQ));
         out.tok[t] = s16;
         const float sf = __half2float(s16);
         const float inv = sf > 0.0f ? __fdiv_rn(1.0f, sf) : 0.0f;
-        const f2_t I2 = f2_pack(inv, inv), C2 = f2_pack(kC, kC);
-#pragma unroll
-        for (int j = 0; j < H2; ++j) {
-            float lo, hi;
-            f2_unpack(f2_fma(P[j], I2, C2), lo, hi);
-            lo = fminf(fmaxf(lo, kC - kQ), kC + kQ);
-            hi = fminf(fmaxf(hi, kC - kQ), kC + kQ);
-            cw[j] = __float_as_uint(lo);
-            cw[j + H2] = __float_as_uint(hi);
-        }
+        // some |x * inv| of this row rounds past qmax (an fp16 subnormal
+        // scale): the exact sign of m * inv - (qmax + 1/2); the warp takes
+        // the clamped packer only when one of its rows needs it
+        const bool clamp = __fmaf_rn(m, inv, -(kQ + 0.5f)) >= 0.0f;
         uint32_t w[L::kWords];
-        pack_codes<D, BITS>(cw, w);
+        if (__any_sync(0xffffffffu, clamp)) codes_from_regs<D, BITS, true, true>(P, nullptr, w, inv);
+        else codes_from_regs<D, BITS, false, true>(P, nullptr, w, inv);
         store_codes<D, BITS>(out, t, w);
     } else {
         // per-channel absmax over the block: one redux per channel and warp
