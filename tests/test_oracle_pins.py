@@ -231,6 +231,47 @@ def test_naive_closed_form():
     _check_codes(x, f16val(c["tok"][..., 0])[..., None], q, 7)
 
 
+@pytest.mark.parametrize("bits", [4, 3])
+def test_nsep_only_ablation_closed_form(bits):
+    """[P1] the norm-separation ablation (the post's "nsep only" row): FP16
+    norm, then a per-token absmax scale of the unit direction (the snippet's
+    amax over the channels), no per-channel scale.  Token parameters: the
+    norm, then the scale."""
+    K, _ = _data(41 + bits)
+    x = K.astype(np.float64)
+    cfg = oracle.Cfg(d=128, bits=bits, flags=oracle.NORM_SEP)
+    c = oracle.quantize(cfg, f16bits(K))
+    assert c["chan"] is None and c["tok"].shape[-1] == 2
+    qm = oracle.qmax(bits)
+    n64 = np.linalg.norm(x, axis=-1)
+    assert np.all(near_f16(c["tok"][..., 0], n64))
+    u = x / n64[..., None]
+    assert np.all(near_f16(c["tok"][..., 1], np.abs(u).max(axis=-1) / qm))
+    q, bad = _unpack_cache(c, 128, bits)
+    assert bad == 0
+    _check_codes(u, f16val(c["tok"][..., 1])[..., None], q, qm)
+    # the largest |u| of every token codes to +-qmax
+    hit = np.take_along_axis(np.abs(q), np.abs(u).argmax(axis=-1)[..., None], axis=-1)
+    assert np.all(hit == qm)
+
+
+def test_pchan_only_ablation_closed_form():
+    """[P1]/[P2] the per-channel ablation (the post's "pchan only" row): the
+    raw x scaled per channel by its absmax over each 128-token block, no
+    norm."""
+    K, _ = _data(47)
+    x = K.astype(np.float64)
+    cfg = oracle.Cfg(d=128, bits=4, flags=oracle.PER_CHANNEL)
+    c = oracle.quantize(cfg, f16bits(K))
+    B, H, S, d = x.shape
+    xb = x.reshape(B, H, S // T, T, d)
+    assert np.all(near_f16(c["chan"], np.abs(xb).max(axis=3) / 7))
+    assert c["tok"] is None                     # no token parameter
+    q, bad = _unpack_cache(c, d, 4)
+    assert bad == 0
+    _check_codes(xb, f16val(c["chan"])[:, :, :, None, :], q.reshape(xb.shape), 7)
+
+
 def test_rht_closed_form():
     d = 128
     K, _ = _data(31)
