@@ -1058,7 +1058,7 @@ __global__ void __launch_bounds__(128) decode_combine_mma_kernel(DecodeArgs a) {
     static_assert(D == 128, "one channel per thread");
     constexpr float kLog2e = 1.4426950408889634f;
     constexpr int PS = part_stride<D>();
-    constexpr int KB = 32 / GP;  // candidates per batch of accumulator loads
+    constexpr int KB = 64 / GP;  // candidates per batch of accumulator loads (64 floats a thread)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int pair = blockIdx.x;
     const int G = a.G;  // <= GP
