@@ -216,6 +216,10 @@ size_t kvq_decode_workspace_bytes(const kvq_config* cfg, const kvq_cache* cache,
  *   ws    workspace of at least kvq_decode_workspace_bytes() (contents
  *         need no initialization); calls that share a workspace must not
  *         overlap in time
+ * Stream order: at head dim 128 the call's kernels are launched as
+ * programmatic dependents (their launch overlaps the tail of the kernel
+ * ahead of them in the stream; they wait for it to finish before reading
+ * or writing any memory), so ordinary stream order holds for the caller.
  * Errors: INVALID_ARG; WORKSPACE; UNSUPPORTED; CUDA.
  */
 kvq_status kvq_decode_attention(const kvq_config* cfg, const kvq_cache* cache,
